@@ -1,0 +1,237 @@
+"""Plain, slow, fp64 reference of the LISA attention layer.
+
+TEST INFRASTRUCTURE ONLY: the CUDA library never imports or calls this module,
+and this module imports nothing from the CUDA side.  Every function works on
+float64 NumPy arrays and follows one step of the method in the order the pages
+give it.
+
+Sources (web pages about arXiv 2607.19358, "LISA: Linear-Indexed Sparse
+Attention for Efficient Long-Context Reasoning"):
+  [abs]  the English abstract (arxivdaily.com page; same text on fugumt.com):
+         a Lightning Indexer keeps the top-M tokens of the full context for a
+         sparse self-attention; a linear-attention branch runs in parallel;
+         a gate fuses the two; n generated tokens cost O(nM).
+  [meth] gptget.net digest, section "方法详解" (method details): linear
+         attention with phi = identity and a state matrix S_t updated in O(1)
+         per step; indexer = query/key projections and a ReLU dot product;
+         a learned gate g mixes the two branch outputs.
+  [exp]  gptget.net digest, section "实验设计" (experiment design): M = 256.
+
+The pages leave these points open; this library fixes them as definitions
+(the same in the oracle and on the GPU):
+  * indexer score of key s for KV head g: sum over the R = HI/Hkv indexer heads
+    j = g*R + r of w[j] * max(0, qidx[j] . kidx[g, s]); no extra scale;
+  * one top-M set per KV head, shared by its G = Hq/Hkv query heads
+    (query head h belongs to KV head h // G);
+  * order: higher score first, equal scores -> lower position first;
+    a prefix with <= M tokens is selected whole; the current token is a
+    candidate (causal prefix s <= t);
+  * softmax scale 1/sqrt(d);
+  * linear branch: S_h <- S_h + k_t^T v_t, then o_lin = q_t S_h (the update
+    includes the current token), no normaliser, no decay; k and v are the
+    attention's own k/v of KV head h // G, S is kept per query head;
+  * gate: g = sigmoid(lambda_h), o = g * o_sparse + (1 - g) * o_lin.
+
+Parity status of each function is stated in its docstring; every function here
+is pinned by tests in tests/test_oracle.py.
+"""
+
+import numpy as np
+
+
+# --------------------------------------------------------------------------
+# step 1: Lightning Indexer score      [abs], [meth]
+# --------------------------------------------------------------------------
+def indexer_scores(qidx_t: np.ndarray, w_t: np.ndarray, kidx_keys: np.ndarray) -> np.ndarray:
+    """Scores of every candidate key for one query token.
+
+    qidx_t    [HI, dI]      indexer queries of the token
+    w_t       [HI]          indexer head weights of the token
+    kidx_keys [Hkv, n, dI]  indexer keys of the candidate positions 0..n-1
+    returns   [Hkv, n]      I_g(s) = sum_r w[gR+r] * max(0, qidx[gR+r] . kidx[g, s])
+    """
+    HI = qidx_t.shape[0]
+    Hkv, n, _ = kidx_keys.shape
+    R = HI // Hkv
+    out = np.zeros((Hkv, n), dtype=np.float64)
+    for g in range(Hkv):
+        for r in range(R):
+            j = g * R + r
+            dots = kidx_keys[g] @ qidx_t[j]
+            out[g] += w_t[j] * np.maximum(dots, 0.0)
+    return out
+
+
+# --------------------------------------------------------------------------
+# step 2: top-M selection              [abs], [exp]
+# --------------------------------------------------------------------------
+def _order(scores: np.ndarray) -> np.ndarray:
+    """Positions sorted by (score descending, position ascending)."""
+    n = scores.shape[0]
+    # np.lexsort sorts by the last key first: primary -score, secondary position.
+    return np.lexsort((np.arange(n), -scores))
+
+
+def topm_select(scores: np.ndarray, M: int) -> np.ndarray:
+    """The first min(M, n) positions of the order, listed in ascending position,
+    padded with -1 up to M entries."""
+    n = scores.shape[0]
+    keep = np.sort(_order(scores)[: min(M, n)])
+    out = np.full(M, -1, dtype=np.int64)
+    out[: keep.shape[0]] = keep
+    return out
+
+
+def topm_threshold(scores: np.ndarray, M: int) -> float:
+    """Score of the M-th entry of the order (the lowest selected score)."""
+    n = scores.shape[0]
+    return float(scores[_order(scores)[min(M, n) - 1]])
+
+
+def borderline_mask(scores: np.ndarray, M: int, rel: float = 1e-4, floor: float = 1e-3) -> np.ndarray:
+    """Tokens whose selection may legitimately differ between the fp64 oracle
+    and an fp32 device: |I(s) - s_M| <= rel * max(|s_M|, floor * max_s I(s)).
+    Empty when n <= M (everything is selected)."""
+    n = scores.shape[0]
+    if n <= M:
+        return np.zeros(n, dtype=bool)
+    sM = topm_threshold(scores, M)
+    tol = rel * max(abs(sM), floor * float(np.max(np.abs(scores))))
+    return np.abs(scores - sM) <= tol
+
+
+# --------------------------------------------------------------------------
+# step 3: sparse softmax attention over the selected rows     [abs]
+# --------------------------------------------------------------------------
+def sparse_attention(q_h: np.ndarray, K_sel: np.ndarray, V_sel: np.ndarray) -> np.ndarray:
+    """softmax_s(q . k_s / sqrt(d)) weighted sum of v_s over the given rows.
+
+    q_h [d]; K_sel, V_sel [m, d] with m >= 1."""
+    d = q_h.shape[0]
+    logits = (K_sel @ q_h) / np.sqrt(d)
+    p = np.exp(logits - np.max(logits))
+    p = p / np.sum(p)
+    return p @ V_sel
+
+
+# --------------------------------------------------------------------------
+# step 4: linear attention, phi = identity     [meth]
+# --------------------------------------------------------------------------
+def linear_update(S_h: np.ndarray, k_t: np.ndarray, v_t: np.ndarray) -> np.ndarray:
+    """S <- S + k^T v  (S[i, j] += k[i] * v[j]); returns the new state."""
+    return S_h + np.outer(k_t, v_t)
+
+
+def linear_readout(q_h: np.ndarray, S_h: np.ndarray) -> np.ndarray:
+    """o_lin[j] = sum_i q[i] * S[i, j]."""
+    return q_h @ S_h
+
+
+# --------------------------------------------------------------------------
+# step 5: gate                                   [abs], [meth]
+# --------------------------------------------------------------------------
+def gate_fuse(lam: float, o_sp: np.ndarray, o_lin: np.ndarray) -> np.ndarray:
+    """g = 1 / (1 + exp(-lam)); o = g * o_sp + (1 - g) * o_lin."""
+    with np.errstate(over="ignore"):
+        g = 1.0 / (1.0 + np.exp(-float(lam)))
+    return g * o_sp + (1.0 - g) * o_lin
+
+
+# --------------------------------------------------------------------------
+# whole layer: one decode step
+# --------------------------------------------------------------------------
+def decode_step(q, k, v, qidx, kidx, w, lam, k_cache, v_cache, kidx_cache, S, pos, M,
+                sel_override=None):
+    """One decode step for a batch.
+
+    q [B,Hq,d]; k, v [B,Hkv,d]; qidx [B,HI,dI]; kidx [B,Hkv,dI]; w [B,HI];
+    lam [B,Hq]; caches [B,Hkv,>=pos[b],*] hold rows 0..pos[b]-1; S [B,Hq,d,d];
+    pos [B] = position t of the new token.
+    sel_override: optional [B,Hkv,M] index sets to use for the sparse branch
+    instead of the oracle's own (the "conditional oracle").
+
+    Returns dict: out [B,Hq,d], idx [B,Hkv,M], S [B,Hq,d,d],
+    scores list (per b) of [Hkv, t+1] arrays, o_sp, o_lin [B,Hq,d].
+    """
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d))
+    o_sp_all = np.zeros((B, Hq, d))
+    o_lin_all = np.zeros((B, Hq, d))
+    idx = np.full((B, Hkv, M), -1, dtype=np.int64)
+    S_new = np.array(S, dtype=np.float64, copy=True)
+    scores_all = []
+    for b in range(B):
+        t = int(pos[b])
+        # candidate keys 0..t: cached rows then the new token
+        K = np.concatenate([k_cache[b, :, :t, :], k[b][:, None, :]], axis=1)          # [Hkv, t+1, d]
+        V = np.concatenate([v_cache[b, :, :t, :], v[b][:, None, :]], axis=1)
+        KI = np.concatenate([kidx_cache[b, :, :t, :], kidx[b][:, None, :]], axis=1)   # [Hkv, t+1, dI]
+        sc = indexer_scores(qidx[b], w[b], KI)
+        scores_all.append(sc)
+        for g in range(Hkv):
+            idx[b, g] = topm_select(sc[g], M)
+        use = idx[b] if sel_override is None else np.asarray(sel_override[b])
+        for h in range(Hq):
+            g = h // G
+            sel = use[g][use[g] >= 0]
+            o_sp = sparse_attention(q[b, h], K[g, sel], V[g, sel])
+            S_new[b, h] = linear_update(S_new[b, h], k[b, g], v[b, g])
+            o_lin = linear_readout(q[b, h], S_new[b, h])
+            o_sp_all[b, h] = o_sp
+            o_lin_all[b, h] = o_lin
+            out[b, h] = gate_fuse(lam[b, h], o_sp, o_lin)
+    return dict(out=out, idx=idx, S=S_new, scores=scores_all, o_sp=o_sp_all, o_lin=o_lin_all)
+
+
+# --------------------------------------------------------------------------
+# whole layer: causal prefill of T tokens
+# --------------------------------------------------------------------------
+def prefill(q, k, v, qidx, kidx, w, lam, S0, M, rows=None, sel_override=None):
+    """Causal prefill of T tokens starting from an empty cache.
+
+    q [B,T,Hq,d]; k, v [B,T,Hkv,d]; qidx [B,T,HI,dI]; kidx [B,T,Hkv,dI];
+    w [B,T,HI]; lam [B,T,Hq]; S0 [B,Hq,d,d].
+    rows: optional iterable of token indices t whose outputs are wanted (the
+    state always runs over all T tokens); default all.
+    sel_override: optional callable (b, t) -> [Hkv, M] index sets for the
+    sparse branch (the "conditional oracle"), or None.
+
+    Returns dict: out [B,T,Hq,d] (rows not requested stay 0), idx [B,T,Hkv,M]
+    (-1 for rows not requested), S [B,Hq,d,d] = state after token T-1,
+    scores {(b, t): [Hkv, t+1]} for the requested rows.
+    """
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    want = np.zeros(T, dtype=bool)
+    if rows is None:
+        want[:] = True
+    else:
+        want[np.asarray(list(rows), dtype=np.int64)] = True
+    out = np.zeros((B, T, Hq, d))
+    idx = np.full((B, T, Hkv, M), -1, dtype=np.int64)
+    S = np.array(S0, dtype=np.float64, copy=True)
+    scores = {}
+    for b in range(B):
+        Kb = np.transpose(k[b], (1, 0, 2))        # [Hkv, T, d]
+        Vb = np.transpose(v[b], (1, 0, 2))
+        KIb = np.transpose(kidx[b], (1, 0, 2))    # [Hkv, T, dI]
+        for t in range(T):
+            for h in range(Hq):
+                S[b, h] = linear_update(S[b, h], k[b, t, h // G], v[b, t, h // G])
+            if not want[t]:
+                continue
+            sc = indexer_scores(qidx[b, t], w[b, t], KIb[:, : t + 1, :])
+            scores[(b, t)] = sc
+            for g in range(Hkv):
+                idx[b, t, g] = topm_select(sc[g], M)
+            use = idx[b, t] if sel_override is None else np.asarray(sel_override(b, t))
+            for h in range(Hq):
+                g = h // G
+                sel = use[g][use[g] >= 0]
+                o_sp = sparse_attention(q[b, t, h], Kb[g, sel], Vb[g, sel])
+                o_lin = linear_readout(q[b, t, h], S[b, h])
+                out[b, t, h] = gate_fuse(lam[b, t, h], o_sp, o_lin)
+    return dict(out=out, idx=idx, S=S, scores=scores)
