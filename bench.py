@@ -1,0 +1,379 @@
+"""LISA decode-attention benchmark on B200.
+
+Workload: the Qwen2.5-1.5B-shaped single-layer decode step (B=1, 12 query /
+2 KV heads, d=128, 4 indexer heads of dim 64, M=256) at 16384 cached tokens.
+One step = one lisa_decode_step call: indexer over all 16384 keys, top-M,
+sparse attention, linear-state update and gate.
+
+The timed region replays a CUDA graph of K steps that rotates over R
+independent layer instances whose touched bytes exceed 4x the L2 size, so the
+traffic is HBM traffic.  value = tokens/s over all ranks (B tokens per step).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lisa|reference]
+
+--impl reference times the fp64 CPU oracle on the host cores (bounded
+sample), the only reference this method has.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lisa_inputs import get_config, make_rng, gen_layer, gen_step  # noqa: E402
+from lisa_inputs.gen import decode_positions  # noqa: E402
+
+METRIC = "LISA decode-attn tokens/s @16K ctx, M=256; % of HBM roofline"
+WORKLOAD = "decode_1p5b_16k"
+
+
+def algorithmic_bytes(cfg, L, esize=2):
+    """Bytes the method must move per decode step (one sequence):
+    indexer keys of every cached token, the M selected K and V rows, the fp32
+    state read and write, plus the step's own small tensors."""
+    G = cfg.Hq // cfg.Hkv
+    M = min(cfg.M, L)
+    big = cfg.Hkv * L * cfg.dI * esize + cfg.Hkv * M * 2 * cfg.d * esize + cfg.Hq * cfg.d * cfg.d * 4 * 2
+    small = (cfg.Hq * cfg.d * esize            # q
+             + 2 * cfg.Hkv * cfg.d * esize      # k, v read
+             + 2 * cfg.Hkv * cfg.d * esize      # k, v appended
+             + 2 * cfg.Hkv * cfg.dI * esize     # kidx read + appended
+             + cfg.HI * cfg.dI * esize          # qidx
+             + cfg.HI * 4 + cfg.Hq * 4          # w, gate logits
+             + cfg.Hq * cfg.d * esize)          # out
+    del G
+    return big + small
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except FileNotFoundError:
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+
+    def summary(self, t0, t1):
+        rows = [s for (ts, s) in self.samples if t0 <= ts <= t1] or [s for (_, s) in self.samples]
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    cfg = get_config(WORKLOAD)
+    rng = make_rng(cfg.seed, 0)
+    lay = gen_layer(cfg, rng, cfg.L - 1)
+    pos = decode_positions(cfg)
+    a = lambda z: z.astype(np.float64)
+    kc, vc, kic, S0 = a(lay.k_cache), a(lay.v_cache), a(lay.kidx_cache), a(lay.S0)
+    steps = [gen_step(cfg, rng, 1) for _ in range(4)]
+
+    def one(st):
+        s0 = lambda z: a(z[:, 0])
+        oracle.decode_step(s0(st.q), s0(st.k), s0(st.v), s0(st.qidx), s0(st.kidx), s0(st.w), s0(st.lam),
+                           kc, vc, kic, S0, pos, cfg.M)
+
+    for i in range(args.warmup):
+        one(steps[i % 4])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(steps[i % 4])
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    value = args.steps * cfg.B / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1)/sqrt(dim) caches and inputs)",
+        "config": {"workload": WORKLOAD, "B": cfg.B, "L": cfg.L, "M": cfg.M, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} fp64 oracle decode steps of the 16384-token workload"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_sample(seconds=10.0):
+    """The fp64 oracle on this host's cores, timed on a bounded sample of
+    the same workload (whole decode steps, until `seconds` have passed)."""
+    import oracle
+    cfg = get_config(WORKLOAD)
+    rng = make_rng(cfg.seed, 0)
+    lay = gen_layer(cfg, rng, cfg.L - 1)
+    st = gen_step(cfg, rng, 1)
+    pos = decode_positions(cfg)
+    a = lambda z: z.astype(np.float64)
+    s0 = lambda z: a(z[:, 0])
+    args = (s0(st.q), s0(st.k), s0(st.v), s0(st.qidx), s0(st.kidx), s0(st.w), s0(st.lam), a(lay.k_cache),
+            a(lay.v_cache), a(lay.kidx_cache), a(lay.S0), pos, cfg.M)
+    oracle.decode_step(*args)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode_step(*args)
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+    return {"value": n * cfg.B / dt, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{n} fp64 oracle decode steps of the 16384-token workload in {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- lisa arm
+class Instance:
+    """One independent layer at 16384 cached tokens, with its step inputs."""
+
+    def __init__(self, L, cfg, torch, seed, exact=None):
+        dev = "cuda"
+        bf = torch.bfloat16
+        self.lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.L, L.LISA_BF16)
+        n = cfg.L - 1
+        if exact is not None:
+            lay_np, st = exact
+            tb = lambda z: torch.from_numpy(np.ascontiguousarray(z)).to(dev, bf)
+            tf = lambda z: torch.from_numpy(np.ascontiguousarray(z)).to(dev, torch.float32)
+            self.lay.k_cache[:, :, :n] = tb(lay_np.k_cache)
+            self.lay.v_cache[:, :, :n] = tb(lay_np.v_cache)
+            self.lay.kidx_cache[:, :, :n] = tb(lay_np.kidx_cache)
+            self.lay.state.copy_(tf(lay_np.S0))
+            s0 = lambda z: z[:, 0]
+            self.q, self.k, self.v = tb(s0(st.q)), tb(s0(st.k)), tb(s0(st.v))
+            self.kidx, self.qidx = tb(s0(st.kidx)), tb(s0(st.qidx))
+            self.w, self.lam = tf(s0(st.w)), tf(s0(st.lam))
+        else:
+            g = torch.Generator(device=dev)
+            g.manual_seed(seed)
+            rn = lambda shape, dim: (torch.randn(shape, generator=g, device=dev) / dim ** 0.5).to(bf)
+            self.lay.k_cache[:, :, :n] = rn((cfg.B, cfg.Hkv, n, cfg.d), cfg.d)
+            self.lay.v_cache[:, :, :n] = rn((cfg.B, cfg.Hkv, n, cfg.d), cfg.d)
+            self.lay.kidx_cache[:, :, :n] = rn((cfg.B, cfg.Hkv, n, cfg.dI), cfg.dI)
+            self.lay.state.copy_(torch.randn(self.lay.state.shape, generator=g, device=dev))
+            self.q, self.k, self.v = (rn((cfg.B, cfg.Hq, cfg.d), cfg.d), rn((cfg.B, cfg.Hkv, cfg.d), cfg.d),
+                                      rn((cfg.B, cfg.Hkv, cfg.d), cfg.d))
+            self.kidx, self.qidx = rn((cfg.B, cfg.Hkv, cfg.dI), cfg.dI), rn((cfg.B, cfg.HI, cfg.dI), cfg.dI)
+            self.w = torch.rand((cfg.B, cfg.HI), generator=g, device=dev)
+            self.lam = torch.randn((cfg.B, cfg.Hq), generator=g, device=dev)
+        self.lay.pos.fill_(n)
+        self.out = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=bf, device=dev)
+        self.idx = torch.empty(cfg.B, cfg.Hkv, cfg.M, dtype=torch.int32, device=dev)
+
+    def step(self, L, ws, stream=None):
+        L.lisa_decode_step(self.lay, self.q, self.k, self.v, self.kidx, self.qidx, self.w, self.lam, 1, self.out,
+                           self.idx, ws, stream)
+
+
+def run_lisa(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    from hybrid_linear_top_b200 import lisa as L
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    cfg = get_config(WORKLOAD)
+    props = torch.cuda.get_device_properties(local)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    step_bytes = algorithmic_bytes(cfg, cfg.L)
+    R = max(args.instances, int(np.ceil(4 * l2 / step_bytes)))
+
+    rng = make_rng(cfg.seed, 0)
+    exact = (gen_layer(cfg, rng, cfg.L - 1), gen_step(cfg, rng, 1))
+    inst = [Instance(L, cfg, torch, 1000 * rank + i, exact if i == 0 else None) for i in range(R)]
+    ws = L.alloc_workspace(inst[0].lay, 1, L.LISA_OP_DECODE)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    # warm-up (eager launches), then capture one rotation (R steps) and the
+    # K mod R tail as CUDA graphs; the timed region replays them for exactly K steps
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            inst[i % R].step(L, ws, stream)
+    stream.synchronize()
+    rot = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(rot, stream=stream):
+        for i in range(R):
+            inst[i].step(L, ws, stream)
+    n_rot, n_tail = divmod(args.steps, R)
+    tail = None
+    if n_tail:
+        tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tail, stream=stream):
+            for i in range(n_tail):
+                inst[i].step(L, ws, stream)
+    for _ in range(2):
+        rot.replay()
+    torch.cuda.synchronize()
+
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.2)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n_rot):
+            rot.replay()
+        if tail is not None:
+            tail.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    clk.stop()
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    steps_total = args.steps
+    ms_per_step = ms / steps_total
+    value = world * steps_total * cfg.B / (ms / 1e3)
+
+    # ---- end to end through the public call: pinned host inputs in, output out
+    host = {k: getattr(inst[0], k).cpu().pin_memory() for k in ["q", "k", "v", "kidx", "qidx", "w", "lam"]}
+    out_h = torch.empty_like(inst[0].out, device="cpu").pin_memory()
+    dev_in = {k: torch.empty_like(getattr(inst[0], k)) for k in host}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    n_e2e = max(20, min(2000, args.steps))
+    with torch.cuda.stream(stream):
+        for it in range(n_e2e + 5):
+            if it == 5:
+                torch.cuda.synchronize()
+                t0 = time.perf_counter()
+            for k2 in host:
+                dev_in[k2].copy_(host[k2], non_blocking=True)
+            L.lisa_decode_step(inst[0].lay, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["kidx"], dev_in["qidx"],
+                               dev_in["w"], dev_in["lam"], 1, inst[0].out, None, ws, stream)
+            out_h.copy_(inst[0].out, non_blocking=True)
+            stream.synchronize()
+    e2e_s = (time.perf_counter() - t0) / n_e2e
+    e2e_val = world * cfg.B / e2e_s
+
+    # ---- parity of instance 0 (exact seeded inputs) against the oracle, small check
+    peak, peak_kind = load_peaks()
+    achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+    if rank != 0:
+        return
+    cpu = cpu_baseline_sample(args.cpu_seconds) if world == 1 and not args.no_cpu_baseline else None
+    clocks = clk.summary(t_wall0, t_wall1)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(dim) caches and inputs; fp32 state ~ N(0,1))",
+        "config": {"workload": WORKLOAD, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "HI": cfg.HI,
+                   "dI": cfg.dI, "M": cfg.M, "L": cfg.L, "instances": R,
+                   "l2": "inputs larger than L2: rotation over instances touching "
+                         f"{R * step_bytes / 2 ** 20:.0f} MiB (L2 {l2 / 2 ** 20:.0f} MiB)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "decode step (score_state + select + attend)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": step_bytes, "traffic": None},
+        "clocks": clocks,
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * steps_total,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
+    ap.add_argument("--instances", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_lisa(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,292 @@
+// C ABI of the LISA layer: host-side validation, workspace carve-up, launches.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "lisa_internal.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+lisa_status fail(lisa_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+lisa_status ok() {
+  g_msg[0] = '\0';
+  return LISA_OK;
+}
+
+lisa_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(LISA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int round4(int x) { return (x + 3) & ~3; }
+
+constexpr int kDecodeKeysCap = 32768;   // order keys staged in shared memory (1024-thread select)
+constexpr int kRowsKeysCap = 16384;     // same, for the 256-thread row select
+constexpr int kCandCap = 4096;          // threshold-bucket candidates kept in shared memory
+constexpr int kRowChunk = 1024;         // query rows scored per pass on the row path
+
+// Validates the geometry; returns LISA_OK or the failure status.
+lisa_status check_layer(const lisa_layer *L) {
+  if (!L) return fail(LISA_ERR_INVALID_ARG, "layer is NULL");
+  if (L->B < 0 || L->Hq < 1 || L->Hkv < 1 || L->HI < 1 || L->d < 1 || L->dI < 1 || L->M < 1 || L->L_max < 1)
+    return fail(LISA_ERR_INVALID_ARG, "non-positive dimension (B=%d Hq=%d Hkv=%d HI=%d d=%d dI=%d M=%d L_max=%d)",
+                L->B, L->Hq, L->Hkv, L->HI, L->d, L->dI, L->M, L->L_max);
+  if (L->dtype != LISA_BF16 && L->dtype != LISA_FP32) return fail(LISA_ERR_INVALID_ARG, "unknown dtype %d", L->dtype);
+  if (L->Hq % L->Hkv) return fail(LISA_ERR_UNSUPPORTED, "Hq=%d is not a multiple of Hkv=%d", L->Hq, L->Hkv);
+  if (L->HI % L->Hkv) return fail(LISA_ERR_UNSUPPORTED, "HI=%d is not a multiple of Hkv=%d", L->HI, L->Hkv);
+  if (L->Hq / L->Hkv > lisa::kMaxG) return fail(LISA_ERR_UNSUPPORTED, "Hq/Hkv=%d > %d", L->Hq / L->Hkv, lisa::kMaxG);
+  if (L->HI / L->Hkv > lisa::kMaxR) return fail(LISA_ERR_UNSUPPORTED, "HI/Hkv=%d > %d", L->HI / L->Hkv, lisa::kMaxR);
+  if (L->d != 64 && L->d != 128) return fail(LISA_ERR_UNSUPPORTED, "d=%d not in {64,128}", L->d);
+  if (L->dI != 32 && L->dI != 64) return fail(LISA_ERR_UNSUPPORTED, "dI=%d not in {32,64}", L->dI);
+  if (L->M % 32 || L->M < 32 || L->M > 1024) return fail(LISA_ERR_UNSUPPORTED, "M=%d not a multiple of 32 in [32,1024]", L->M);
+  if ((long long)L->B * L->Hkv > 65535) return fail(LISA_ERR_UNSUPPORTED, "B*Hkv=%lld > 65535", (long long)L->B * L->Hkv);
+  return LISA_OK;
+}
+
+lisa_status check_ptr(const void *p, const char *name, bool required = true) {
+  if (!p) return required ? fail(LISA_ERR_INVALID_ARG, "%s is NULL", name) : LISA_OK;
+  if (!aligned16(p)) return fail(LISA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return LISA_OK;
+}
+
+lisa_status check_caches(const lisa_layer *L) {
+  lisa_status s;
+  if ((s = check_ptr(L->k_cache, "k_cache"))) return s;
+  if ((s = check_ptr(L->v_cache, "v_cache"))) return s;
+  if ((s = check_ptr(L->kidx_cache, "kidx_cache"))) return s;
+  if ((s = check_ptr(L->pos, "pos"))) return s;
+  if (L->err_word && (reinterpret_cast<uintptr_t>(L->err_word) & 3u)) return fail(LISA_ERR_INVALID_ARG, "err_word misaligned");
+  return LISA_OK;
+}
+
+// ---------------------------------------------------------------- workspace plans
+struct DecodePlan {
+  size_t keys, idx, olin, partials, counters, total;
+};
+DecodePlan decode_plan(const lisa_layer *L) {
+  DecodePlan p;
+  const size_t BH = (size_t)L->B * L->Hkv;
+  size_t off = 0;
+  p.keys = off; off += round256(BH * round4(L->L_max) * 4);
+  p.idx = off; off += round256(BH * L->M * 4);
+  p.olin = off; off += round256((size_t)L->B * L->Hq * L->d * 4);
+  p.partials = off; off += round256(BH * (L->M / lisa::kAttnRows) * (L->Hq / L->Hkv) * (L->d + 2) * 4);
+  p.counters = off; off += round256(BH * 4);
+  p.total = off;
+  return p;
+}
+
+struct RowsPlan {
+  int row_chunk, L_keys;
+  size_t keys, idx, olin, dS, Ptot, total;
+};
+RowsPlan rows_plan(const lisa_layer *L, int T, bool prefill) {
+  RowsPlan p;
+  const size_t BH = (size_t)L->B * L->Hkv;
+  p.row_chunk = T < kRowChunk ? T : kRowChunk;
+  p.L_keys = round4(prefill ? T : L->L_max);
+  size_t off = 0;
+  p.keys = off; off += round256(BH * p.row_chunk * p.L_keys * 4);
+  p.idx = p.olin = p.dS = p.Ptot = 0;
+  if (prefill) {
+    const size_t nc = (T + lisa::kLinChunk - 1) / lisa::kLinChunk;
+    p.idx = off; off += round256((size_t)L->B * T * L->Hkv * L->M * 4);
+    p.olin = off; off += round256((size_t)L->B * T * L->Hq * L->d * 4);
+    p.dS = off; off += round256(BH * nc * L->d * L->d * 4);
+    p.Ptot = off; off += round256(BH * L->d * L->d * 4);
+  }
+  p.total = off;
+  return p;
+}
+
+void fill_rows(lisa::RowsParams &r, const lisa_layer *L, int T) {
+  memset(&r, 0, sizeof(r));
+  r.B = L->B; r.Hq = L->Hq; r.Hkv = L->Hkv; r.G = L->Hq / L->Hkv; r.HI = L->HI; r.R = L->HI / L->Hkv;
+  r.D = L->d; r.DI = L->dI; r.M = L->M; r.L_max = L->L_max; r.T = T;
+  r.scale = (float)(1.0 / sqrt((double)L->d));
+  r.k_cache = L->k_cache; r.v_cache = L->v_cache; r.kidx_cache = L->kidx_cache;
+  r.state = L->state; r.pos = L->pos; r.err_word = L->err_word;
+}
+
+void set_select_smem(lisa::RowsParams &r, int n_max) {
+  const int cap = n_max < kRowsKeysCap ? n_max : kRowsKeysCap;
+  r.smem_keys_cap = (cap + 3) & ~3;
+  r.cand_cap = kCandCap;
+  r.select_smem = (size_t)(r.smem_keys_cap + r.cand_cap) * 4;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *lisa_version(void) { return "lisa-b200 0.1 (sm_100a)"; }
+
+const char *lisa_last_error_msg(void) { return g_msg; }
+
+const char *lisa_status_str(lisa_status s) {
+  switch (s) {
+    case LISA_OK: return "LISA_OK";
+    case LISA_ERR_INVALID_ARG: return "LISA_ERR_INVALID_ARG";
+    case LISA_ERR_UNSUPPORTED: return "LISA_ERR_UNSUPPORTED";
+    case LISA_ERR_CUDA: return "LISA_ERR_CUDA";
+    case LISA_ERR_WORKSPACE: return "LISA_ERR_WORKSPACE";
+  }
+  return "LISA_ERR_UNKNOWN";
+}
+
+size_t lisa_workspace_bytes(const lisa_layer *layer, int T, int op) {
+  if (check_layer(layer) != LISA_OK || T < 0) return 0;
+  if (op == LISA_OP_DECODE) return decode_plan(layer).total;
+  if (op == LISA_OP_PREFILL) return T ? rows_plan(layer, T, true).total : 0;
+  if (op == LISA_OP_INDEXER_TOPK) return T ? rows_plan(layer, T, false).total : 0;
+  return 0;
+}
+
+lisa_status lisa_append_cache(const lisa_layer *L, const void *k, const void *v, const void *kidx, int T,
+                              void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) || (s = check_ptr(kidx, "kidx"))) return s;
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.k = k; r.v = v; r.kidx = kidx;
+  cudaError_t e = lisa::launch_append(r, L->dtype, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "append");
+  return ok();
+}
+
+lisa_status lisa_indexer_topk(const lisa_layer *L, const void *qidx, const float *w, int T, int *idx_out,
+                              void *workspace, size_t ws_bytes, void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(idx_out, "idx_out"))) return s;
+  const RowsPlan plan = rows_plan(L, T, false);
+  if (!workspace || ws_bytes < plan.total)
+    return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
+  if ((s = check_ptr(workspace, "workspace"))) return s;
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.qidx = qidx; r.w = w; r.idx = idx_out;
+  char *ws = static_cast<char *>(workspace);
+  r.keys = reinterpret_cast<uint32_t *>(ws + plan.keys);
+  r.row_chunk = plan.row_chunk;
+  r.L_keys = plan.L_keys;
+  set_select_smem(r, L->L_max);
+  cudaError_t e = lisa::launch_rows_topk(r, L->dtype, (cudaStream_t)stream, L->L_max);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer_topk");
+  return ok();
+}
+
+lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, const void *v, const void *kidx,
+                             const void *qidx, const float *w, const float *gate_logit, int fuse_append, void *out,
+                             int *idx_out, void *workspace, size_t ws_bytes, void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (L->B == 0) return ok();
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(L->state, "state"))) return s;
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) || (s = check_ptr(kidx, "kidx")) ||
+      (s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(gate_logit, "gate_logit")) ||
+      (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)))
+    return s;
+  const DecodePlan plan = decode_plan(L);
+  if (!workspace || ws_bytes < plan.total)
+    return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
+  if ((s = check_ptr(workspace, "workspace"))) return s;
+
+  lisa::DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.B = L->B; p.Hq = L->Hq; p.Hkv = L->Hkv; p.G = L->Hq / L->Hkv; p.HI = L->HI; p.R = L->HI / L->Hkv;
+  p.D = L->d; p.DI = L->dI; p.M = L->M; p.L_max = L->L_max; p.fuse_append = fuse_append ? 1 : 0;
+  p.scale = (float)(1.0 / sqrt((double)L->d));
+  p.k_cache = L->k_cache; p.v_cache = L->v_cache; p.kidx_cache = L->kidx_cache;
+  p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;
+  p.q = q; p.k = k; p.v = v; p.kidx = kidx; p.qidx = qidx; p.w = w; p.gate = gate_logit;
+  p.out = out; p.idx_out = idx_out;
+  char *ws = static_cast<char *>(workspace);
+  p.keys = reinterpret_cast<uint32_t *>(ws + plan.keys);
+  p.keys_stride = round4(L->L_max);
+  p.idx = reinterpret_cast<int *>(ws + plan.idx);
+  p.olin = reinterpret_cast<float *>(ws + plan.olin);
+  p.partials = reinterpret_cast<float *>(ws + plan.partials);
+  p.counters = reinterpret_cast<unsigned *>(ws + plan.counters);
+  p.n_chunks = (L->L_max + 127) / 128;
+  p.n_score_blocks = L->B * L->Hkv * p.n_chunks;
+  p.n_state_blocks = L->B * L->Hq * (L->d / 32);
+  const int cap = L->L_max < kDecodeKeysCap ? L->L_max : kDecodeKeysCap;
+  p.smem_keys_cap = (cap + 3) & ~3;
+  p.cand_cap = kCandCap;
+  p.select_smem = (size_t)(p.smem_keys_cap + p.cand_cap) * 4;
+  if ((long long)p.n_score_blocks + p.n_state_blocks > 0x7fffffffLL)
+    return fail(LISA_ERR_UNSUPPORTED, "grid too large");
+  cudaError_t e = lisa::launch_decode(p, L->dtype, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step");
+  return ok();
+}
+
+lisa_status lisa_prefill(const lisa_layer *L, int T, const void *q, const void *k, const void *v, const void *kidx,
+                         const void *qidx, const float *w, const float *gate_logit, void *out, int *idx_out,
+                         void *workspace, size_t ws_bytes, void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(L->state, "state"))) return s;
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) || (s = check_ptr(kidx, "kidx")) ||
+      (s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(gate_logit, "gate_logit")) ||
+      (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)))
+    return s;
+  const RowsPlan plan = rows_plan(L, T, true);
+  if (!workspace || ws_bytes < plan.total)
+    return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
+  if ((s = check_ptr(workspace, "workspace"))) return s;
+
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.require_pos0 = 1;
+  r.q = q; r.k = k; r.v = v; r.kidx = kidx; r.qidx = qidx; r.w = w; r.gate = gate_logit; r.out = out;
+  char *ws = static_cast<char *>(workspace);
+  r.keys = reinterpret_cast<uint32_t *>(ws + plan.keys);
+  r.idx = idx_out ? idx_out : reinterpret_cast<int *>(ws + plan.idx);
+  r.olin = reinterpret_cast<float *>(ws + plan.olin);
+  r.dS = reinterpret_cast<float *>(ws + plan.dS);
+  r.Ptot = reinterpret_cast<float *>(ws + plan.Ptot);
+  r.row_chunk = plan.row_chunk;
+  r.L_keys = plan.L_keys;
+  set_select_smem(r, T);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = lisa::launch_append(r, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill append");
+  e = lisa::launch_prefill_linear(r, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill linear");
+  e = lisa::launch_rows_topk(r, L->dtype, st, T);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill indexer");
+  e = lisa::launch_prefill_attend(r, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill attend");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// Internal launch parameters shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lisa.h"
+
+namespace lisa {
+
+constexpr int kMaxR = 8;        // indexer heads per KV head
+constexpr int kMaxG = 16;       // query heads per KV head
+constexpr int kAttnRows = 32;   // selected rows per attention CTA / tile
+constexpr int kLinChunk = 64;   // chunk length of the chunked linear attention
+constexpr int kRowTile = 64;    // query rows per indexer score tile (row path)
+
+// ------------------------------------------------------------- decode
+struct DecodeParams {
+  int B, Hq, Hkv, G, HI, R, D, DI, M, L_max;
+  int fuse_append;
+  float scale;                          // 1 / sqrt(d)
+  // layer buffers
+  void *k_cache, *v_cache, *kidx_cache;
+  float *state;
+  const int *pos;
+  int *err_word;
+  // step inputs / outputs
+  const void *q, *k, *v, *kidx, *qidx;
+  const float *w, *gate;
+  void *out;
+  int *idx_out;
+  // workspace carve-up
+  uint32_t *keys;       // [B, Hkv, keys_stride] order keys
+  int keys_stride;      // L_max rounded up to a multiple of 4
+  int *idx;             // [B, Hkv, M]
+  float *olin;          // [B, Hq, d]
+  float *partials;      // [B, Hkv, M/kAttnRows, G, d+2]
+  unsigned *counters;   // [B, Hkv]
+  // launch geometry
+  int n_chunks, n_score_blocks, n_state_blocks;
+  int smem_keys_cap, cand_cap;
+  size_t select_smem;
+};
+
+cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t st);
+
+// ------------------------------------------------------------- row path
+// (prefill and lisa_indexer_topk): T query tokens at positions pos[b] + tau.
+struct RowsParams {
+  int B, Hq, Hkv, G, HI, R, D, DI, M, L_max, T;
+  float scale;
+  void *k_cache, *v_cache, *kidx_cache;
+  float *state;
+  const int *pos;
+  int *err_word;
+  int require_pos0;                     // prefill: pos[b] must be 0
+  const void *q, *k, *v, *kidx, *qidx;
+  const float *w, *gate;
+  void *out;
+  int *idx;                             // [B, T, Hkv, M] (caller's idx_out or workspace)
+  // workspace
+  uint32_t *keys;                       // [B, Hkv, row_chunk, L_keys]
+  float *olin;                          // [B, T, Hq, d]
+  float *dS;                            // [B, Hkv, n_lin_chunks, d, d]
+  float *Ptot;                          // [B, Hkv, d, d]
+  int row_chunk;                        // query rows scored per pass
+  int L_keys;                           // key slots per row in `keys` (multiple of 4)
+  int smem_keys_cap, cand_cap;
+  size_t select_smem;
+};
+
+cudaError_t launch_append(const RowsParams &p, int dtype, cudaStream_t st);
+cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, int key_limit);
+cudaError_t launch_prefill_linear(const RowsParams &p, int dtype, cudaStream_t st);
+cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st);
+
+}  // namespace lisa

@@ -1,0 +1,314 @@
+// Row path of LISA on sm_100a: cache append, indexer scores + top-M for a
+// block of query rows (prefill and lisa_indexer_topk), and the per-row sparse
+// attention with the gate epilogue (prefill).
+//
+// Method: arXiv 2607.19358 (LISA), abstract (indexer -> top-M -> sparse
+// attention, gated with a linear branch) and the gptget.net digest's method
+// section (ReLU dot-product indexer); exact formulas as stated in lisa.h.
+#include "lisa_internal.h"
+#include "lisa_select.cuh"
+
+namespace lisa {
+
+__device__ __forceinline__ bool rows_pos_ok(const RowsParams &p, int b) {
+  const int p0 = p.pos[b];
+  return p0 >= 0 && p0 + p.T <= p.L_max && (!p.require_pos0 || p0 == 0);
+}
+
+// ============================================================ append
+// grid (T, B*Hkv); copies k, v, kidx row tau of (b, g) to cache row pos[b]+tau.
+template <typename T>
+__global__ void append_kernel(RowsParams p) {
+  const int tau = blockIdx.x;
+  const int bg = blockIdx.y;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  if (!rows_pos_ok(p, b)) {
+    if (tau == 0 && g == 0 && threadIdx.x == 0) set_err(p.err_word, LISA_DEVERR_POS);
+    return;
+  }
+  const size_t dst = ((size_t)bg * p.L_max + p.pos[b] + tau);
+  const size_t src = ((size_t)b * p.T + tau) * p.Hkv + g;
+  const int nd = p.D * (int)sizeof(T) / 16, ndi = p.DI * (int)sizeof(T) / 16;
+  const uint4 *ks = reinterpret_cast<const uint4 *>(p.k) + src * nd;
+  const uint4 *vs = reinterpret_cast<const uint4 *>(p.v) + src * nd;
+  const uint4 *kis = reinterpret_cast<const uint4 *>(p.kidx) + src * ndi;
+  uint4 *kd = reinterpret_cast<uint4 *>(p.k_cache) + dst * nd;
+  uint4 *vd = reinterpret_cast<uint4 *>(p.v_cache) + dst * nd;
+  uint4 *kid = reinterpret_cast<uint4 *>(p.kidx_cache) + dst * ndi;
+  for (int i = threadIdx.x; i < nd; i += blockDim.x) {
+    kd[i] = ks[i];
+    vd[i] = vs[i];
+  }
+  for (int i = threadIdx.x; i < ndi; i += blockDim.x) kid[i] = kis[i];
+}
+
+cudaError_t launch_append(const RowsParams &p, int dtype, cudaStream_t st) {
+  dim3 grid(p.T, p.B * p.Hkv);
+  if (dtype == LISA_BF16)
+    append_kernel<__nv_bfloat16><<<grid, 64, 0, st>>>(p);
+  else
+    append_kernel<float><<<grid, 64, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+// ============================================================ scores (CUDA cores)
+// grid (key tiles, row tiles of the pass, B*Hkv); 256 threads, 4x4 scores each.
+// Row tau of the pass sits at position pos[b] + tau; key s is a candidate iff
+// s <= pos[b] + tau.  Output: order keys, keys[(bg*row_chunk + tau - tau0)*L_keys + s].
+template <typename T, int DI>
+__global__ void __launch_bounds__(256) rows_score_kernel(RowsParams p, int tau0, int rows) {
+  __shared__ float s_k[64][DI + 1];
+  __shared__ float s_q[64][DI + 1];
+  __shared__ float s_w[64];
+  const int kt = blockIdx.x, rt = blockIdx.y, bg = blockIdx.z;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  if (!rows_pos_ok(p, b)) return;
+  const int p0 = p.pos[b];
+  const int r_lo = rt * 64;                      // within the pass
+  if (r_lo >= rows) return;
+  const int r_hi = min(r_lo + 64, rows);
+  const int s_lo = kt * 64;
+  const int last_pos = p0 + tau0 + r_hi - 1;
+  if (s_lo > last_pos) return;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+
+  // indexer keys of the tile
+  for (int i = tid; i < 64 * DI; i += 256) {
+    const int r = i / DI, c = i % DI;
+    const int s = s_lo + r;
+    float x = 0.f;
+    if (s <= last_pos)
+      x = Dt<T>::to_f(reinterpret_cast<const T *>(p.kidx_cache)[((size_t)bg * p.L_max + s) * DI + c]);
+    s_k[r][c] = x;
+  }
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int r = 0; r < p.R; ++r) {
+    const int hi = g * p.R + r;
+    __syncthreads();
+    for (int i = tid; i < 64 * DI; i += 256) {
+      const int rr = i / DI, c = i % DI;
+      const int tau = tau0 + r_lo + rr;
+      float x = 0.f;
+      if (r_lo + rr < r_hi)
+        x = Dt<T>::to_f(reinterpret_cast<const T *>(p.qidx)[(((size_t)b * p.T + tau) * p.HI + hi) * DI + c]);
+      s_q[rr][c] = x;
+    }
+    if (tid < 64) {
+      const int tau = tau0 + r_lo + tid;
+      s_w[tid] = (r_lo + tid < r_hi) ? p.w[((size_t)b * p.T + tau) * p.HI + hi] : 0.f;
+    }
+    __syncthreads();
+    float dot[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dot[i][j] = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < DI; ++c) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = s_q[ty * 4 + i][c];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bb[j] = s_k[tx * 4 + j][c];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dot[i][j] = fmaf(a[i], bb[j], dot[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(s_w[ty * 4 + i], fmaxf(dot[i][j], 0.f), acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = r_lo + ty * 4 + i;
+    if (rr >= r_hi) continue;
+    const int tpos = p0 + tau0 + rr;
+    uint32_t *krow = p.keys + ((size_t)bg * p.row_chunk + rr) * p.L_keys;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int s = s_lo + tx * 4 + j;
+      if (s <= tpos) krow[s] = score_key(acc[i][j]);
+    }
+  }
+}
+
+// ============================================================ select
+// grid (rows of the pass, B*Hkv)
+template <int NT>
+__global__ void __launch_bounds__(NT) rows_select_kernel(RowsParams p, int tau0, int rows) {
+  extern __shared__ __align__(16) uint32_t s_dyn[];
+  __shared__ TopmShared sm;
+  const int rr = blockIdx.x, bg = blockIdx.y;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  if (rr >= rows || !rows_pos_ok(p, b)) return;
+  const int tau = tau0 + rr;
+  const int n = p.pos[b] + tau + 1;
+  const uint32_t *gkeys = p.keys + ((size_t)bg * p.row_chunk + rr) * p.L_keys;
+  const uint32_t *keys = gkeys;
+  uint32_t *cand = s_dyn;
+  if (n > p.M && n <= p.smem_keys_cap) {
+    const int n4 = n & ~3;
+    for (int i = threadIdx.x * 4; i < n4; i += NT * 4)
+      *reinterpret_cast<uint4 *>(s_dyn + i) = __ldcg(reinterpret_cast<const uint4 *>(gkeys + i));
+    for (int i = n4 + threadIdx.x; i < n; i += NT) s_dyn[i] = __ldcg(gkeys + i);
+    __syncthreads();
+    keys = s_dyn;
+    cand = s_dyn + p.smem_keys_cap;
+  }
+  int *out = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M;
+  block_topm<NT>(keys, n, p.M, out, sm, cand, p.cand_cap);
+}
+
+template <typename T, int DI>
+static cudaError_t rows_topk_t(const RowsParams &p, cudaStream_t st, int key_limit) {
+  constexpr int NT = 256;
+  cudaError_t e = cudaFuncSetAttribute(rows_select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)p.select_smem);
+  if (e != cudaSuccess) return e;
+  for (int tau0 = 0; tau0 < p.T; tau0 += p.row_chunk) {
+    const int rows = min(p.row_chunk, p.T - tau0);
+    // prefill (pos 0): keys up to tau0 + rows; general positions: up to key_limit
+    const int key_hi = p.require_pos0 ? min(key_limit, tau0 + rows) : key_limit;
+    dim3 g1((key_hi + 63) / 64, (rows + 63) / 64, p.B * p.Hkv);
+    rows_score_kernel<T, DI><<<g1, 256, 0, st>>>(p, tau0, rows);
+    dim3 g2(rows, p.B * p.Hkv);
+    rows_select_kernel<NT><<<g2, NT, p.select_smem, st>>>(p, tau0, rows);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, int key_limit) {
+  if (dtype == LISA_BF16) {
+    if (p.DI == 64) return rows_topk_t<__nv_bfloat16, 64>(p, st, key_limit);
+    if (p.DI == 32) return rows_topk_t<__nv_bfloat16, 32>(p, st, key_limit);
+  } else {
+    if (p.DI == 64) return rows_topk_t<float, 64>(p, st, key_limit);
+    if (p.DI == 32) return rows_topk_t<float, 32>(p, st, key_limit);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ============================================================ attention + gate
+// grid (T, B*Hkv); 256 threads.  Online softmax over tiles of 32 selected rows.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
+  constexpr int kRows = kAttnRows;
+  constexpr int kDPL = D / 32;
+  constexpr int kSlots = kMaxG / 8;   // heads per warp
+  __shared__ __align__(16) T s_k[kRows][D];
+  __shared__ __align__(16) T s_v[kRows][D];
+  __shared__ float s_q[kMaxG][D];
+  __shared__ float s_logit[kMaxG][kRows];
+  __shared__ int s_idx[kRows];
+  const int tau = blockIdx.x, bg = blockIdx.y;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  if (!rows_pos_ok(p, b)) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = p.G;
+  for (int i = tid; i < G * D; i += 256) {
+    const int hh = i / D, dd = i % D;
+    s_q[hh][dd] = Dt<T>::to_f(reinterpret_cast<const T *>(p.q)[(((size_t)b * p.T + tau) * p.Hq + g * G + hh) * D + dd]);
+  }
+  float m[kSlots], l[kSlots], acc[kSlots][kDPL];
+#pragma unroll
+  for (int s = 0; s < kSlots; ++s) {
+    m[s] = -INFINITY;
+    l[s] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kDPL; ++j) acc[s][j] = 0.f;
+  }
+  const int *idx = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M;
+  const T *kc = reinterpret_cast<const T *>(p.k_cache) + (size_t)bg * p.L_max * D;
+  const T *vc = reinterpret_cast<const T *>(p.v_cache) + (size_t)bg * p.L_max * D;
+  constexpr int kSlices = D * (int)sizeof(T) / 16;
+  for (int tile = 0; tile < p.M / kRows; ++tile) {
+    __syncthreads();
+    if (tid < kRows) s_idx[tid] = idx[tile * kRows + tid];
+    __syncthreads();
+    if (s_idx[0] < 0) break;
+    for (int i = tid; i < kRows * kSlices; i += 256) {
+      const int r = i / kSlices, sl = i % kSlices;
+      const int s = s_idx[r];
+      uint4 uk = make_uint4(0, 0, 0, 0), uv = make_uint4(0, 0, 0, 0);
+      if (s >= 0) {
+        uk = *reinterpret_cast<const uint4 *>(kc + (size_t)s * D + sl * (16 / sizeof(T)));
+        uv = *reinterpret_cast<const uint4 *>(vc + (size_t)s * D + sl * (16 / sizeof(T)));
+      }
+      reinterpret_cast<uint4 *>(&s_k[r][0])[sl] = uk;
+      reinterpret_cast<uint4 *>(&s_v[r][0])[sl] = uv;
+    }
+    __syncthreads();
+    for (int r = warp; r < kRows; r += 8) {
+      float kx[kDPL];
+#pragma unroll
+      for (int j = 0; j < kDPL; ++j) kx[j] = Dt<T>::to_f(s_k[r][lane * kDPL + j]);
+      const bool valid = s_idx[r] >= 0;
+      for (int hh = 0; hh < G; ++hh) {
+        float dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < kDPL; ++j) dot = fmaf(s_q[hh][lane * kDPL + j], kx[j], dot);
+        dot = warp_sum(dot);
+        if (lane == 0) s_logit[hh][r] = valid ? dot * p.scale : -INFINITY;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int s = 0; s < kSlots; ++s) {
+      const int hh = warp + 8 * s;
+      if (hh >= G) continue;
+      const float x = s_logit[hh][lane];
+      const float mt = warp_max(x);
+      const float mn = fmaxf(m[s], mt);
+      const float f = (m[s] == -INFINITY) ? 0.f : expf(m[s] - mn);
+      const float e = (x == -INFINITY) ? 0.f : expf(x - mn);
+      l[s] = l[s] * f + warp_sum(e);
+      m[s] = mn;
+#pragma unroll
+      for (int j = 0; j < kDPL; ++j) acc[s][j] *= f;
+      for (int r = 0; r < kRows; ++r) {
+        const float pr = __shfl_sync(0xffffffffu, e, r);
+#pragma unroll
+        for (int j = 0; j < kDPL; ++j) acc[s][j] = fmaf(pr, Dt<T>::to_f(s_v[r][lane * kDPL + j]), acc[s][j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < kSlots; ++s) {
+    const int hh = warp + 8 * s;
+    if (hh >= G) continue;
+    const int h = g * G + hh;
+    const size_t row = ((size_t)b * p.T + tau) * p.Hq + h;
+    const float gam = 1.f / (1.f + expf(-p.gate[row]));
+#pragma unroll
+    for (int j = 0; j < kDPL; ++j) {
+      const int dd = lane * kDPL + j;
+      const float o_sp = acc[s][j] / l[s];
+      const float o_lin = p.olin[row * D + dd];
+      reinterpret_cast<T *>(p.out)[row * D + dd] = Dt<T>::from_f(gam * o_sp + (1.f - gam) * o_lin);
+    }
+  }
+}
+
+cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st) {
+  dim3 grid(p.T, p.B * p.Hkv);
+  if (dtype == LISA_BF16) {
+    if (p.D == 128) prefill_attend_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(p);
+    else prefill_attend_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(p);
+  } else {
+    if (p.D == 128) prefill_attend_kernel<float, 128><<<grid, 256, 0, st>>>(p);
+    else prefill_attend_kernel<float, 64><<<grid, 256, 0, st>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lisa

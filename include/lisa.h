@@ -1,0 +1,175 @@
+/*
+ * lisa.h -- C ABI of the LISA (Linear-Indexed Sparse Attention) layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "LISA: Linear-Indexed Sparse Attention for Efficient Long-Context
+ * Reasoning" (arXiv 2607.19358).  Its abstract defines the layer: a Lightning
+ * Indexer picks the top-M tokens of the whole context for a sparse softmax
+ * self-attention, a linear-attention branch runs beside it, and a gate fuses
+ * the two outputs, so n generated tokens cost O(nM).  The gptget.net digest of
+ * the paper (section "方法详解", method details) adds: phi = identity with a
+ * state matrix S_t, an indexer made of query/key projections and a ReLU dot
+ * product, and a learned gate g; its "实验设计" (experiment design) section
+ * gives M = 256.
+ *
+ * Definitions this library fixes where the pages are silent (the oracle used
+ * by the tests applies the same ones):
+ *   score   I_g(t,s) = sum_{r<R} w[t, g*R+r] * max(0, qidx[t, g*R+r] . kidx[g, s]),
+ *           R = HI / Hkv, candidates s = 0..t (the current token included);
+ *   select  per KV head g the first min(M, t+1) positions in the order
+ *           (score descending, position ascending); -0.0 equals +0.0;
+ *   sparse  o_sp[h] = softmax_{s in Sel_g}(q_h . k_s / sqrt(d)) . v_s for each
+ *           query head h of group g = h / (Hq / Hkv);
+ *   linear  S_h <- S_h + k_t^T v_t, then o_lin[h] = q_h S_h (no normaliser);
+ *   gate    g = 1 / (1 + exp(-lambda_h)), o = g * o_sp + (1 - g) * o_lin.
+ *
+ * Conventions for every entry point
+ *   - All tensor arguments are DEVICE pointers to dense row-major arrays owned
+ *     by the caller.  The library never allocates, frees or synchronises.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL =
+ *     legacy default stream) and returns immediately.
+ *   - Arguments are validated on the host before anything is launched; on
+ *     failure nothing is launched and a status other than LISA_OK is returned.
+ *     lisa_last_error_msg() then describes the failure (thread-local).
+ *   - Launch failures reported by the CUDA runtime map to LISA_ERR_CUDA.
+ *   - Checks that need device data (pos[b] out of range) are made on the
+ *     device: the kernels skip the affected sequence and OR a bit into
+ *     *err_word (when err_word is non-NULL); they never trap.
+ *   - Storage dtype (q, k, v, caches, out): bf16 or fp32, per lisa_layer.dtype.
+ *     w, gate logits and the state are always fp32; indices are int32.
+ *   - Supported shapes: d in {64, 128}; dI in {32, 64}; M a multiple of 32 in
+ *     [32, 1024]; Hq % Hkv == 0, HI % Hkv == 0, HI / Hkv <= 8, Hq / Hkv <= 16;
+ *     L_max >= 1.  Anything else returns LISA_ERR_UNSUPPORTED.
+ *   - All pointers must be 16-byte aligned.
+ */
+#ifndef LISA_H_
+#define LISA_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LISA_API __attribute__((visibility("default")))
+#else
+#define LISA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LISA_OK = 0,
+  LISA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned pointer */
+  LISA_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes */
+  LISA_ERR_CUDA = 3,          /* the CUDA runtime rejected a launch */
+  LISA_ERR_WORKSPACE = 4      /* workspace NULL or smaller than lisa_workspace_bytes() */
+} lisa_status;
+
+typedef enum { LISA_BF16 = 0, LISA_FP32 = 1 } lisa_dtype;
+
+/* Bits a kernel ORs into *err_word. */
+#define LISA_DEVERR_POS      1   /* pos[b] < 0, or pos[b] + T > L_max: sequence b skipped */
+#define LISA_DEVERR_TIMEOUT  2   /* a bounded wait on an asynchronous copy gave up */
+
+/* Operation codes for lisa_workspace_bytes(). */
+#define LISA_OP_DECODE       0
+#define LISA_OP_PREFILL      1
+#define LISA_OP_INDEXER_TOPK 2
+
+/* One attention layer: geometry plus the caller-owned per-layer buffers. */
+typedef struct {
+  int B;        /* sequences in the batch */
+  int Hq;       /* query heads */
+  int Hkv;      /* key/value heads; G = Hq / Hkv query heads share one */
+  int d;        /* head dim of q, k, v */
+  int HI;       /* indexer heads; R = HI / Hkv belong to each KV head */
+  int dI;       /* indexer head dim */
+  int M;        /* tokens kept per KV head by the top-M selection */
+  int L_max;    /* rows of every cache buffer */
+  int dtype;    /* lisa_dtype of q, k, v, caches and outputs */
+  void *k_cache;     /* [B, Hkv, L_max, d]  */
+  void *v_cache;     /* [B, Hkv, L_max, d]  */
+  void *kidx_cache;  /* [B, Hkv, L_max, dI] indexer keys, one per KV head */
+  float *state;      /* [B, Hq, d, d] fp32 linear state S[i][j] (key dim i, value dim j),
+                        updated in place */
+  const int *pos;    /* [B] device: position of the first new token of this call
+                        (= tokens already cached) */
+  int *err_word;     /* device int or NULL: LISA_DEVERR_* bits are ORed in */
+} lisa_layer;
+
+/*
+ * Bytes of scratch the caller must pass as `workspace` for operation `op`
+ * (LISA_OP_*) with T new tokens per sequence.  Returns 0 for invalid input.
+ * The workspace holds no state between calls (each call initialises what it
+ * uses) but one workspace must not be used by two calls that overlap on the
+ * device.
+ */
+LISA_API size_t lisa_workspace_bytes(const lisa_layer *layer, int T, int op);
+
+/*
+ * Append T new tokens per sequence to the caches (the cache write that
+ * generating a token implies; abstract of arXiv 2607.19358).
+ *   k, v  [B, T, Hkv, d]; kidx [B, T, Hkv, dI]   (storage dtype)
+ * Row tau of sequence b goes to cache row pos[b] + tau.  Re-appending at the
+ * same positions rewrites the same rows.  pos is not advanced.
+ */
+LISA_API lisa_status lisa_append_cache(const lisa_layer *layer, const void *k, const void *v,
+                              const void *kidx, int T, void *stream);
+
+/*
+ * Lightning Indexer + top-M only (abstract of arXiv 2607.19358; score and order
+ * as defined above) for T query tokens per sequence at positions
+ * pos[b] .. pos[b]+T-1, against cache rows 0 .. pos[b]+tau (the caller must
+ * have appended the T tokens first).
+ *   qidx    [B, T, HI, dI] (storage dtype); w [B, T, HI] fp32
+ *   idx_out [B, T, Hkv, M] int32: selected positions in ascending order,
+ *           padded with -1 when the prefix holds fewer than M tokens.
+ */
+LISA_API lisa_status lisa_indexer_topk(const lisa_layer *layer, const void *qidx, const float *w, int T,
+                              int *idx_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * One decode step: the new token of every sequence sits at position t = pos[b].
+ *   q [B, Hq, d]; k, v [B, Hkv, d]; kidx [B, Hkv, dI]; qidx [B, HI, dI]
+ *   (storage dtype); w [B, HI] fp32; gate_logit [B, Hq] fp32
+ *   out [B, Hq, d] (storage dtype)
+ *   idx_out: NULL or [B, Hkv, M] int32 (the selected positions)
+ * The new token's k, v, kidx are taken from the arguments (not the cache) and,
+ * when fuse_append != 0, also written to cache row t.  With fuse_append == 0
+ * the caller must already have stored them there.  The state is updated in
+ * place (S <- S + k^T v).  pos is not advanced.
+ */
+LISA_API lisa_status lisa_decode_step(const lisa_layer *layer, const void *q, const void *k, const void *v,
+                             const void *kidx, const void *qidx, const float *w,
+                             const float *gate_logit, int fuse_append, void *out, int *idx_out,
+                             void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Causal prefill of T tokens per sequence starting from an empty cache
+ * (pos[b] must be 0; a sequence with another pos is skipped and flagged).
+ *   q [B, T, Hq, d]; k, v [B, T, Hkv, d]; kidx [B, T, Hkv, dI];
+ *   qidx [B, T, HI, dI] (storage dtype); w [B, T, HI] fp32;
+ *   gate_logit [B, T, Hq] fp32; out [B, T, Hq, d] (storage dtype);
+ *   idx_out: NULL or [B, T, Hkv, M] int32.
+ * The T tokens are appended to the caches.  The state is read as S_0 and
+ * overwritten with S_T.  Row tau's output equals the decode step of token tau.
+ */
+LISA_API lisa_status lisa_prefill(const lisa_layer *layer, int T, const void *q, const void *k,
+                         const void *v, const void *kidx, const void *qidx, const float *w,
+                         const float *gate_logit, void *out, int *idx_out, void *workspace,
+                         size_t ws_bytes, void *stream);
+
+/* Human-readable name of a status. */
+LISA_API const char *lisa_status_str(lisa_status s);
+
+/* Description of the last failure on the calling thread ("" if none). */
+LISA_API const char *lisa_last_error_msg(void);
+
+/* Library version string. */
+LISA_API const char *lisa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LISA_H_ */

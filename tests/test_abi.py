@@ -1,0 +1,133 @@
+"""The C ABI without a GPU: the library loads, exports what include/lisa.h
+declares, and rejects bad arguments on the host before launching anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+L = pytest.importorskip("hybrid_linear_top_b200.lisa")
+
+HEADER = os.path.join(ROOT, "include", "lisa.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"LISA_API\s+[\w\s\*]*?\b(lisa_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_symbols()
+    for n in ["lisa_prefill", "lisa_decode_step", "lisa_indexer_topk", "lisa_append_cache",
+              "lisa_workspace_bytes", "lisa_status_str", "lisa_last_error_msg"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(L.LIB_PATH)
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+    assert sorted(L.EXPORTED) == sorted(declared_symbols())
+
+
+def _layer(**kw):
+    f = dict(B=1, Hq=12, Hkv=2, d=128, HI=4, dI=64, M=256, L_max=16384, dtype=L.LISA_BF16)
+    f.update(kw)
+    c = L.LisaLayerC(f["B"], f["Hq"], f["Hkv"], f["d"], f["HI"], f["dI"], f["M"], f["L_max"], f["dtype"])
+    fake = 0x10000  # aligned, never dereferenced: every call below fails validation first
+    for name in ["k_cache", "v_cache", "kidx_cache", "state", "pos", "err_word"]:
+        setattr(c, name, kw.get(name, fake))
+    return c
+
+
+FAKE = ctypes.c_void_p(0x20000)
+
+
+def _decode(c, ws=FAKE, ws_bytes=1 << 40, **ptrs):
+    args = {n: ptrs.get(n, FAKE) for n in ["q", "k", "v", "kidx", "qidx", "w", "gate", "out"]}
+    lib = L.lib()
+    return lib.lisa_decode_step(ctypes.byref(c), args["q"], args["k"], args["v"], args["kidx"], args["qidx"],
+                                args["w"], args["gate"], 1, args["out"], None, ws, ws_bytes, None)
+
+
+def test_status_strings():
+    assert L.status_str(L.LISA_OK) == "LISA_OK"
+    assert L.status_str(L.LISA_ERR_UNSUPPORTED) == "LISA_ERR_UNSUPPORTED"
+    assert L.status_str(99) == "LISA_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), L.LISA_ERR_UNSUPPORTED),
+    (dict(dI=48), L.LISA_ERR_UNSUPPORTED),
+    (dict(Hq=13), L.LISA_ERR_UNSUPPORTED),
+    (dict(HI=3), L.LISA_ERR_UNSUPPORTED),
+    (dict(M=48), L.LISA_ERR_UNSUPPORTED),
+    (dict(M=2048), L.LISA_ERR_UNSUPPORTED),
+    (dict(Hq=34, Hkv=2, HI=2), L.LISA_ERR_UNSUPPORTED),     # G = 17 > 16
+    (dict(HI=18, Hkv=2, Hq=2), L.LISA_ERR_UNSUPPORTED),     # R = 9 > 8
+    (dict(L_max=0), L.LISA_ERR_INVALID_ARG),
+    (dict(B=-1), L.LISA_ERR_INVALID_ARG),
+    (dict(dtype=7), L.LISA_ERR_INVALID_ARG),
+    (dict(k_cache=0), L.LISA_ERR_INVALID_ARG),
+    (dict(pos=0), L.LISA_ERR_INVALID_ARG),
+    (dict(state=0), L.LISA_ERR_INVALID_ARG),
+    (dict(v_cache=0x10008), L.LISA_ERR_INVALID_ARG),        # misaligned
+])
+def test_decode_rejects_bad_layer(kw, status):
+    assert _decode(_layer(**kw)) == status
+    assert L.last_error_msg() != ""
+
+
+def test_decode_rejects_null_and_misaligned_inputs():
+    c = _layer()
+    assert _decode(c, q=None) == L.LISA_ERR_INVALID_ARG
+    assert "q" in L.last_error_msg()
+    assert _decode(c, out=ctypes.c_void_p(0x20004)) == L.LISA_ERR_INVALID_ARG
+
+
+def test_decode_rejects_small_workspace():
+    c = _layer()
+    need = L.lisa_workspace_bytes(c, 1, L.LISA_OP_DECODE)
+    assert need > 0
+    assert _decode(c, ws_bytes=need - 1) == L.LISA_ERR_WORKSPACE
+    assert _decode(c, ws=None) == L.LISA_ERR_WORKSPACE
+
+
+def test_empty_inputs_are_noops():
+    c = _layer(B=0)
+    assert _decode(c) == L.LISA_OK
+    lib = L.lib()
+    c1 = _layer()
+    assert lib.lisa_append_cache(ctypes.byref(c1), FAKE, FAKE, FAKE, 0, None) == L.LISA_OK
+    assert lib.lisa_prefill(ctypes.byref(c1), 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 0,
+                            None) == L.LISA_OK
+    assert lib.lisa_indexer_topk(ctypes.byref(c1), FAKE, FAKE, 0, FAKE, FAKE, 0, None) == L.LISA_OK
+
+
+def test_row_calls_validate():
+    lib = L.lib()
+    c = _layer(L_max=100)
+    assert lib.lisa_append_cache(ctypes.byref(c), FAKE, FAKE, FAKE, -1, None) == L.LISA_ERR_INVALID_ARG
+    assert lib.lisa_append_cache(ctypes.byref(c), FAKE, FAKE, FAKE, 101, None) == L.LISA_ERR_INVALID_ARG
+    assert lib.lisa_append_cache(ctypes.byref(c), None, FAKE, FAKE, 5, None) == L.LISA_ERR_INVALID_ARG
+    assert lib.lisa_indexer_topk(ctypes.byref(c), FAKE, FAKE, 5, None, FAKE, 1 << 40, None) == L.LISA_ERR_INVALID_ARG
+    assert lib.lisa_indexer_topk(ctypes.byref(c), FAKE, FAKE, 5, FAKE, FAKE, 16, None) == L.LISA_ERR_WORKSPACE
+    assert lib.lisa_prefill(ctypes.byref(c), 5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16,
+                            None) == L.LISA_ERR_WORKSPACE
+    assert lib.lisa_prefill(ctypes.byref(c), 5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, 1 << 40,
+                            None) == L.LISA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes():
+    c = _layer()
+    dec = L.lisa_workspace_bytes(c, 1, L.LISA_OP_DECODE)
+    # decode needs at least one fp32 order key per cached position per KV head
+    assert dec >= 1 * 2 * 16384 * 4
+    pre = L.lisa_workspace_bytes(c, 16384, L.LISA_OP_PREFILL)
+    assert pre >= 16384 * 12 * 128 * 4          # per-token linear outputs
+    assert L.lisa_workspace_bytes(c, 4, L.LISA_OP_INDEXER_TOPK) > 0
+    assert L.lisa_workspace_bytes(_layer(d=96), 1, L.LISA_OP_DECODE) == 0
+    assert L.lisa_workspace_bytes(c, 1, 42) == 0

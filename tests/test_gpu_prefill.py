@@ -1,0 +1,151 @@
+"""GPU parity of lisa_prefill (and prefill followed by decode steps) against
+the fp64 oracle, through the C ABI."""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lisa_inputs import get_config, make_rng, gen_layer, gen_step
+from harness import make_layer, step_tensors, check_set, check_out, check_state, f64, dev
+
+pytestmark = pytest.mark.gpu
+
+L = pytest.importorskip("hybrid_linear_top_b200.lisa")
+
+
+def gpu_prefill(cfg, layer_np, step, T, L_max):
+    lay = make_layer(L, cfg, L_max, layer_np, n_rows=0)
+    x = step_tensors(step, cfg)
+    ws = L.alloc_workspace(lay, T, L.LISA_OP_PREFILL)
+    out = torch.empty(cfg.B, T, cfg.Hq, cfg.d, dtype=lay.torch_dtype, device="cuda")
+    idx = torch.full((cfg.B, T, cfg.Hkv, cfg.M), -7, dtype=torch.int32, device="cuda")
+    L.lisa_prefill(lay, T, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], out, idx, ws)
+    torch.cuda.synchronize()
+    assert int(lay.err_word.item()) == 0
+    return lay, out, idx
+
+
+def check_prefill(cfg, layer_np, step, lay, out, idx, rows=None):
+    a = lambda z: z.astype(np.float64)
+    idx_g = idx.cpu().numpy().astype(np.int64)
+    ref = oracle.prefill(a(step.q), a(step.k), a(step.v), a(step.qidx), a(step.kidx), a(step.w), a(step.lam),
+                         a(layer_np.S0), cfg.M, rows=rows, sel_override=lambda b, t: idx_g[b, t])
+    T = step.q.shape[1]
+    rows = range(T) if rows is None else rows
+    for (b, t), sc in ref["scores"].items():
+        for g in range(cfg.Hkv):
+            check_set(idx_g[b, t, g], sc[g], cfg.M, t, where=f"b={b} t={t} g={g}")
+    o = f64(out)
+    r = np.asarray(list(rows))
+    check_out(o[:, r], ref["out"][:, r], cfg.dtype, where="prefill out")
+    check_state(f64(lay.state), ref["S"], where="prefill state")
+    # the caches hold the T tokens
+    np.testing.assert_array_equal(f64(lay.k_cache[:, :, :T]), np.transpose(a(step.k), (0, 2, 1, 3)))
+    np.testing.assert_array_equal(f64(lay.kidx_cache[:, :, :T]), np.transpose(a(step.kidx), (0, 2, 1, 3)))
+    return ref
+
+
+def test_tiny_fp32_prefill_then_decode():
+    """Tiny fp32 layer: prefill 512 tokens, then 16 decode steps, each checked."""
+    cfg = get_config("tiny_fp32")
+    rng = make_rng(cfg.seed, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    pre = gen_step(cfg, rng, cfg.T)
+    lay, out, idx = gpu_prefill(cfg, layer_np, pre, cfg.T, cfg.L_max)
+    ref = check_prefill(cfg, layer_np, pre, lay, out, idx)
+
+    a = lambda z: z.astype(np.float64)
+    kc = np.transpose(a(pre.k), (0, 2, 1, 3))
+    vc = np.transpose(a(pre.v), (0, 2, 1, 3))
+    kic = np.transpose(a(pre.kidx), (0, 2, 1, 3))
+    S = ref["S"]
+    ws = L.alloc_workspace(lay, 1, L.LISA_OP_DECODE)
+    o = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=lay.torch_dtype, device="cuda")
+    ig = torch.empty(cfg.B, cfg.Hkv, cfg.M, dtype=torch.int32, device="cuda")
+    lay.pos.fill_(cfg.T)
+    for n in range(cfg.n_decode):
+        st = gen_step(cfg, rng, 1)
+        x = step_tensors(st, cfg, tau=0)
+        L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, o, ig, ws)
+        lay.pos.add_(1)
+        torch.cuda.synchronize()
+        s0 = lambda z: a(z[:, 0])
+        t = cfg.T + n
+        idx_g = ig.cpu().numpy().astype(np.int64)
+        r = oracle.decode_step(s0(st.q), s0(st.k), s0(st.v), s0(st.qidx), s0(st.kidx), s0(st.w), s0(st.lam),
+                               kc, vc, kic, S, np.array([t]), cfg.M, sel_override=idx_g)
+        for g in range(cfg.Hkv):
+            check_set(idx_g[0, g], r["scores"][0][g], cfg.M, t, where=f"step {n}")
+        check_out(f64(o), r["out"], cfg.dtype, where=f"decode step {n}")
+        check_state(f64(lay.state), r["S"], where=f"state step {n}")
+        S = r["S"]
+        kc = np.concatenate([kc, s0(st.k)[:, :, None]], axis=2)
+        vc = np.concatenate([vc, s0(st.v)[:, :, None]], axis=2)
+        kic = np.concatenate([kic, s0(st.kidx)[:, :, None]], axis=2)
+    assert int(lay.err_word.item()) == 0
+
+
+@pytest.mark.parametrize("T", [1, 2, 64, 255, 256, 257, 1500])
+def test_prefill_1p5b_shape_small(T):
+    """1.5B geometry at small T: chunk edges, prefixes around M, two row passes."""
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=T, B=1 if T > 300 else 2, S0="normal")
+    rng = make_rng(200 + T, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = gen_step(cfg, rng, T)
+    lay, out, idx = gpu_prefill(cfg, layer_np, step, T, T + 5)
+    check_prefill(cfg, layer_np, step, lay, out, idx)
+
+
+@pytest.mark.slow
+def test_prefill_1p5b_16k_sampled():
+    """Full 16384-token prefill; outputs and sets checked on sampled rows,
+    the final state in full."""
+    cfg = get_config("prefill_1p5b_16k")
+    rng = make_rng(cfg.seed, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = gen_step(cfg, rng, cfg.T)
+    lay, out, idx = gpu_prefill(cfg, layer_np, step, cfg.T, cfg.L_max)
+    sr = np.random.default_rng(0)
+    rows = sorted(set([0, 1, 63, 64, 255, 256, 1023, 1024, 8191, 16383] + sr.integers(0, cfg.T, 14).tolist()))
+    check_prefill(cfg, layer_np, step, lay, out, idx, rows=rows)
+
+
+def test_prefill_rejects_nonzero_position():
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=40, B=2)
+    rng = make_rng(9, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = gen_step(cfg, rng, 40)
+    lay = make_layer(L, cfg, 100, layer_np, n_rows=0, poison=False)
+    lay.pos.copy_(torch.tensor([0, 3], dtype=torch.int32))
+    x = step_tensors(step, cfg)
+    ws = L.alloc_workspace(lay, 40, L.LISA_OP_PREFILL)
+    out = torch.zeros(2, 40, cfg.Hq, cfg.d, dtype=lay.torch_dtype, device="cuda")
+    L.lisa_prefill(lay, 40, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], out, None, ws)
+    torch.cuda.synchronize()
+    assert int(lay.err_word.item()) & L.LISA_DEVERR_POS
+    assert (out[1] == 0).all()
+    assert torch.isfinite(out[0].float()).all()
+
+
+def test_indexer_topk_rows_match_prefill_sets():
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=700, B=1)
+    rng = make_rng(21, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = gen_step(cfg, rng, 700)
+    lay = make_layer(L, cfg, 800, layer_np, n_rows=0)
+    x = step_tensors(step, cfg)
+    L.lisa_append_cache(lay, x["k"], x["v"], x["kidx"], 700)
+    ws = L.alloc_workspace(lay, 700, L.LISA_OP_INDEXER_TOPK)
+    idx = torch.full((1, 700, cfg.Hkv, cfg.M), -7, dtype=torch.int32, device="cuda")
+    L.lisa_indexer_topk(lay, x["qidx"], x["w"], 700, idx, ws)
+    torch.cuda.synchronize()
+    idx_g = idx.cpu().numpy()
+    a = lambda z: z.astype(np.float64)
+    keys = np.transpose(a(step.kidx[0]), (1, 0, 2))
+    for t in [0, 5, 255, 256, 300, 699]:
+        sc = oracle.indexer_scores(a(step.qidx[0, t]), a(step.w[0, t]), keys[:, : t + 1])
+        for g in range(cfg.Hkv):
+            check_set(idx_g[0, t, g], sc[g], cfg.M, t, where=f"t={t} g={g}")
