@@ -296,6 +296,11 @@ def run_lisa(args, rank, world):
     ms_per_step = ms / steps_total
     value = world * steps_total * cfg.B / (ms / 1e3)
 
+    bad = [i for i, x in enumerate(inst) if int(x.lay.err_word.item()) != 0]
+    if bad:
+        raise RuntimeError(f"device-side checks flagged instances {bad[:8]} "
+                           f"(err words {[int(inst[i].lay.err_word.item()) for i in bad[:8]]})")
+
     # ---- end to end through the public call: pinned host inputs in, output out
     host = {k: getattr(inst[0], k).cpu().pin_memory() for k in ["q", "k", "v", "kidx", "qidx", "w", "lam"]}
     out_h = torch.empty_like(inst[0].out, device="cpu").pin_memory()

@@ -4,6 +4,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+#include <unordered_map>
+
 #include "lisa_internal.h"
 
 namespace {
@@ -129,6 +132,32 @@ void set_select_smem(lisa::RowsParams &r, int n_max) {
 }
 
 }  // namespace
+
+namespace lisa {
+
+cudaError_t prepare_kernel_ptr(const void *fn, int dyn_smem) {
+  static std::mutex mu;
+  static std::unordered_map<const void *, int> done[64];   // per device: kernel -> dynamic smem limit set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto &m = done[dev & 63];
+  auto it = m.find(fn);
+  if (it == m.end()) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    it = m.emplace(fn, 0).first;
+  }
+  if (dyn_smem > it->second) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+    if (e != cudaSuccess) return e;
+    it->second = dyn_smem;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace lisa
 
 extern "C" {
 

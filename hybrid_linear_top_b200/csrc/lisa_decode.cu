@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(NT) decode_select_kernel(DecodeParams p) {
     cand = s_dyn + p.smem_keys_cap;
   }
   int *out = p.idx + (size_t)bg * p.M;
-  block_topm<NT>(keys, n, p.M, out, sm, cand, p.cand_cap);
+  if (!block_topm<NT>(keys, n, p.M, out, sm, cand, p.cand_cap) && threadIdx.x == 0)
+    set_err(p.err_word, LISA_DEVERR_CHECK);
   if (p.idx_out) {
     __syncthreads();
     for (int i = threadIdx.x; i < p.M; i += NT) p.idx_out[(size_t)bg * p.M + i] = __ldcg(out + i);
@@ -264,7 +265,14 @@ __global__ void __launch_bounds__(256) decode_attend_kernel(DecodeParams p) {
   if (t < 0 || t >= p.L_max) return;
   const int G = p.G;
 
-  if (tid < kRows) s_idx[tid] = __ldcg(p.idx + (size_t)bg * p.M + sp * kRows + tid);
+  if (tid < kRows) {
+    int s = __ldcg(p.idx + (size_t)bg * p.M + sp * kRows + tid);
+    if (s < -1 || s > t) {
+      set_err(p.err_word, LISA_DEVERR_CHECK);
+      s = -1;
+    }
+    s_idx[tid] = s;
+  }
   for (int i = tid; i < G * D; i += blockDim.x) {
     const int hh = i / D, dd = i % D;
     s_q[hh][dd] = Dt<T>::to_f(reinterpret_cast<const T *>(p.q)[((size_t)b * p.Hq + g * G + hh) * D + dd]);
@@ -372,11 +380,13 @@ static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t st) {
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
 
   {
+    cudaError_t e = prepare_kernel(decode_score_state_kernel<T, D, DI>);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.n_score_blocks + p.n_state_blocks);
     cfg.blockDim = dim3(256);
     cfg.stream = st;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_score_state_kernel<T, D, DI>, p);
+    e = cudaLaunchKernelEx(&cfg, decode_score_state_kernel<T, D, DI>, p);
     if (e != cudaSuccess) return e;
   }
   {
@@ -388,20 +398,21 @@ static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaFuncSetAttribute(decode_select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         p.select_smem);
+    cudaError_t e = prepare_kernel(decode_select_kernel<NT>, (int)p.select_smem);
     if (e != cudaSuccess) return e;
     e = cudaLaunchKernelEx(&cfg, decode_select_kernel<NT>, p);
     if (e != cudaSuccess) return e;
   }
   {
+    cudaError_t e = prepare_kernel(decode_attend_kernel<T, D>);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.B * p.Hkv * (p.M / kAttnRows));
     cfg.blockDim = dim3(256);
     cfg.stream = st;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_attend_kernel<T, D>, p);
+    e = cudaLaunchKernelEx(&cfg, decode_attend_kernel<T, D>, p);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -212,10 +212,11 @@ static cudaError_t prefill_linear_t(const RowsParams &p, cudaStream_t st) {
   const int nc = (p.T + C - 1) / C;
   const size_t smem1 = 2 * C * D * sizeof(float);
   const size_t smem3 = (3 * C * D + C * (C + 1) + 16 * D) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(lin_dS_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  cudaError_t e = prepare_kernel(lin_dS_kernel<T, D>, (int)smem1);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(lin_out_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
-  if (e != cudaSuccess) return e;
+  if ((e = prepare_kernel(lin_out_kernel<T, D>, (int)smem3)) != cudaSuccess) return e;
+  if ((e = prepare_kernel(lin_prefix_kernel<D>)) != cudaSuccess) return e;
+  if ((e = prepare_kernel(lin_state_kernel<D>)) != cudaSuccess) return e;
   lin_dS_kernel<T, D><<<dim3(nc, p.B * p.Hkv), 256, smem1, st>>>(p);
   lin_prefix_kernel<D><<<dim3(D * D / 256, p.B * p.Hkv), 256, 0, st>>>(p);
   lin_out_kernel<T, D><<<dim3(nc, p.Hq, p.B), 256, smem3, st>>>(p);

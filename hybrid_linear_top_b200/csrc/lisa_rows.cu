@@ -44,10 +44,15 @@ __global__ void append_kernel(RowsParams p) {
 
 cudaError_t launch_append(const RowsParams &p, int dtype, cudaStream_t st) {
   dim3 grid(p.T, p.B * p.Hkv);
-  if (dtype == LISA_BF16)
+  if (dtype == LISA_BF16) {
+    cudaError_t e = prepare_kernel(append_kernel<__nv_bfloat16>);
+    if (e != cudaSuccess) return e;
     append_kernel<__nv_bfloat16><<<grid, 64, 0, st>>>(p);
-  else
+  } else {
+    cudaError_t e = prepare_kernel(append_kernel<float>);
+    if (e != cudaSuccess) return e;
     append_kernel<float><<<grid, 64, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -164,14 +169,16 @@ __global__ void __launch_bounds__(NT) rows_select_kernel(RowsParams p, int tau0,
     cand = s_dyn + p.smem_keys_cap;
   }
   int *out = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M;
-  block_topm<NT>(keys, n, p.M, out, sm, cand, p.cand_cap);
+  if (!block_topm<NT>(keys, n, p.M, out, sm, cand, p.cand_cap) && threadIdx.x == 0)
+    set_err(p.err_word, LISA_DEVERR_CHECK);
 }
 
 template <typename T, int DI>
 static cudaError_t rows_topk_t(const RowsParams &p, cudaStream_t st, int key_limit) {
   constexpr int NT = 256;
-  cudaError_t e = cudaFuncSetAttribute(rows_select_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)p.select_smem);
+  cudaError_t e = prepare_kernel(rows_select_kernel<NT>, (int)p.select_smem);
+  if (e != cudaSuccess) return e;
+  e = prepare_kernel(rows_score_kernel<T, DI>);
   if (e != cudaSuccess) return e;
   for (int tau0 = 0; tau0 < p.T; tau0 += p.row_chunk) {
     const int rows = min(p.row_chunk, p.T - tau0);
@@ -233,7 +240,14 @@ __global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
   constexpr int kSlices = D * (int)sizeof(T) / 16;
   for (int tile = 0; tile < p.M / kRows; ++tile) {
     __syncthreads();
-    if (tid < kRows) s_idx[tid] = idx[tile * kRows + tid];
+    if (tid < kRows) {
+      int s = idx[tile * kRows + tid];
+      if (s < -1 || s > p.pos[b] + tau) {
+        set_err(p.err_word, LISA_DEVERR_CHECK);
+        s = -1;
+      }
+      s_idx[tid] = s;
+    }
     __syncthreads();
     if (s_idx[0] < 0) break;
     for (int i = tid; i < kRows * kSlices; i += 256) {
@@ -301,12 +315,23 @@ __global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
 
 cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st) {
   dim3 grid(p.T, p.B * p.Hkv);
+  cudaError_t e;
   if (dtype == LISA_BF16) {
-    if (p.D == 128) prefill_attend_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(p);
-    else prefill_attend_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(p);
+    if (p.D == 128) {
+      if ((e = prepare_kernel(prefill_attend_kernel<__nv_bfloat16, 128>)) != cudaSuccess) return e;
+      prefill_attend_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(p);
+    } else {
+      if ((e = prepare_kernel(prefill_attend_kernel<__nv_bfloat16, 64>)) != cudaSuccess) return e;
+      prefill_attend_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(p);
+    }
   } else {
-    if (p.D == 128) prefill_attend_kernel<float, 128><<<grid, 256, 0, st>>>(p);
-    else prefill_attend_kernel<float, 64><<<grid, 256, 0, st>>>(p);
+    if (p.D == 128) {
+      if ((e = prepare_kernel(prefill_attend_kernel<float, 128>)) != cudaSuccess) return e;
+      prefill_attend_kernel<float, 128><<<grid, 256, 0, st>>>(p);
+    } else {
+      if ((e = prepare_kernel(prefill_attend_kernel<float, 64>)) != cudaSuccess) return e;
+      prefill_attend_kernel<float, 64><<<grid, 256, 0, st>>>(p);
+    }
   }
   return cudaGetLastError();
 }

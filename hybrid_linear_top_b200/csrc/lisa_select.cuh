@@ -71,8 +71,9 @@ __device__ __forceinline__ void find_bucket(TopmShared &sm, uint32_t rem) {
 // keys: n order keys (shared or global memory), position i has key keys[i].
 // cand: shared scratch of cand_cap uint32.  out: M int32 (global).
 // Must be called by all NT threads of the block.
+// Returns false (and writes -1 everywhere) if an internal check failed.
 template <int NT>
-__device__ void block_topm(const uint32_t *keys, int n, int M, int *out, TopmShared &sm, uint32_t *cand,
+__device__ bool block_topm(const uint32_t *keys, int n, int M, int *out, TopmShared &sm, uint32_t *cand,
                            int cand_cap) {
   constexpr int NW = NT / 32;
   const int tid = threadIdx.x;
@@ -81,7 +82,7 @@ __device__ void block_topm(const uint32_t *keys, int n, int M, int *out, TopmSha
 
   if (n <= M) {
     for (int i = tid; i < M; i += NT) out[i] = i < n ? i : -1;
-    return;
+    return true;
   }
 
   uint32_t prefix = 0, pmask = 0, rem = (uint32_t)M;
@@ -116,10 +117,15 @@ __device__ void block_topm(const uint32_t *keys, int n, int M, int *out, TopmSha
         hist_add(sm.hist, act, (u >> shift) & 255u);
       }
     }
+    if (tid == 0) sm.bc_digit = 0xFFFFFFFFu;
     __syncthreads();
     find_bucket(sm, rem);
     __syncthreads();
     const uint32_t dig = sm.bc_digit;
+    if (dig > 255u) {  // counts inconsistent: cannot happen for a valid key array
+      for (int i = tid; i < M; i += NT) out[i] = -1;
+      return false;
+    }
     const uint32_t above = sm.bc_above;
     const uint32_t in_bucket = sm.hist[dig];
     rem -= above;
@@ -190,6 +196,7 @@ __device__ void block_topm(const uint32_t *keys, int n, int M, int *out, TopmSha
   g = sm.wg[warp];
   e = sm.we[warp];
   const unsigned lt = (1u << lane) - 1u;
+  bool bad = false;
   for (int base = c0; base < c1; base += 32) {
     const int i = base + lane;
     const uint32_t u = i < c1 ? keys[i] : 0u;
@@ -200,11 +207,13 @@ __device__ void block_topm(const uint32_t *keys, int n, int M, int *out, TopmSha
     const bool eq = (be >> lane) & 1u;
     if (gt || (eq && pe < need_eq)) {
       const uint32_t o = g + __popc(bg & lt) + min(pe, need_eq);
-      out[o] = i;
+      if (o < (uint32_t)M) out[o] = i;
+      else bad = true;
     }
     g += __popc(bg);
     e += __popc(be);
   }
+  return !__syncthreads_or(bad);
 }
 
 }  // namespace lisa

@@ -24,6 +24,7 @@ LISA_BF16 = 0
 LISA_FP32 = 1
 LISA_DEVERR_POS = 1
 LISA_DEVERR_TIMEOUT = 2
+LISA_DEVERR_CHECK = 4
 LISA_OP_DECODE = 0
 LISA_OP_PREFILL = 1
 LISA_OP_INDEXER_TOPK = 2

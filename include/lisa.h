@@ -70,6 +70,8 @@ typedef enum { LISA_BF16 = 0, LISA_FP32 = 1 } lisa_dtype;
 /* Bits a kernel ORs into *err_word. */
 #define LISA_DEVERR_POS      1   /* pos[b] < 0, or pos[b] + T > L_max: sequence b skipped */
 #define LISA_DEVERR_TIMEOUT  2   /* a bounded wait on an asynchronous copy gave up */
+#define LISA_DEVERR_CHECK    4   /* an internal consistency check failed (a selected index out of
+                                    range, or no threshold bucket); the access was skipped */
 
 /* Operation codes for lisa_workspace_bytes(). */
 #define LISA_OP_DECODE       0
