@@ -144,11 +144,7 @@ cudaError_t prepare_kernel_ptr(const void *fn, int dyn_smem) {
   std::lock_guard<std::mutex> lock(mu);
   auto &m = done[dev & 63];
   auto it = m.find(fn);
-  if (it == m.end()) {
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    it = m.emplace(fn, 0).first;
-  }
+  if (it == m.end()) it = m.emplace(fn, 0).first;
   if (dyn_smem > it->second) {
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
     if (e != cudaSuccess) return e;

@@ -15,12 +15,8 @@ constexpr int kAttnRows = 32;   // selected rows per attention CTA / tile
 constexpr int kLinChunk = 64;   // chunk length of the chunked linear attention
 constexpr int kRowTile = 64;    // query rows per indexer score tile (row path)
 
-// Requests the full shared-memory carveout for kernel `fn` (and raises its
-// dynamic shared-memory limit to `dyn_smem`) once per device.  Every kernel of
-// the library uses the same carveout: on B200 a CTA's shared memory was
-// observed to change under it when programmatic dependent launch co-scheduled
-// kernels whose carveouts differed; with one common carveout that no longer
-// happens.
+// Raises the dynamic shared-memory limit of kernel `fn` to `dyn_smem` (once per
+// device and size; host-side bookkeeping only).
 cudaError_t prepare_kernel_ptr(const void *fn, int dyn_smem);
 
 template <typename F>

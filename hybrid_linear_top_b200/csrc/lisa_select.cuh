@@ -92,6 +92,8 @@ __device__ bool block_topm(const uint32_t *keys, int n, int M, int *out, TopmSha
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
+    // every thread has read the previous pass's bucket before it is cleared
+    __syncthreads();
     for (int i = tid; i < 256; i += NT) sm.hist[i] = 0;
     __syncthreads();
     if (use_cand) {

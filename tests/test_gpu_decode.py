@@ -185,3 +185,46 @@ def test_indexer_topk_single_token():
         sc = oracle.indexer_scores(step.qidx[b, 0].astype(np.float64), step.w[b, 0].astype(np.float64), keys)
         for g in range(cfg.Hkv):
             check_set(idx_g[b, 0, g], sc[g], cfg.M, t, where=f"b={b} g={g}")
+
+
+def test_decode_graph_replays_are_stable():
+    """Back-to-back decode steps of independent layers, captured in one CUDA
+    graph and replayed many times: every replay must select the same sets and
+    no device-side check may fire (guards the barriers of the radix select and
+    the ordering of the chained launches)."""
+    cfg = get_config("decode_1p5b_16k")
+    n_inst = 12
+    lays, steps = [], []
+    for i in range(n_inst):
+        rng = make_rng(cfg.seed, 100 + i)
+        lay_np = gen_layer(cfg, rng, cfg.L - 1)
+        st = gen_step(cfg, rng, 1)
+        lay = make_layer(L, cfg, cfg.L_max, lay_np, n_rows=cfg.L - 1, poison=False)
+        lay.pos.fill_(cfg.L - 1)
+        lays.append(lay)
+        steps.append(step_tensors(st, cfg, tau=0))
+    ws = L.alloc_workspace(lays[0], 1, L.LISA_OP_DECODE)
+    outs = [torch.empty(1, cfg.Hq, cfg.d, dtype=torch.bfloat16, device="cuda") for _ in range(n_inst)]
+    idxs = [torch.empty(1, cfg.Hkv, cfg.M, dtype=torch.int32, device="cuda") for _ in range(n_inst)]
+    s = torch.cuda.Stream()
+
+    def run_all():
+        for lay, x, o, ix in zip(lays, steps, outs, idxs):
+            L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, o, ix, ws,
+                               s)
+
+    with torch.cuda.stream(s):
+        run_all()
+    s.synchronize()
+    ref = [ix.clone() for ix in idxs]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run_all()
+    for rep in range(150):
+        with torch.cuda.stream(s):
+            g.replay()
+        if rep % 10 == 9:
+            torch.cuda.synchronize()
+            assert all(int(l.err_word.item()) == 0 for l in lays), f"replay {rep}"
+            assert all(torch.equal(a, b) for a, b in zip(idxs, ref)), f"replay {rep}"
+    torch.cuda.synchronize()
