@@ -155,6 +155,39 @@ cudaError_t prepare_kernel_ptr(const void *fn, int dyn_smem) {
 
 }  // namespace lisa
 
+// ---------------------------------------------------------------- fixed scratch
+// Scratch of lisa_indexer_topk_noalloc(): a fixed array in device memory that
+// every GPU loading this library holds until the process exits.  Host code
+// must not pass `g_noalloc_scratch` itself to a kernel (on the host that name
+// is only a stand-in); it asks the runtime for the array's device address once
+// per device, with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LISA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call for that device, cached afterwards).
+lisa_status noalloc_scratch(void **addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LISA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return LISA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *lisa_version(void) { return "lisa-b200 0.1 (sm_100a)"; }
@@ -311,6 +344,38 @@ lisa_status lisa_prefill(const lisa_layer *L, int T, const void *q, const void *
   if (e != cudaSuccess) return cuda_fail(e, "prefill indexer");
   e = lisa::launch_prefill_attend(r, L->dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "prefill attend");
+  return ok();
+}
+
+lisa_status lisa_indexer_topk_noalloc(const lisa_layer *L, const void *qidx, const float *w, int T, int *idx_out,
+                                      void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(idx_out, "idx_out"))) return s;
+  // one order key per (sequence, KV head, cached position) for every query row of a pass
+  const size_t per_row = (size_t)L->B * L->Hkv * round4(L->L_max) * 4;
+  if (per_row > (size_t)LISA_NOALLOC_SCRATCH_BYTES)
+    return fail(LISA_ERR_UNSUPPORTED,
+                "B*Hkv*L_max needs %zu bytes of scratch per query row; the fixed scratch holds %u bytes",
+                per_row, (unsigned)LISA_NOALLOC_SCRATCH_BYTES);
+  size_t rows = (size_t)LISA_NOALLOC_SCRATCH_BYTES / per_row;
+  if (rows > (size_t)kRowChunk) rows = kRowChunk;
+  if (rows > (size_t)T) rows = T;
+  void *scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch))) return s;
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.qidx = qidx; r.w = w; r.idx = idx_out;
+  r.keys = static_cast<uint32_t *>(scratch);   // every slot read is written earlier in the same call
+  r.row_chunk = (int)rows;
+  r.L_keys = round4(L->L_max);
+  set_select_smem(r, L->L_max);
+  cudaError_t e = lisa::launch_rows_topk(r, L->dtype, (cudaStream_t)stream, L->L_max);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc");
   return ok();
 }
 

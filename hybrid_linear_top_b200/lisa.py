@@ -33,6 +33,7 @@ EXPORTED = [
     "lisa_workspace_bytes",
     "lisa_append_cache",
     "lisa_indexer_topk",
+    "lisa_indexer_topk_noalloc",
     "lisa_decode_step",
     "lisa_prefill",
     "lisa_status_str",
@@ -69,6 +70,8 @@ def _load():
     lib.lisa_append_cache.restype = ctypes.c_int
     lib.lisa_indexer_topk.argtypes = [L, P, P, ctypes.c_int, P, P, ctypes.c_size_t, P]
     lib.lisa_indexer_topk.restype = ctypes.c_int
+    lib.lisa_indexer_topk_noalloc.argtypes = [L, P, P, ctypes.c_int, P, P]
+    lib.lisa_indexer_topk_noalloc.restype = ctypes.c_int
     lib.lisa_decode_step.argtypes = [L, P, P, P, P, P, P, P, ctypes.c_int, P, P, P, ctypes.c_size_t, P]
     lib.lisa_decode_step.restype = ctypes.c_int
     lib.lisa_prefill.argtypes = [L, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -179,6 +182,15 @@ def lisa_indexer_topk(layer, qidx, w, T, idx_out, workspace, stream=None):
     c = layer.c_struct()
     _check(_lib.lisa_indexer_topk(ctypes.byref(c), _ptr(qidx), _ptr(w), int(T), _ptr(idx_out), _ptr(workspace),
                                   workspace.numel() if workspace is not None else 0, _stream(stream)))
+
+
+def lisa_indexer_topk_noalloc(layer, qidx, w, T, idx_out, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_indexer_topk_noalloc(ctypes.byref(c), _ptr(qidx), _ptr(w), int(T), _ptr(idx_out),
+                                          _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def lisa_decode_step(layer, q, k, v, kidx, qidx, w, gate_logit, fuse_append, out, idx_out, workspace,

@@ -161,6 +161,32 @@ LISA_API lisa_status lisa_prefill(const lisa_layer *layer, int T, const void *q,
                          const float *gate_logit, void *out, int *idx_out, void *workspace,
                          size_t ws_bytes, void *stream);
 
+/*
+ * lisa_indexer_topk without a workspace argument, for callers that cannot
+ * allocate device memory: for example a plugin running inside a host program
+ * that owns all device memory and gives the plugin no allocator, or code that
+ * may not call cudaMalloc because it can synchronise the device.  The method's
+ * pages have no counterpart for this call; it is a convenience of this library.
+ *
+ * Arguments, results and checks are those of lisa_indexer_topk.  The scratch
+ * comes from one fixed array of LISA_NOALLOC_SCRATCH_BYTES in device memory
+ * that every GPU which loads the library holds until the process exits.  A
+ * call needs B * Hkv * L_max * 4 bytes (L_max rounded up to a multiple of 4)
+ * of it per query row: larger sizes return LISA_ERR_UNSUPPORTED before
+ * anything is launched, and smaller ones process the T rows in as many passes
+ * as the array requires.  The call allocates and frees nothing.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents (nothing in it needs to start at zero: every entry a call reads it
+ * has written first).  Calls that overlap on the GPU, from any stream or
+ * thread, race on the array and must be avoided.
+ */
+#define LISA_NOALLOC_SCRATCH_BYTES (16u << 20)
+LISA_API lisa_status lisa_indexer_topk_noalloc(const lisa_layer *layer, const void *qidx, const float *w,
+                                               int T, int *idx_out, void *stream);
+
 /* Human-readable name of a status. */
 LISA_API const char *lisa_status_str(lisa_status s);
 

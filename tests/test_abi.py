@@ -131,3 +131,14 @@ def test_workspace_sizes():
     assert L.lisa_workspace_bytes(c, 4, L.LISA_OP_INDEXER_TOPK) > 0
     assert L.lisa_workspace_bytes(_layer(d=96), 1, L.LISA_OP_DECODE) == 0
     assert L.lisa_workspace_bytes(c, 1, 42) == 0
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    lib = L.lib()
+    # 2 KV heads x 4M positions x 4 bytes = 32 MiB per query row > the fixed scratch
+    c = _layer(L_max=1 << 22)
+    st = lib.lisa_indexer_topk_noalloc(ctypes.byref(c), FAKE, FAKE, 1, FAKE, None)
+    assert st == L.LISA_ERR_UNSUPPORTED
+    assert "scratch" in L.last_error_msg()
+    assert lib.lisa_indexer_topk_noalloc(ctypes.byref(c), FAKE, FAKE, 0, FAKE, None) == L.LISA_OK
+    assert lib.lisa_indexer_topk_noalloc(ctypes.byref(_layer()), FAKE, None, 1, FAKE, None) == L.LISA_ERR_INVALID_ARG
