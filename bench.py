@@ -339,12 +339,12 @@ def run_lisa(args, rank, world):
                    "l2": "inputs larger than L2: rotation over instances touching "
                          f"{R * step_bytes / 2 ** 20:.0f} MiB (L2 {l2 / 2 ** 20:.0f} MiB)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "decode step (score_state + select + attend)",
+        "roofline": {"bound": "hbm", "kernel": "decode_cluster_kernel (whole decode step)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind, "algorithmic_bytes_per_launch": step_bytes, "traffic": None},
         "clocks": clocks,
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * steps_total,
+        "gpu_launches": steps_total,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

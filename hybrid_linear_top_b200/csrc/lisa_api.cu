@@ -40,6 +40,7 @@ constexpr int kDecodeKeysCap = 32768;   // order keys staged in shared memory (1
 constexpr int kRowsKeysCap = 16384;     // same, for the 256-thread row select
 constexpr int kCandCap = 4096;          // threshold-bucket candidates kept in shared memory
 constexpr int kRowChunk = 1024;         // query rows scored per pass on the row path
+constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory a CTA may use on sm_100
 
 // Validates the geometry; returns LISA_OK or the failure status.
 lisa_status check_layer(const lisa_layer *L) {
@@ -76,22 +77,6 @@ lisa_status check_caches(const lisa_layer *L) {
 }
 
 // ---------------------------------------------------------------- workspace plans
-struct DecodePlan {
-  size_t keys, idx, olin, partials, counters, total;
-};
-DecodePlan decode_plan(const lisa_layer *L) {
-  DecodePlan p;
-  const size_t BH = (size_t)L->B * L->Hkv;
-  size_t off = 0;
-  p.keys = off; off += round256(BH * round4(L->L_max) * 4);
-  p.idx = off; off += round256(BH * L->M * 4);
-  p.olin = off; off += round256((size_t)L->B * L->Hq * L->d * 4);
-  p.partials = off; off += round256(BH * (L->M / lisa::kAttnRows) * (L->Hq / L->Hkv) * (L->d + 2) * 4);
-  p.counters = off; off += round256(BH * 4);
-  p.total = off;
-  return p;
-}
-
 struct RowsPlan {
   int row_chunk, L_keys;
   size_t keys, idx, olin, dS, Ptot, total;
@@ -207,7 +192,7 @@ const char *lisa_status_str(lisa_status s) {
 
 size_t lisa_workspace_bytes(const lisa_layer *layer, int T, int op) {
   if (check_layer(layer) != LISA_OK || T < 0) return 0;
-  if (op == LISA_OP_DECODE) return decode_plan(layer).total;
+  if (op == LISA_OP_DECODE) return 0;   // the decode step keeps its intermediates on chip
   if (op == LISA_OP_PREFILL) return T ? rows_plan(layer, T, true).total : 0;
   if (op == LISA_OP_INDEXER_TOPK) return T ? rows_plan(layer, T, false).total : 0;
   return 0;
@@ -268,10 +253,11 @@ lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, 
       (s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(gate_logit, "gate_logit")) ||
       (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)))
     return s;
-  const DecodePlan plan = decode_plan(L);
-  if (!workspace || ws_bytes < plan.total)
-    return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
-  if ((s = check_ptr(workspace, "workspace"))) return s;
+  (void)workspace;
+  (void)ws_bytes;
+  const int esz = L->dtype == LISA_BF16 ? 2 : 4;
+  if (lisa::decode_smem_bytes(L->L_max, L->M, L->Hq / L->Hkv, L->d, L->dI, esz, 8) > kMaxSmem)
+    return fail(LISA_ERR_UNSUPPORTED, "L_max=%d needs more shared memory per CTA than a B200 SM has", L->L_max);
 
   lisa::DecodeParams p;
   memset(&p, 0, sizeof(p));
@@ -282,22 +268,6 @@ lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, 
   p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;
   p.q = q; p.k = k; p.v = v; p.kidx = kidx; p.qidx = qidx; p.w = w; p.gate = gate_logit;
   p.out = out; p.idx_out = idx_out;
-  char *ws = static_cast<char *>(workspace);
-  p.keys = reinterpret_cast<uint32_t *>(ws + plan.keys);
-  p.keys_stride = round4(L->L_max);
-  p.idx = reinterpret_cast<int *>(ws + plan.idx);
-  p.olin = reinterpret_cast<float *>(ws + plan.olin);
-  p.partials = reinterpret_cast<float *>(ws + plan.partials);
-  p.counters = reinterpret_cast<unsigned *>(ws + plan.counters);
-  p.n_chunks = (L->L_max + 127) / 128;
-  p.n_score_blocks = L->B * L->Hkv * p.n_chunks;
-  p.n_state_blocks = L->B * L->Hq * (L->d / 32);
-  const int cap = L->L_max < kDecodeKeysCap ? L->L_max : kDecodeKeysCap;
-  p.smem_keys_cap = (cap + 3) & ~3;
-  p.cand_cap = kCandCap;
-  p.select_smem = (size_t)(p.smem_keys_cap + p.cand_cap) * 4;
-  if ((long long)p.n_score_blocks + p.n_state_blocks > 0x7fffffffLL)
-    return fail(LISA_ERR_UNSUPPORTED, "grid too large");
   cudaError_t e = lisa::launch_decode(p, L->dtype, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode_step");
   return ok();

@@ -1,421 +1,964 @@
-// LISA decode step on sm_100a: three kernels chained with programmatic
-// dependent launch.
+// LISA decode step on sm_100a: one kernel, one thread-block cluster of NC CTAs
+// (NC = 16, or 8 where 16 cannot be scheduled) per (sequence b, KV head g).
 //
-//   1. score_state: streams the indexer-key cache with 1-D TMA bulk copies into
-//      shared memory and writes one order key per (b, g, s); in the same grid,
-//      extra CTAs do the linear-state read-modify-write S <- S + k^T v and
-//      o_lin = q S, and the CTA owning the new row appends it to the caches.
-//   2. select: one CTA per (b, g) turns the order keys into the top-M set.
-//   3. attend: split-M sparse attention over the gathered K/V rows, merged by
-//      the last CTA of each (b, g), which also applies the gate.
+// Method: arXiv 2607.19358 (LISA).  Abstract: a Lightning Indexer keeps the
+// top-M tokens of the context for a sparse softmax attention, a linear
+// attention runs beside it and a gate fuses the two.  gptget.net digest,
+// method section: phi = identity with a state matrix S_t; indexer = ReLU dot
+// products of small query/key projections.  Exact formulas: include/lisa.h.
 //
-// Method: arXiv 2607.19358 (LISA), abstract and the gptget.net digest's method
-// section; exact formulas as stated in lisa.h.
+// Work of one cluster (CTA rank r of NC):
+//   1. stream its contiguous slice of the (b, g) indexer-key cache through a
+//      4-stage TMA ring and score every key, keeping 32-bit order keys in
+//      shared memory.  bf16: 2-D tiled TMA with a 64/128-byte swizzle and warp
+//      tensor-core MMAs (keys x indexer heads); fp32: 1-D bulk copies and one
+//      thread per key on the CUDA cores.  Meanwhile the columns
+//      [r*d/NC, (r+1)*d/NC) of the linear state of the G query heads are
+//      loaded, updated (S += k^T v) and read out (o_lin = q S);
+//   2. exact top-M: every CTA takes the smallest of kl group maxima of its
+//      keys; if enough CTAs hold kl keys, the smallest of those values over
+//      the cluster is <= the M-th largest key, so only keys at or above it go
+//      to CTA 0, which selects exactly among them and emits the ascending
+//      index list.  When too many keys pass, a cluster-wide radix select
+//      (histograms summed over distributed shared memory) runs instead;
+//   3. gather M/NC of the selected K/V rows, partial softmax for the G heads;
+//   4. merge the NC partials for its own column slice, apply the gate, store.
+// Only cluster barriers synchronise; nothing leaves the cluster but the
+// outputs, the state and the appended cache row.
+#include <cooperative_groups.h>
+#include <string.h>
+
 #include "lisa_internal.h"
-#include "lisa_select.cuh"
+#include "lisa_common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace lisa {
 
-// ============================================================ kernel 1
+constexpr int kDecThreads = 256;
+constexpr int kStages = 4;
+constexpr int kStageBytes = 32768;
+constexpr int kCandCap = 4096;   // candidate (key, position) pairs CTA 0 can hold
+
 template <typename T, int DI>
-struct ScoreCfg {
-  static constexpr int kRowBytes = DI * Dt<T>::kBytes;
-  static constexpr int kLanesPerKey = kRowBytes / 16;          // 16-byte slices per key row
-  static constexpr int kVec = 16 / Dt<T>::kBytes;              // elements per slice
-  static constexpr int kThreads = 256;
-  static constexpr int kKeysPerIter = kThreads / kLanesPerKey;
-  static constexpr int kChunk = 128;                           // keys per CTA
+struct ScoreGeom {
+  static constexpr int RB = DI * (int)sizeof(T);                              // key row bytes
+  static constexpr int SUB = (kStageBytes / RB) < 256 ? kStageBytes / RB : 256; // keys per ring stage
+  static constexpr bool kMma = sizeof(T) == 2;                                // bf16: swizzled tiles + MMA
 };
 
-template <typename T, int D, int DI>
-__global__ void __launch_bounds__(256) decode_score_state_kernel(DecodeParams p) {
-  using C = ScoreCfg<T, DI>;
-  __shared__ __align__(128) unsigned char s_rows[C::kChunk * C::kRowBytes];
-  __shared__ __align__(8) uint64_t s_bar;
-  __shared__ float s_red[256 / 8][33];
+struct DecLayout {
+  int region0, cand_key, cand_pos, gtb, eqb;
+  int keys, hist, tot, misc, sel, qs, qi, ks, vs, part, pml, olin, logit, sidx, bars, total;
+};
 
-  // Let the select kernel get scheduled as soon as every CTA of this grid runs.
-  grid_dep_launch();
+__host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 
-  const int tid = threadIdx.x;
-  if (blockIdx.x == 0)
-    for (int i = tid; i < p.B * p.Hkv; i += blockDim.x) p.counters[i] = 0;
+// Byte offsets of the dynamic shared-memory carve-up, relative to a
+// 1024-byte aligned base (host and device agree; `total` includes the slack
+// needed to align the base).  region0 holds, one after the other in time: the
+// TMA ring (scoring), the candidate lists and position bitmaps (selection, in
+// CTA 0), and the gathered K / V rows (attention).
+__host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, int G, int D, int DI, int esize,
+                                                int NC) {
+  DecLayout L;
+  const int rpc = M / NC;
+  const int kv = 2 * rpc * (D * esize + 16);
+  const int nw = (L_max + 31) / 32;
+  const int ring = kStages * kStageBytes;
+  const int sel_bytes = 8 * kCandCap + 2 * align16(nw * 4);
+  int r0 = ring > kv ? ring : kv;
+  r0 = r0 > sel_bytes ? r0 : sel_bytes;
+  int off = 0;
+  L.region0 = off; off += align16(r0);
+  L.cand_key = L.region0;
+  L.cand_pos = L.region0 + 4 * kCandCap;
+  L.gtb = L.region0 + 8 * kCandCap;
+  L.eqb = L.gtb + align16(nw * 4);
+  L.keys = off; off += align16(kpc_max * 4);
+  L.hist = off; off += 8 * 256 * 4;
+  L.tot = off; off += 256 * 4;
+  L.misc = off; off += 64 * 4;
+  L.sel = off; off += align16(M * 4);
+  L.qs = off; off += align16(G * D * 4);
+  L.qi = off; off += align16(kMaxR * DI * 4 + kMaxR * 4);
+  L.ks = off; off += align16(D * 4);
+  L.vs = off; off += align16(D * 4);
+  L.part = off; off += align16(G * D * 4);
+  L.pml = off; off += align16(2 * G * 4);
+  L.olin = off; off += align16(G * (D / NC) * 4);
+  {
+    const int a = G * rpc * 4, bred = 8 * 8 * (D / NC) * 4;   // logits, or the o_lin reduction scratch
+    L.logit = off; off += align16(a > bred ? a : bred);
+  }
+  L.sidx = off; off += align16(rpc * 4);
+  L.bars = off; off += kStages * 8;
+  L.total = align16(off) + 1024;
+  return L;
+}
 
-  if ((int)blockIdx.x < p.n_score_blocks) {
-    // -------------------------------------------------- indexer score
-    const int chunks = p.n_chunks;
-    const int c = blockIdx.x % chunks;
-    const int bg = blockIdx.x / chunks;
-    const int g = bg % p.Hkv;
-    const int b = bg / p.Hkv;
-    const int t = p.pos[b];
-    if (t < 0 || t >= p.L_max) {
-      if (c == 0 && tid == 0) set_err(p.err_word, LISA_DEVERR_POS);
-      return;
+// Warp 0 scans 256 bins from the top and finds the one holding the rem-th
+// largest key: misc[0] = bin, misc[1] = keys in higher bins.  Other lanes idle.
+__device__ __forceinline__ void dec_find_bucket(const uint32_t *tot, uint32_t *misc, uint32_t rem) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      c[j] = tot[255 - (8 * lane + j)];
+      sum += c[j];
     }
-    const int s0 = c * C::kChunk;
-    if (s0 > t) return;
-    const int s_end = min(s0 + C::kChunk, t + 1);  // exclusive
-    const int n_cached = min(s_end, t) - s0;       // rows read from the cache
-
-    // append the new token (row t) when this CTA owns it
-    if (p.fuse_append && t >= s0 && t < s0 + C::kChunk) {
-      const size_t row = ((size_t)b * p.Hkv + g) * p.L_max + t;
-      const T *kin = reinterpret_cast<const T *>(p.k) + ((size_t)b * p.Hkv + g) * D;
-      const T *vin = reinterpret_cast<const T *>(p.v) + ((size_t)b * p.Hkv + g) * D;
-      const T *kiin = reinterpret_cast<const T *>(p.kidx) + ((size_t)b * p.Hkv + g) * DI;
-      T *kc = reinterpret_cast<T *>(p.k_cache) + row * D;
-      T *vc = reinterpret_cast<T *>(p.v_cache) + row * D;
-      T *kic = reinterpret_cast<T *>(p.kidx_cache) + row * DI;
-      for (int i = tid; i < D; i += blockDim.x) {
-        kc[i] = kin[i];
-        vc[i] = vin[i];
+    uint32_t inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const uint32_t exc = inc - sum;
+    if (exc < rem && rem <= inc) {
+      uint32_t cum = exc;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (cum + c[j] >= rem) {
+          misc[0] = 255u - (uint32_t)(8 * lane + j);
+          misc[1] = cum;
+          break;
+        }
+        cum += c[j];
       }
-      for (int i = tid; i < DI; i += blockDim.x) kic[i] = kiin[i];
     }
+  }
+}
 
-    const unsigned char *src = reinterpret_cast<const unsigned char *>(p.kidx_cache) +
-                               (((size_t)b * p.Hkv + g) * p.L_max + s0) * C::kRowBytes;
-    if (tid == 0) {
-      mbar_init(&s_bar, 1);
-      fence_mbar_init();
+// CTA-wide: the top 8*passes bits of the k-th largest of keys[0..cnt)
+// (1 <= k <= cnt), lower bits zero -- a lower bound of that key, exact when
+// passes == 4.  Histograms are kept per warp (hw[8][256]) so no warp-level
+// matching is needed.  All kDecThreads threads call it; uses tot[256] and
+// misc[0..1].
+__device__ uint32_t cta_kth_prefix(const uint32_t *keys, int cnt, uint32_t k, int passes, uint32_t *hw,
+                                   uint32_t *tot, uint32_t *misc) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  uint32_t prefix = 0, pmask = 0, rem = k;
+  for (int pass = 0; pass < passes; ++pass) {
+    const int shift = 24 - 8 * pass;
+    __syncthreads();                       // readers of the previous pass are done
+    for (int i = tid; i < 8 * 256; i += kDecThreads) hw[i] = 0;
+    if (tid == 0) misc[0] = 0xFFFFFFFFu;
+    __syncthreads();
+    for (int j = tid; j < cnt; j += kDecThreads) {
+      const uint32_t u = keys[j];
+      if ((u & pmask) == prefix) atomicAdd(&hw[warp * 256 + ((u >> shift) & 255u)], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      const uint32_t bytes = (uint32_t)n_cached * C::kRowBytes;
-      if (bytes) {
-        mbar_arrive_expect_tx(&s_bar, bytes);
-        bulk_g2s(s_rows, src, bytes, &s_bar);
-      } else {
-        mbar_arrive(&s_bar);
-      }
+    {
+      uint32_t s = 0;
+#pragma unroll
+      for (int w8 = 0; w8 < 8; ++w8) s += hw[w8 * 256 + tid];
+      tot[tid] = s;
     }
-    // the new token's indexer key comes from the argument
-    if (t < s_end) {
-      const unsigned char *kin =
-          reinterpret_cast<const unsigned char *>(p.kidx) + ((size_t)b * p.Hkv + g) * C::kRowBytes;
-      for (int i = tid; i < C::kRowBytes / 16; i += blockDim.x)
-        reinterpret_cast<uint4 *>(s_rows + (size_t)(t - s0) * C::kRowBytes)[i] =
-            reinterpret_cast<const uint4 *>(kin)[i];
-    }
+    __syncthreads();
+    dec_find_bucket(tot, misc, rem);
+    __syncthreads();
+    const uint32_t dig = misc[0];
+    if (dig > 255u) break;                 // counts inconsistent (cannot happen); keep the bound found so far
+    rem -= misc[1];
+    prefix |= dig << shift;
+    pmask |= 255u << shift;
+  }
+  __syncthreads();
+  return prefix;
+}
 
-    // indexer queries and weights of the R heads of this KV head -> registers
-    const int part = tid % C::kLanesPerKey;
-    float qv[kMaxR][C::kVec];
-    float wv[kMaxR];
+// CTA-wide exclusive prefix sums of two counters, plus their totals.
+__device__ __forceinline__ void cta_scan2(uint32_t a, uint32_t b, uint32_t &ea, uint32_t &eb, uint32_t &ta,
+                                          uint32_t &tb, uint32_t *misc) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t ia = a, ib = b;
 #pragma unroll
-    for (int r = 0; r < kMaxR; ++r) {
-      wv[r] = 0.f;
-#pragma unroll
-      for (int j = 0; j < C::kVec; ++j) qv[r][j] = 0.f;
-      if (r < p.R) {
-        const int hi = g * p.R + r;
-        const T *qrow = reinterpret_cast<const T *>(p.qidx) + ((size_t)b * p.HI + hi) * DI;
-        uint4 u = *reinterpret_cast<const uint4 *>(qrow + part * C::kVec);
-        Vec16<T>::unpack(u, qv[r]);
-        wv[r] = p.w[(size_t)b * p.HI + hi];
-      }
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += ya;
+      ib += yb;
     }
-    __syncthreads();  // new-token row visible
-    if (!mbar_wait_bounded(&s_bar, 0)) {
-      if (tid == 0) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
-      return;
+  }
+  __syncthreads();
+  if (lane == 31) {
+    misc[32 + warp] = ia;
+    misc[40 + warp] = ib;
+  }
+  __syncthreads();
+  uint32_t wa = 0, wb = 0;
+  ta = 0;
+  tb = 0;
+  for (int w8 = 0; w8 < kDecThreads / 32; ++w8) {
+    if (w8 < warp) {
+      wa += misc[32 + w8];
+      wb += misc[40 + w8];
     }
+    ta += misc[32 + w8];
+    tb += misc[40 + w8];
+  }
+  ea = wa + ia - a;
+  eb = wb + ib - b;
+}
 
-    uint32_t *keys_out = p.keys + ((size_t)b * p.Hkv + g) * p.keys_stride;
-    const int n = s_end - s0;
-    for (int base = 0; base < n; base += C::kKeysPerIter) {
-      const int kk = base + tid / C::kLanesPerKey;
-      float x[C::kVec];
-      if (kk < n) {
-        uint4 u = *reinterpret_cast<const uint4 *>(s_rows + (size_t)kk * C::kRowBytes + part * 16);
-        Vec16<T>::unpack(u, x);
-      } else {
-#pragma unroll
-        for (int j = 0; j < C::kVec; ++j) x[j] = 0.f;
-      }
-      float score = 0.f;
-#pragma unroll
-      for (int r = 0; r < kMaxR; ++r) {
-        if (r < p.R) {
-          float dot = 0.f;
-#pragma unroll
-          for (int j = 0; j < C::kVec; ++j) dot = fmaf(qv[r][j], x[j], dot);
-#pragma unroll
-          for (int o = C::kLanesPerKey / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-          score = fmaf(wv[r], fmaxf(dot, 0.f), score);
-        }
-      }
-      if (part == 0 && kk < n) keys_out[s0 + kk] = score_key(score);
-    }
+template <typename T, int D, int DI, int NC>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    decode_cluster_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  using SG = ScoreGeom<T, DI>;
+  constexpr int RB = SG::RB;                     // indexer-key row bytes
+  constexpr int SUB = SG::SUB;                   // keys per ring stage
+  constexpr int NCH = RB / 16;                   // 16-byte chunks per key row
+  constexpr int VEC = 16 / (int)sizeof(T);       // elements per chunk
+  constexpr int COLS = D / NC;                   // state / output columns of this CTA
+  constexpr int QPR = COLS / 4;                  // float4 per state row slice
+  constexpr int ITER = (D * QPR + kDecThreads - 1) / kDecThreads;
+  constexpr int ROWB = D * (int)sizeof(T);       // K / V row bytes
+  constexpr int RS = ROWB + 16;                  // padded K / V row stride in shared memory
+  constexpr int SL = ROWB / 16;                  // 16-byte slices per K / V row
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int bg = blockIdx.x / NC;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = p.G, M = p.M, R = p.R;
+  const int rpc = M / NC;
+
+  // 1024-byte aligned base: the swizzled TMA tiles depend on address bits 4..9
+  unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC);
+  unsigned char *ring = smem + lay.region0;
+  uint32_t *keys = reinterpret_cast<uint32_t *>(smem + lay.keys);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist);
+  uint32_t *tot = reinterpret_cast<uint32_t *>(smem + lay.tot);
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + lay.misc);
+  int *sel = reinterpret_cast<int *>(smem + lay.sel);
+  float *qs = reinterpret_cast<float *>(smem + lay.qs);
+  float *qis = reinterpret_cast<float *>(smem + lay.qi);   // [R][DI] indexer queries, then [R] weights
+  float *ks = reinterpret_cast<float *>(smem + lay.ks);
+  float *vs = reinterpret_cast<float *>(smem + lay.vs);
+  float *part = reinterpret_cast<float *>(smem + lay.part);
+  float *pml = reinterpret_cast<float *>(smem + lay.pml);
+  float *olin = reinterpret_cast<float *>(smem + lay.olin);
+  float *logit = reinterpret_cast<float *>(smem + lay.logit);
+  int *sidx = reinterpret_cast<int *>(smem + lay.sidx);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
+
+  // Everything read below may have been written by the previous kernel.
+  grid_dep_wait();
+  grid_dep_launch();
+
+  const int t = p.pos[b];
+  if (t < 0 || t >= p.L_max) {  // same value in every CTA of the cluster: all leave together
+    if (rank == 0 && tid == 0) set_err(p.err_word, LISA_DEVERR_POS);
     return;
   }
-
-  // -------------------------------------------------- linear state
-  // CTA = (b, h, 32-column slab); thread = (row group, float4 column)
-  const int sb = blockIdx.x - p.n_score_blocks;
-  constexpr int kSlabs = D / 32;
-  const int slab = sb % kSlabs;
-  const int bh = sb / kSlabs;
-  const int h = bh % p.Hq;
-  const int b = bh / p.Hq;
-  const int t = p.pos[b];
-  if (t < 0 || t >= p.L_max) return;
-  const int g = h / p.G;
-  const int cg = tid & 7;           // float4 column within the slab
-  const int rg = tid >> 3;          // 32 row groups
-  const int j0 = slab * 32 + cg * 4;
-  const T *kin = reinterpret_cast<const T *>(p.k) + ((size_t)b * p.Hkv + g) * D;
-  const T *vin = reinterpret_cast<const T *>(p.v) + ((size_t)b * p.Hkv + g) * D;
-  const T *qin = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + h) * D;
-  float vj[4];
-#pragma unroll
-  for (int c4 = 0; c4 < 4; ++c4) vj[c4] = Dt<T>::to_f(vin[j0 + c4]);
-  float* S = p.state + ((size_t)b * p.Hq + h) * D * D;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  float4 sv[D / 32];
-#pragma unroll
-  for (int it = 0; it < D / 32; ++it) {
-    const int i = rg + 32 * it;
-    sv[it] = *reinterpret_cast<const float4 *>(S + (size_t)i * D + j0);
-  }
-#pragma unroll
-  for (int it = 0; it < D / 32; ++it) {
-    const int i = rg + 32 * it;
-    const float ki = Dt<T>::to_f(kin[i]);
-    const float qi = Dt<T>::to_f(qin[i]);
-    float4 s = sv[it];
-    s.x = fmaf(ki, vj[0], s.x);
-    s.y = fmaf(ki, vj[1], s.y);
-    s.z = fmaf(ki, vj[2], s.z);
-    s.w = fmaf(ki, vj[3], s.w);
-    *reinterpret_cast<float4 *>(S + (size_t)i * D + j0) = s;
-    acc[0] = fmaf(qi, s.x, acc[0]);
-    acc[1] = fmaf(qi, s.y, acc[1]);
-    acc[2] = fmaf(qi, s.z, acc[2]);
-    acc[3] = fmaf(qi, s.w, acc[3]);
-  }
-  // reduce over the 32 row groups: s_red[rg][col]
-#pragma unroll
-  for (int c4 = 0; c4 < 4; ++c4) s_red[rg][cg * 4 + c4] = acc[c4];
-  __syncthreads();
-  if (tid < 32) {
-    float o = 0.f;
-    for (int r = 0; r < 32; ++r) o += s_red[r][tid];
-    p.olin[((size_t)b * p.Hq + h) * D + slab * 32 + tid] = o;
-  }
-}
-
-// ============================================================ kernel 2
-template <int NT>
-__global__ void __launch_bounds__(NT) decode_select_kernel(DecodeParams p) {
-  extern __shared__ __align__(16) uint32_t s_dyn[];
-  __shared__ TopmShared sm;
-  grid_dep_wait();
-  grid_dep_launch();
-  const int bg = blockIdx.x;
-  const int b = bg / p.Hkv;
-  const int t = p.pos[b];
-  if (t < 0 || t >= p.L_max) return;
   const int n = t + 1;
-  const uint32_t *gkeys = p.keys + (size_t)bg * p.keys_stride;
-  const uint32_t *keys = gkeys;
-  uint32_t *cand = s_dyn;
-  if (n <= p.smem_keys_cap && n > p.M) {
-    uint32_t *sk = s_dyn;
-    const int n4 = n & ~3;
-    for (int i = threadIdx.x * 4; i < n4; i += NT * 4)
-      *reinterpret_cast<uint4 *>(sk + i) = __ldcg(reinterpret_cast<const uint4 *>(gkeys + i));
-    for (int i = n4 + threadIdx.x; i < n; i += NT) sk[i] = __ldcg(gkeys + i);
-    __syncthreads();
-    keys = sk;
-    cand = s_dyn + p.smem_keys_cap;
+  const int kpc = (((n + NC - 1) / NC) + 31) & ~31;
+  const int k0 = min(n, rank * kpc);
+  const int k1 = min(n, k0 + kpc);
+  const int cnt = k1 - k0;
+  const int nsub = (cnt + SUB - 1) / SUB;
+
+  const T *kidx_cache = reinterpret_cast<const T *>(p.kidx_cache) + (size_t)bg * p.L_max * DI;
+  const T *kidx_new = reinterpret_cast<const T *>(p.kidx) + (size_t)bg * DI;
+
+  // ---------------------------------------------------------------- TMA prologue
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
   }
-  int *out = p.idx + (size_t)bg * p.M;
-  if (!block_topm<NT>(keys, n, p.M, out, sm, cand, p.cand_cap) && threadIdx.x == 0)
-    set_err(p.err_word, LISA_DEVERR_CHECK);
-  if (p.idx_out) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < p.M; i += NT) p.idx_out[(size_t)bg * p.M + i] = __ldcg(out + i);
+  __syncthreads();
+  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % kStages
+    const int s_lo = k0 + i * SUB;
+    const int s_hi = min(k1, s_lo + SUB);
+    const int ncopy = max(0, min(s_hi, t) - s_lo);   // row t comes from the argument
+    uint64_t *bar = &bars[i % kStages];
+    unsigned char *dst = ring + (i % kStages) * kStageBytes;
+    if (ncopy > 0) {
+      if constexpr (SG::kMma) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(SUB * RB));   // the whole box lands, out-of-range rows zero
+        tma_load_2d(dst, &kmap, 0, bg * p.L_max + s_lo, bar);
+      } else {
+        mbar_arrive_expect_tx(bar, (uint32_t)(ncopy * RB));
+        bulk_g2s(dst, kidx_cache + (size_t)s_lo * DI, (uint32_t)(ncopy * RB), bar);
+      }
+    } else {
+      mbar_arrive(bar);
+    }
+  };
+  if (tid == 0)
+    for (int i = 0; i < min(kStages, nsub); ++i) issue(i);
+
+  // ---------------------------------------------------------------- early loads
+  // state slab of the first (up to) 8 query heads: in flight during scoring
+  const int c0s = rank * COLS;
+  const int cq = tid % QPR;                // same float4 column for every row this thread visits
+  const int gA = min(G, 8);
+  float4 sv[8][ITER];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    if (hh >= gA) continue;
+    const float *S = p.state + ((size_t)b * p.Hq + g * G + hh) * D * D;
+#pragma unroll
+    for (int it = 0; it < ITER; ++it) {
+      const int idx = tid + it * kDecThreads;
+      if (idx < D * QPR) sv[hh][it] = *reinterpret_cast<const float4 *>(S + (size_t)(idx / QPR) * D + c0s + cq * 4);
+    }
   }
-}
+  const T *qin = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + g * G) * D;
+  for (int i = tid; i < G * D; i += kDecThreads) qs[i] = Dt<T>::to_f(qin[i]);
+  const T *kin = reinterpret_cast<const T *>(p.k) + (size_t)bg * D;
+  const T *vin = reinterpret_cast<const T *>(p.v) + (size_t)bg * D;
+  for (int i = tid; i < D; i += kDecThreads) {
+    ks[i] = Dt<T>::to_f(kin[i]);
+    vs[i] = Dt<T>::to_f(vin[i]);
+  }
+  for (int i = tid; i < R * DI; i += kDecThreads)
+    qis[i] = Dt<T>::to_f(reinterpret_cast<const T *>(p.qidx)[((size_t)b * p.HI + g * R) * DI + i]);
+  if (tid < R) qis[kMaxR * DI + tid] = p.w[(size_t)b * p.HI + g * R + tid];
+  // MMA operand B (indexer queries, heads = columns, padded to 8) and the head weights of this lane
+  uint32_t bq[DI / 16][2];
+  float wq0 = 0.f, wq1 = 0.f;
+  if constexpr (SG::kMma) {
+    const int nh = lane >> 2, kc = 2 * (lane & 3);
+    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(reinterpret_cast<const T *>(p.qidx) +
+                                                               ((size_t)b * p.HI + g * R + (nh < R ? nh : 0)) * DI);
+#pragma unroll
+    for (int s = 0; s < DI / 16; ++s) {
+      bq[s][0] = nh < R ? qrow[(s * 16 + kc) >> 1] : 0u;
+      bq[s][1] = nh < R ? qrow[(s * 16 + kc + 8) >> 1] : 0u;
+    }
+    if (kc < R) wq0 = p.w[(size_t)b * p.HI + g * R + kc];
+    if (kc + 1 < R) wq1 = p.w[(size_t)b * p.HI + g * R + kc + 1];
+  }
+  // append the new token (row t) from the CTA whose key slice holds it
+  if (p.fuse_append && t >= k0 && t < k1) {
+    const size_t row = (size_t)bg * p.L_max + t;
+    T *kc = reinterpret_cast<T *>(p.k_cache) + row * D;
+    T *vc = reinterpret_cast<T *>(p.v_cache) + row * D;
+    T *kic = reinterpret_cast<T *>(p.kidx_cache) + row * DI;
+    for (int i = tid; i < D; i += kDecThreads) {
+      kc[i] = kin[i];
+      vc[i] = vin[i];
+    }
+    for (int i = tid; i < DI; i += kDecThreads) kic[i] = kidx_new[i];
+  }
+  __syncthreads();
 
-// ============================================================ kernel 3
-// CTA = (b, g, split of kRows selected rows); 256 threads = 8 warps.
-template <typename T, int D>
-__global__ void __launch_bounds__(256) decode_attend_kernel(DecodeParams p) {
-  constexpr int kRows = kAttnRows;     // selected rows per CTA
-  constexpr int kDPL = D / 32;         // dims per lane
-  __shared__ __align__(16) T s_k[kRows][D];
-  __shared__ __align__(16) T s_v[kRows][D];
-  __shared__ float s_q[kMaxG][D];
-  __shared__ float s_logit[kMaxG][kRows];
-  __shared__ int s_idx[kRows];
-  __shared__ int s_last;
+  // ---------------------------------------------------------------- indexer scores
+  for (int i = 0; i < nsub; ++i) {
+    const int stage = i % kStages;
+    if (!mbar_wait_bounded(&bars[stage], (uint32_t)((i / kStages) & 1)) && tid == 0)
+      set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+    const int s_lo = k0 + i * SUB;
+    const int nk = min(k1, s_lo + SUB) - s_lo;
+    const unsigned char *st = ring + stage * kStageBytes;
+    if constexpr (SG::kMma) {
+      // tiles of 16 keys; A = keys (row-major, swizzled by TMA), B = queries
+      const uint32_t st_u32 = smem_u32(st);
+      for (int tile = warp; tile * 16 < nk; tile += kDecThreads / 32) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        const int row = tile * 16 + (lane & 15);
+        const int swz = RB == 128 ? (row & 7) : ((row >> 1) & 3);
+#pragma unroll
+        for (int s = 0; s < DI / 16; ++s) {
+          const int chunk = 2 * s + (lane >> 4);
+          uint32_t a[4];
+          ldmatrix_x4(st_u32 + row * RB + ((chunk ^ swz) << 4), a[0], a[1], a[2], a[3]);
+          mma_16816_bf16(d, a, bq[s]);
+        }
+        // columns 2*(lane&3), +1 are indexer heads; rows lane/4 and lane/4 + 8
+        float p0 = fmaf(wq1, fmaxf(d[1], 0.f), wq0 * fmaxf(d[0], 0.f));
+        float p1 = fmaf(wq1, fmaxf(d[3], 0.f), wq0 * fmaxf(d[2], 0.f));
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+        if ((lane & 3) == 0) {
+          const int r0 = tile * 16 + (lane >> 2);
+          if (r0 < nk) keys[s_lo - k0 + r0] = score_key(p0);
+          if (r0 + 8 < nk) keys[s_lo - k0 + r0 + 8] = score_key(p1);
+        }
+      }
+    } else {
+      // one thread per key; chunk order rotated by the row so a wavefront
+      // touches different bank groups
+      const float *wsm = qis + kMaxR * DI;
+      for (int kk = tid; kk < nk; kk += kDecThreads) {
+        const unsigned char *row = st + kk * RB;
+        float acc[kMaxR][2];
+#pragma unroll
+        for (int r = 0; r < kMaxR; ++r) acc[r][0] = acc[r][1] = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < NCH; ++c0) {
+          const int c = (c0 + kk) & (NCH - 1);
+          float x[VEC];
+          Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(row + c * 16), x);
+#pragma unroll
+          for (int r = 0; r < kMaxR; ++r) {
+            if (r < R) {
+              const float *qr = qis + r * DI + c * VEC;
+#pragma unroll
+              for (int j = 0; j < VEC; ++j) acc[r][j & 1] = fmaf(qr[j], x[j], acc[r][j & 1]);
+            }
+          }
+        }
+        float score = 0.f;
+#pragma unroll
+        for (int r = 0; r < kMaxR; ++r)
+          if (r < R) score = fmaf(wsm[r], fmaxf(acc[r][0] + acc[r][1], 0.f), score);
+        keys[s_lo - k0 + kk] = score_key(score);
+      }
+    }
+    __syncthreads();   // every thread is done with this stage
+    if (tid == 0 && i + kStages < nsub) issue(i + kStages);
+  }
+  // the new token's score, from the argument row (its cache row may be stale)
+  if (t >= k0 && t < k1 && warp == 0) {
+    const float *wsm = qis + kMaxR * DI;
+    float score = 0.f;
+    for (int r = 0; r < R; ++r) {
+      float dot = 0.f;
+      for (int c = lane; c < DI; c += 32) dot = fmaf(qis[r * DI + c], Dt<T>::to_f(kidx_new[c]), dot);
+      dot = warp_sum(dot);
+      score = fmaf(wsm[r], fmaxf(dot, 0.f), score);
+    }
+    if (lane == 0) keys[t - k0] = score_key(score);
+  }
 
-  grid_dep_wait();
-  grid_dep_launch();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nsplit = p.M / kRows;
-  const int sp = blockIdx.x % nsplit;
-  const int bg = blockIdx.x / nsplit;
-  const int g = bg % p.Hkv;
-  const int b = bg / p.Hkv;
-  const int t = p.pos[b];
-  if (t < 0 || t >= p.L_max) return;
-  const int G = p.G;
+  // ---------------------------------------------------------------- linear state
+  // S_h <- S_h + k^T v on columns [c0s, c0s + COLS); o_lin[h][c] = sum_i q_h[i] S_h[i][c]
+  {
+    float vj[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) vj[j] = vs[c0s + cq * 4 + j];
+    float *red = logit;                  // scratch [8 heads][8 warps][COLS]
+    for (int h0 = 0; h0 < G; h0 += 8) {
+      const int hn = min(8, G - h0);
+      if (h0 > 0) {                      // heads beyond the first 8 are loaded now
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh) {
+          if (hh >= hn) continue;
+          const float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
+#pragma unroll
+          for (int it = 0; it < ITER; ++it) {
+            const int idx = tid + it * kDecThreads;
+            if (idx < D * QPR)
+              sv[hh][it] = *reinterpret_cast<const float4 *>(S + (size_t)(idx / QPR) * D + c0s + cq * 4);
+          }
+        }
+      }
+      __syncthreads();                   // red is free
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) {
+        if (hh >= hn) continue;
+        float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
+        const float *qh = qs + (h0 + hh) * D;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int it = 0; it < ITER; ++it) {
+          const int idx = tid + it * kDecThreads;
+          if (idx < D * QPR) {
+            const int i = idx / QPR;
+            const float ki = ks[i], qi = qh[i];
+            float4 sn = sv[hh][it];
+            sn.x = fmaf(ki, vj[0], sn.x);
+            sn.y = fmaf(ki, vj[1], sn.y);
+            sn.z = fmaf(ki, vj[2], sn.z);
+            sn.w = fmaf(ki, vj[3], sn.w);
+            *reinterpret_cast<float4 *>(S + (size_t)i * D + c0s + cq * 4) = sn;
+            a0 = fmaf(qi, sn.x, a0);
+            a1 = fmaf(qi, sn.y, a1);
+            a2 = fmaf(qi, sn.z, a2);
+            a3 = fmaf(qi, sn.w, a3);
+          }
+        }
+#pragma unroll
+        for (int o = QPR; o < 32; o <<= 1) {
+          a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+          a3 += __shfl_xor_sync(0xffffffffu, a3, o);
+        }
+        if (lane < QPR) {
+          float *rw = red + (hh * 8 + warp) * COLS + lane * 4;
+          rw[0] = a0;
+          rw[1] = a1;
+          rw[2] = a2;
+          rw[3] = a3;
+        }
+      }
+      __syncthreads();
+      for (int i = tid; i < hn * COLS; i += kDecThreads) {
+        const int hh = i / COLS, c = i % COLS;
+        float o = 0.f;
+#pragma unroll
+        for (int w8 = 0; w8 < 8; ++w8) o += red[(hh * 8 + w8) * COLS + c];
+        olin[(h0 + hh) * COLS + c] = o;
+      }
+    }
+  }
+  __syncthreads();
 
-  if (tid < kRows) {
-    int s = __ldcg(p.idx + (size_t)bg * p.M + sp * kRows + tid);
+  // ---------------------------------------------------------------- top-M
+  int *sel0 = cluster.map_shared_rank(sel, 0);
+  if (n > M) {
+    // (a) theta = the smallest of kl group maxima of this CTA's keys (groups:
+    //     positions j = g (mod kl)); at least kl of its keys are >= theta.
+    int kl = 1;
+    while (kl < (M + NC - 1) / NC) kl <<= 1;
+    int covered = 0;
+    for (int r = 0; r < NC; ++r) {
+      const int cr = min(n, (r + 1) * kpc) - min(n, r * kpc);
+      if (cr >= kl) covered += kl;
+    }
+    uint32_t theta = 0xFFFFFFFFu;                       // neutral for the minimum
+    if (cnt >= kl) {
+      uint32_t m = 0;
+      for (int j = tid; j < cnt; j += kDecThreads) m = max(m, keys[j]);
+      tot[tid] = m;                                     // thread tid holds group tid % kl
+      __syncthreads();
+      if (tid < kl) {
+        uint32_t gm = 0;
+        for (int j = tid; j < kDecThreads; j += kl) gm = max(gm, tot[j]);
+        hist[tid] = gm;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t mn = 0xFFFFFFFFu;
+        for (int j = lane; j < kl; j += 32) mn = min(mn, hist[j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        theta = mn;
+      }
+    }
+    if (tid == 0) {
+      misc[4] = theta;
+      if (rank == 0) misc[5] = 0;                       // candidate counter in CTA 0
+    }
+    cluster.sync();                                     // bounds published, every ring is free
+    uint32_t lb = 0;
+    if (covered >= M) {
+      lb = 0xFFFFFFFFu;
+#pragma unroll
+      for (int r = 0; r < NC; ++r) lb = min(lb, cluster.map_shared_rank(misc, r)[4]);
+    }
+    // (b) keys >= lb go to CTA 0 (unordered): one slot reservation per warp
+    uint32_t *cnt0 = cluster.map_shared_rank(misc, 0) + 5;
+    uint32_t *ckey0 = cluster.map_shared_rank(reinterpret_cast<uint32_t *>(smem + lay.cand_key), 0);
+    int *cpos0 = cluster.map_shared_rank(reinterpret_cast<int *>(smem + lay.cand_pos), 0);
+    {
+      const int iters = (cnt + kDecThreads - 1) / kDecThreads;
+      const unsigned lt = (1u << lane) - 1u;
+      uint32_t wc = 0;
+      for (int it = 0; it < iters; ++it) {
+        const int j = tid + it * kDecThreads;
+        wc += __popc(__ballot_sync(0xffffffffu, j < cnt && keys[j] >= lb));
+      }
+      uint32_t off = 0;
+      if (lane == 0 && wc) off = atomicAdd(cnt0, wc);
+      off = __shfl_sync(0xffffffffu, off, 0);
+      for (int it = 0; it < iters; ++it) {
+        const int j = tid + it * kDecThreads;
+        const bool act = j < cnt && keys[j] >= lb;
+        const unsigned am = __ballot_sync(0xffffffffu, act);
+        if (act) {
+          const uint32_t slot = off + __popc(am & lt);
+          if (slot < (uint32_t)kCandCap) {
+            ckey0[slot] = keys[j];
+            cpos0[slot] = k0 + j;
+          }
+        }
+        off += __popc(am);
+      }
+    }
+    cluster.sync();                                     // candidates complete
+    const uint32_t n_c = *cnt0;
+    if (n_c <= (uint32_t)kCandCap) {
+      if (rank == 0) {
+        // (c) CTA 0: exact M-th key among the candidates, then the selected
+        //     positions in ascending order through two position bitmaps
+        const uint32_t *ck = reinterpret_cast<const uint32_t *>(smem + lay.cand_key);
+        const int *cp = reinterpret_cast<const int *>(smem + lay.cand_pos);
+        uint32_t *gtb = reinterpret_cast<uint32_t *>(smem + lay.gtb);
+        uint32_t *eqb = reinterpret_cast<uint32_t *>(smem + lay.eqb);
+        const uint32_t kstar = cta_kth_prefix(ck, (int)n_c, (uint32_t)M, 4, hist, tot, misc);
+        const int nw = (n + 31) >> 5;
+        for (int i = tid; i < nw; i += kDecThreads) {
+          gtb[i] = 0;
+          eqb[i] = 0;
+        }
+        __syncthreads();
+        for (int j = tid; j < (int)n_c; j += kDecThreads) {
+          const uint32_t u = ck[j];
+          const int pos = cp[j];
+          if (pos < 0 || pos >= n) {
+            set_err(p.err_word, LISA_DEVERR_CHECK);
+            continue;
+          }
+          if (u > kstar) atomicOr(&gtb[pos >> 5], 1u << (pos & 31));
+          else if (u == kstar) atomicOr(&eqb[pos >> 5], 1u << (pos & 31));
+        }
+        // each thread owns a run of bitmap words, in position order
+        const int wpt = (nw + kDecThreads - 1) / kDecThreads;
+        const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
+        __syncthreads();
+        uint32_t cgt = 0, ceq = 0;
+        for (int w = w0; w < w1; ++w) {
+          cgt += __popc(gtb[w]);
+          ceq += __popc(eqb[w]);
+        }
+        uint32_t eg, ee, tg, te;
+        cta_scan2(cgt, ceq, eg, ee, tg, te, misc);
+        const uint32_t need_eq = (uint32_t)M - tg;      // keys equal to K* still to take
+        for (int w = w0; w < w1; ++w) {
+          const uint32_t gb = gtb[w], eb = eqb[w];
+          uint32_t bits = gb | eb;
+          while (bits) {
+            const int bpos = __ffs(bits) - 1;
+            bits &= bits - 1;
+            const int pos = (w << 5) + bpos;
+            if ((gb >> bpos) & 1u) {
+              const uint32_t o = eg + min(ee, need_eq);
+              if (o < (uint32_t)M) sel[o] = pos;
+              else set_err(p.err_word, LISA_DEVERR_CHECK);
+              ++eg;
+            } else {
+              if (ee < need_eq) {
+                const uint32_t o = eg + ee;
+                if (o < (uint32_t)M) sel[o] = pos;
+                else set_err(p.err_word, LISA_DEVERR_CHECK);
+              }
+              ++ee;
+            }
+          }
+        }
+      }
+    } else {
+      // (d) too many keys passed the bound: cluster-wide radix select over all keys
+      uint32_t prefix = 0, pmask = 0, rem = (uint32_t)M;
+      bool ok = true;
+      const int iters = (cnt + kDecThreads - 1) / kDecThreads;
+#pragma unroll 1
+      for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        // Written here, read by every CTA after the cluster barrier below, and
+        // rewritten two passes later, after another cluster barrier.
+        uint32_t *H = hist + (pass & 1) * 256;
+        __syncthreads();
+        H[tid] = 0;                            // 256 threads, 256 bins
+        __syncthreads();
+        for (int it = 0; it < iters; ++it) {
+          const int j = tid + it * kDecThreads;
+          uint32_t u = 0;
+          bool act = false;
+          if (j < cnt) {
+            u = keys[j];
+            act = (u & pmask) == prefix;
+          }
+          const uint32_t dig = (u >> shift) & 255u;
+          const unsigned am = __ballot_sync(0xffffffffu, act);
+          if (act) {
+            const unsigned peers = __match_any_sync(am, dig);
+            if (lane == __ffs(peers) - 1) atomicAdd(&H[dig], (uint32_t)__popc(peers));
+          }
+        }
+        cluster.sync();                        // every CTA's histogram of this pass is complete
+        {
+          uint32_t s = 0;
+#pragma unroll
+          for (int r = 0; r < NC; ++r) s += cluster.map_shared_rank(H, r)[tid];
+          tot[tid] = s;
+        }
+        if (tid == 0) misc[0] = 0xFFFFFFFFu;
+        __syncthreads();
+        dec_find_bucket(tot, misc, rem);
+        __syncthreads();
+        const uint32_t dig = misc[0];
+        const uint32_t above = misc[1];
+        if (dig > 255u) {                      // inconsistent counts: cannot happen for valid keys
+          ok = false;
+          continue;                            // keep every cluster barrier matched
+        }
+        rem -= above;
+        prefix |= dig << shift;
+        pmask |= 255u << shift;
+      }
+      if (!ok) {
+        if (tid == 0) set_err(p.err_word, LISA_DEVERR_CHECK);
+        prefix = 0xFFFFFFFFu;                  // nothing is above; emits no more than need_eq = 0
+        rem = 0;
+      }
+      const uint32_t kstar = prefix, need_eq = rem;
+
+      // counts of keys above / equal to K* in this CTA's slice, then cluster prefix
+      const int per_warp = (((cnt + 7) / 8) + 31) & ~31;
+      const int c0w = warp * per_warp;
+      const int c1w = min(cnt, c0w + per_warp);
+      uint32_t gw = 0, ew = 0;
+      for (int base = c0w; base < c1w; base += 32) {
+        const int j = base + lane;
+        const uint32_t u = j < c1w ? keys[j] : 0u;
+        gw += __popc(__ballot_sync(0xffffffffu, j < c1w && u > kstar));
+        ew += __popc(__ballot_sync(0xffffffffu, j < c1w && u == kstar));
+      }
+      __syncthreads();
+      if (lane == 0) {
+        misc[8 + warp] = gw;
+        misc[16 + warp] = ew;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t sg = 0, se = 0;
+        for (int w8 = 0; w8 < 8; ++w8) {
+          const uint32_t a = misc[8 + w8], c = misc[16 + w8];
+          misc[8 + w8] = sg;       // exclusive prefix within the CTA
+          misc[16 + w8] = se;
+          sg += a;
+          se += c;
+        }
+        misc[2] = sg;              // CTA totals, read by the other CTAs
+        misc[3] = se;
+      }
+      cluster.sync();
+      uint32_t gb = 0, eb = 0;
+      for (int r = 0; r < rank; ++r) {
+        const uint32_t *mr = cluster.map_shared_rank(misc, r);
+        gb += mr[2];
+        eb += mr[3];
+      }
+      uint32_t gcur = gb + misc[8 + warp], ecur = eb + misc[16 + warp];
+      const unsigned lt = (1u << lane) - 1u;
+      for (int base = c0w; base < c1w; base += 32) {
+        const int j = base + lane;
+        const uint32_t u = j < c1w ? keys[j] : 0u;
+        const unsigned bgt = __ballot_sync(0xffffffffu, j < c1w && u > kstar);
+        const unsigned beq = __ballot_sync(0xffffffffu, j < c1w && u == kstar);
+        const uint32_t pe = ecur + __popc(beq & lt);
+        const bool gt = (bgt >> lane) & 1u, eq = (beq >> lane) & 1u;
+        if (gt || (eq && pe < need_eq)) {
+          const uint32_t o = gcur + __popc(bgt & lt) + min(pe, need_eq);
+          if (o < (uint32_t)M) sel0[o] = k0 + j;
+          else set_err(p.err_word, LISA_DEVERR_CHECK);
+        }
+        gcur += __popc(bgt);
+        ecur += __popc(beq);
+      }
+      if (!ok && rank == 0)
+        for (int j = tid; j < M; j += kDecThreads) sel[j] = -1;
+    }
+  } else if (rank == 0) {
+    for (int j = tid; j < M; j += kDecThreads) sel[j] = j < n ? j : -1;
+  }
+  cluster.sync();                            // CTA 0 holds the full ascending index list
+  if (rank == 0 && p.idx_out)
+    for (int j = tid; j < M; j += kDecThreads) p.idx_out[(size_t)bg * M + j] = sel[j];
+
+  // ---------------------------------------------------------------- sparse attention (this CTA's rows)
+  unsigned char *kvs = ring;                 // [rpc] K rows then [rpc] V rows, stride RS
+  for (int r = tid; r < rpc; r += kDecThreads) {
+    int s = sel0[rank * rpc + r];
     if (s < -1 || s > t) {
       set_err(p.err_word, LISA_DEVERR_CHECK);
       s = -1;
     }
-    s_idx[tid] = s;
-  }
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int hh = i / D, dd = i % D;
-    s_q[hh][dd] = Dt<T>::to_f(reinterpret_cast<const T *>(p.q)[((size_t)b * p.Hq + g * G + hh) * D + dd]);
+    sidx[r] = s;
   }
   __syncthreads();
-
-  // gather K and V rows (16-byte loads); the new token comes from the arguments
-  constexpr int kSlices = D * (int)sizeof(T) / 16;
-  const T *kc = reinterpret_cast<const T *>(p.k_cache) + ((size_t)b * p.Hkv + g) * p.L_max * D;
-  const T *vc = reinterpret_cast<const T *>(p.v_cache) + ((size_t)b * p.Hkv + g) * p.L_max * D;
-  const T *kn = reinterpret_cast<const T *>(p.k) + ((size_t)b * p.Hkv + g) * D;
-  const T *vn = reinterpret_cast<const T *>(p.v) + ((size_t)b * p.Hkv + g) * D;
-  for (int i = tid; i < kRows * kSlices; i += blockDim.x) {
-    const int r = i / kSlices, sl = i % kSlices;
-    const int s = s_idx[r];
-    uint4 uk = make_uint4(0, 0, 0, 0), uv = make_uint4(0, 0, 0, 0);
-    if (s >= 0) {
-      const T *ks = (s == t) ? kn : kc + (size_t)s * D;
-      const T *vs = (s == t) ? vn : vc + (size_t)s * D;
-      uk = *reinterpret_cast<const uint4 *>(ks + sl * (16 / sizeof(T)));
-      uv = *reinterpret_cast<const uint4 *>(vs + sl * (16 / sizeof(T)));
-    }
-    reinterpret_cast<uint4 *>(&s_k[r][0])[sl] = uk;
-    reinterpret_cast<uint4 *>(&s_v[r][0])[sl] = uv;
-  }
-  __syncthreads();
-
-  // logits: warp per row, lanes split d
-  for (int r = warp; r < kRows; r += 8) {
-    float kx[kDPL];
-#pragma unroll
-    for (int j = 0; j < kDPL; ++j) kx[j] = Dt<T>::to_f(s_k[r][lane * kDPL + j]);
-    const bool valid = s_idx[r] >= 0;
-    for (int hh = 0; hh < G; ++hh) {
-      float dot = 0.f;
-#pragma unroll
-      for (int j = 0; j < kDPL; ++j) dot = fmaf(s_q[hh][lane * kDPL + j], kx[j], dot);
-      dot = warp_sum(dot);
-      if (lane == 0) s_logit[hh][r] = valid ? dot * p.scale : -INFINITY;
+  {
+    const T *kc = reinterpret_cast<const T *>(p.k_cache) + (size_t)bg * p.L_max * D;
+    const T *vc = reinterpret_cast<const T *>(p.v_cache) + (size_t)bg * p.L_max * D;
+    for (int i = tid; i < rpc * SL; i += kDecThreads) {
+      const int r = i / SL, sl = i % SL;
+      const int s = sidx[r];
+      uint4 uk = make_uint4(0, 0, 0, 0), uv = make_uint4(0, 0, 0, 0);
+      if (s >= 0) {
+        const T *kr = (s == t) ? kin : kc + (size_t)s * D;
+        const T *vr = (s == t) ? vin : vc + (size_t)s * D;
+        uk = *reinterpret_cast<const uint4 *>(kr + sl * VEC);
+        uv = *reinterpret_cast<const uint4 *>(vr + sl * VEC);
+      }
+      *reinterpret_cast<uint4 *>(kvs + r * RS + sl * 16) = uk;
+      *reinterpret_cast<uint4 *>(kvs + (rpc + r) * RS + sl * 16) = uv;
     }
   }
   __syncthreads();
-
-  // per head: local max, exp, sum, and the weighted V sum -> partials
-  float *part = p.partials + (((size_t)bg * nsplit + sp) * G) * (D + 2);
+  // logits[hh][r] = q_h . k_r / sqrt(d)
+  for (int i = tid; i < G * rpc; i += kDecThreads) {
+    const int hh = i / rpc, r = i % rpc;
+    float l = -INFINITY;
+    if (sidx[r] >= 0) {
+      const float *qh = qs + hh * D;
+      const unsigned char *kr = kvs + r * RS;
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+      for (int sl = 0; sl < SL; ++sl) {
+        float x[VEC];
+        Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(kr + sl * 16), x);
+#pragma unroll
+        for (int j = 0; j < VEC; j += 2) {
+          a0 = fmaf(qh[sl * VEC + j], x[j], a0);
+          a1 = fmaf(qh[sl * VEC + j + 1], x[j + 1], a1);
+        }
+      }
+      l = (a0 + a1) * p.scale;
+    }
+    logit[hh * rpc + r] = l;
+  }
+  __syncthreads();
+  // per head: local max and sum of exponentials over this CTA's rows
   for (int hh = warp; hh < G; hh += 8) {
-    float m = s_logit[hh][lane];  // kRows == 32
+    float m = -INFINITY;
+    for (int r = lane; r < rpc; r += 32) m = fmaxf(m, logit[hh * rpc + r]);
     m = warp_max(m);
-    const float e = (m == -INFINITY) ? 0.f : expf(s_logit[hh][lane] - m);
-    const float l = warp_sum(e);
-    s_logit[hh][lane] = e;
-    __syncwarp();
-    float acc[kDPL];
-#pragma unroll
-    for (int j = 0; j < kDPL; ++j) acc[j] = 0.f;
-    for (int r = 0; r < kRows; ++r) {
-      const float pr = s_logit[hh][r];
-#pragma unroll
-      for (int j = 0; j < kDPL; ++j) acc[j] = fmaf(pr, Dt<T>::to_f(s_v[r][lane * kDPL + j]), acc[j]);
+    float l = 0.f;
+    for (int r = lane; r < rpc; r += 32) {
+      const float x = logit[hh * rpc + r];
+      const float e = (x == -INFINITY) ? 0.f : expf(x - m);
+      logit[hh * rpc + r] = e;
+      l += e;
     }
-    float *ph = part + (size_t)hh * (D + 2);
-#pragma unroll
-    for (int j = 0; j < kDPL; ++j) ph[lane * kDPL + j] = acc[j];
+    l = warp_sum(l);
     if (lane == 0) {
-      ph[D] = m;
-      ph[D + 1] = l;
+      pml[2 * hh] = m;
+      pml[2 * hh + 1] = l;
     }
   }
+  __syncthreads();
+  // part[hh][d] = sum_r e[hh][r] v_r[d]
+  for (int i = tid; i < G * D; i += kDecThreads) {
+    const int hh = i / D, d = i % D;
+    const float *e = logit + hh * rpc;
+    const T *vcol = reinterpret_cast<const T *>(kvs + rpc * RS) + d;
+    float a = 0.f;
+    for (int r = 0; r < rpc; ++r) a = fmaf(e[r], Dt<T>::to_f(vcol[(size_t)r * (RS / sizeof(T))]), a);
+    part[i] = a;
+  }
+  cluster.sync();                            // all partials of the cluster are ready
 
-  // last CTA of this (b, g) merges the splits and applies the gate
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(p.counters + bg, 1u) == (unsigned)(nsplit - 1));
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float *pb = p.partials + ((size_t)bg * nsplit) * G * (D + 2);
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int hh = i / D, dd = i % D;
+  // ---------------------------------------------------------------- merge + gate, columns of this CTA
+  for (int i = tid; i < G * COLS; i += kDecThreads) {
+    const int hh = i / COLS, c = i % COLS, d = c0s + c;
     float mx = -INFINITY;
-    for (int s2 = 0; s2 < nsplit; ++s2) mx = fmaxf(mx, __ldcg(pb + ((size_t)s2 * G + hh) * (D + 2) + D));
+#pragma unroll
+    for (int r = 0; r < NC; ++r) mx = fmaxf(mx, cluster.map_shared_rank(pml, r)[2 * hh]);
     float num = 0.f, den = 0.f;
-    for (int s2 = 0; s2 < nsplit; ++s2) {
-      const float *ph = pb + ((size_t)s2 * G + hh) * (D + 2);
-      const float ms = __ldcg(ph + D);
-      if (ms == -INFINITY) continue;
-      const float f = expf(ms - mx);
-      num = fmaf(f, __ldcg(ph + dd), num);
-      den = fmaf(f, __ldcg(ph + D + 1), den);
+#pragma unroll
+    for (int r = 0; r < NC; ++r) {
+      const float *pr = cluster.map_shared_rank(pml, r);
+      const float mr = pr[2 * hh];
+      if (mr == -INFINITY) continue;
+      const float f = expf(mr - mx);
+      num = fmaf(f, cluster.map_shared_rank(part, r)[hh * D + d], num);
+      den = fmaf(f, pr[2 * hh + 1], den);
     }
     const int h = g * G + hh;
     const float o_sp = num / den;
-    const float o_lin = __ldcg(p.olin + ((size_t)b * p.Hq + h) * D + dd);
+    const float o_lin = olin[hh * COLS + c];
     const float gam = 1.f / (1.f + expf(-p.gate[(size_t)b * p.Hq + h]));
-    const float o = gam * o_sp + (1.f - gam) * o_lin;
-    reinterpret_cast<T *>(p.out)[((size_t)b * p.Hq + h) * D + dd] = Dt<T>::from_f(o);
+    reinterpret_cast<T *>(p.out)[((size_t)b * p.Hq + h) * D + d] = Dt<T>::from_f(gam * o_sp + (1.f - gam) * o_lin);
   }
+  cluster.sync();                            // keep this CTA's shared memory alive for its readers
 }
 
 // ============================================================ launcher
-template <typename T, int D, int DI>
-static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t st) {
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+template <typename T, int D, int DI, int NC>
+static cudaError_t launch_cluster_t(const DecodeParams &p, const CUtensorMap &kmap, cudaStream_t st) {
+  auto kern = decode_cluster_kernel<T, D, DI, NC>;
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), NC);
+  cudaError_t e = prepare_kernel(kern, lay.total);
+  if (e != cudaSuccess) return e;
+  if (NC > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = NC;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.B * p.Hkv * NC);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = lay.total;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, p, kmap);
+}
 
-  {
-    cudaError_t e = prepare_kernel(decode_score_state_kernel<T, D, DI>);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.n_score_blocks + p.n_state_blocks);
-    cfg.blockDim = dim3(256);
-    cfg.stream = st;
-    e = cudaLaunchKernelEx(&cfg, decode_score_state_kernel<T, D, DI>, p);
-    if (e != cudaSuccess) return e;
+// 16 when a 16-CTA cluster of this kernel can be scheduled on this device, else 8.
+template <typename T, int D, int DI>
+static int pick_cluster(const DecodeParams &p) {
+  auto kern = decode_cluster_kernel<T, D, DI, 16>;
+  const int kpc = (((p.L_max + 15) / 16) + 31) & ~31;
+  const DecLayout lay = dec_layout(kpc, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), 16);
+  if (prepare_kernel(kern, lay.total) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 8;
   }
-  {
-    constexpr int NT = 1024;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.B * p.Hkv);
-    cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = p.select_smem;
-    cfg.stream = st;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    cudaError_t e = prepare_kernel(decode_select_kernel<NT>, (int)p.select_smem);
-    if (e != cudaSuccess) return e;
-    e = cudaLaunchKernelEx(&cfg, decode_select_kernel<NT>, p);
-    if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 16;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(16);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = lay.total;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int nclusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 8;
   }
-  {
-    cudaError_t e = prepare_kernel(decode_attend_kernel<T, D>);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.B * p.Hkv * (p.M / kAttnRows));
-    cfg.blockDim = dim3(256);
-    cfg.stream = st;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_attend_kernel<T, D>, p);
-    if (e != cudaSuccess) return e;
+  return nclusters > 0 ? 16 : 8;
+}
+
+template <typename T, int D, int DI>
+static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
+  // the cluster size depends on the device and the shared-memory footprint: cache per (device, footprint)
+  static int cache_dev[8] = {-1, -1, -1, -1, -1, -1, -1, -1};
+  static int cache_key[8], cache_nc[8];
+  static int next = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int key = p.L_max * 2 + (p.M << 20) + (p.G << 28);
+  int nc = 0;
+  for (int i = 0; i < 8; ++i)
+    if (cache_dev[i] == dev && cache_key[i] == key) nc = cache_nc[i];
+  if (!nc) {
+    nc = pick_cluster<T, D, DI>(p);
+    const int slot = next++ & 7;
+    cache_dev[slot] = dev;
+    cache_key[slot] = key;
+    cache_nc[slot] = nc;
   }
-  return cudaSuccess;
+  p.nc = nc;
+  p.kpc_max = (((p.L_max + nc - 1) / nc) + 31) & ~31;
+  CUtensorMap kmap;
+  memset(&kmap, 0, sizeof(kmap));
+  if (ScoreGeom<T, DI>::kMma) {
+    using SG = ScoreGeom<T, DI>;
+    if (!make_tmap_2d(&kmap, p.kidx_cache, (int)sizeof(T), (unsigned long long)DI,
+                      (unsigned long long)p.B * p.Hkv * p.L_max, (unsigned long long)SG::RB, DI, SG::SUB, SG::RB))
+      return cudaErrorInvalidValue;
+  }
+  if (nc == 16) return launch_cluster_t<T, D, DI, 16>(p, kmap, st);
+  return launch_cluster_t<T, D, DI, 8>(p, kmap, st);
+}
+
+int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc) {
+  const int kpc = (((L_max + nc - 1) / nc) + 31) & ~31;
+  return dec_layout(kpc, L_max, M, G, D, DI, esize, nc).total;
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t st) {

@@ -1,6 +1,7 @@
 // Internal launch parameters shared by the C-ABI layer and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -24,6 +25,13 @@ cudaError_t prepare_kernel(F *fn, int dyn_smem = 0) {
   return prepare_kernel_ptr(reinterpret_cast<const void *>(fn), dyn_smem);
 }
 
+// 2-D tiled TMA tensor map over a row-major [rows][cols] array (elements of
+// elem_bytes, rows row_stride_bytes apart), box [box_rows][box_cols], with the
+// given shared-memory swizzle span (0, 32, 64 or 128 bytes).  Host only.
+bool make_tmap_2d(CUtensorMap *map, const void *base, int elem_bytes, unsigned long long cols,
+                  unsigned long long rows, unsigned long long row_stride_bytes, unsigned box_cols, unsigned box_rows,
+                  int swizzle_bytes);
+
 // ------------------------------------------------------------- decode
 struct DecodeParams {
   int B, Hq, Hkv, G, HI, R, D, DI, M, L_max;
@@ -39,19 +47,13 @@ struct DecodeParams {
   const float *w, *gate;
   void *out;
   int *idx_out;
-  // workspace carve-up
-  uint32_t *keys;       // [B, Hkv, keys_stride] order keys
-  int keys_stride;      // L_max rounded up to a multiple of 4
-  int *idx;             // [B, Hkv, M]
-  float *olin;          // [B, Hq, d]
-  float *partials;      // [B, Hkv, M/kAttnRows, G, d+2]
-  unsigned *counters;   // [B, Hkv]
-  // launch geometry
-  int n_chunks, n_score_blocks, n_state_blocks;
-  int smem_keys_cap, cand_cap;
-  size_t select_smem;
+  // launch geometry (filled by the launcher)
+  int nc;                               // CTAs per cluster
+  int kpc_max;                          // order keys per CTA, upper bound
 };
 
+// Dynamic shared memory of the decode kernel for a cluster of nc CTAs.
+int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc);
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t st);
 
 // ------------------------------------------------------------- row path

@@ -140,6 +140,10 @@ LISA_API lisa_status lisa_indexer_topk(const lisa_layer *layer, const void *qidx
  * when fuse_append != 0, also written to cache row t.  With fuse_append == 0
  * the caller must already have stored them there.  The state is updated in
  * place (S <- S + k^T v).  pos is not advanced.
+ * The step keeps all intermediates on chip: lisa_workspace_bytes() returns 0
+ * for LISA_OP_DECODE and `workspace` may be NULL.  The indexer keys of one
+ * (sequence, KV head) live in the shared memory of one thread-block cluster,
+ * which bounds L_max to about 280K tokens (LISA_ERR_UNSUPPORTED beyond).
  */
 LISA_API lisa_status lisa_decode_step(const lisa_layer *layer, const void *q, const void *k, const void *v,
                              const void *kidx, const void *qidx, const float *w,

@@ -228,3 +228,17 @@ def test_decode_graph_replays_are_stable():
             assert all(int(l.err_word.item()) == 0 for l in lays), f"replay {rep}"
             assert all(torch.equal(a, b) for a, b in zip(idxs, ref)), f"replay {rep}"
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("L_ctx", [16384, 3000])
+def test_decode_all_scores_equal(L_ctx):
+    """w = 0 makes every score 0: the first M positions must be selected (the
+    tie rule), and at 16384 tokens every key passes the candidate bound, which
+    exercises the cluster-wide radix path."""
+    cfg = _replace(get_config("decode_1p5b_16k"), B=1, L=L_ctx)
+    rng = make_rng(40 + L_ctx, 0)
+    lay = gen_layer(cfg, rng, L_ctx - 1)
+    step = gen_step(cfg, rng, 1)
+    step.w = np.zeros_like(step.w)
+    res = run_decode(cfg, lay, step, np.array([L_ctx - 1]), L_ctx, exact_sets=True)
+    assert res["ndiff"] == 0
