@@ -39,7 +39,7 @@ int round4(int x) { return (x + 3) & ~3; }
 constexpr int kDecodeKeysCap = 32768;   // order keys staged in shared memory (1024-thread select)
 constexpr int kRowsKeysCap = 16384;     // same, for the 256-thread row select
 constexpr int kCandCap = 4096;          // threshold-bucket candidates kept in shared memory
-constexpr int kRowChunk = 1024;         // query rows scored per pass on the row path
+constexpr int kRowChunk = 2048;         // query rows scored per pass on the row path
 constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory a CTA may use on sm_100
 
 // Validates the geometry; returns LISA_OK or the failure status.

@@ -31,6 +31,9 @@ cudaError_t prepare_kernel(F *fn, int dyn_smem = 0) {
 bool make_tmap_2d(CUtensorMap *map, const void *base, int elem_bytes, unsigned long long cols,
                   unsigned long long rows, unsigned long long row_stride_bytes, unsigned box_cols, unsigned box_rows,
                   int swizzle_bytes);
+// Same for rank 1..5: dims[0] innermost; strides_bytes[i] is the stride of dims[i+1].
+bool make_tmap(CUtensorMap *map, const void *base, int elem_bytes, int rank, const unsigned long long *dims,
+               const unsigned long long *strides_bytes, const unsigned *box, int swizzle_bytes);
 
 // ------------------------------------------------------------- decode
 struct DecodeParams {
@@ -83,6 +86,8 @@ struct RowsParams {
 
 cudaError_t launch_append(const RowsParams &p, int dtype, cudaStream_t st);
 cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, int key_limit);
+// bf16 indexer scores of rows [tau0, tau0 + rows) of the pass on the tensor cores.
+cudaError_t launch_rows_score_tc(const RowsParams &p, cudaStream_t st, int tau0, int rows, int key_hi);
 cudaError_t launch_prefill_linear(const RowsParams &p, int dtype, cudaStream_t st);
 cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st);
 

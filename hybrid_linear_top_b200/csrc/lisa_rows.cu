@@ -184,8 +184,13 @@ static cudaError_t rows_topk_t(const RowsParams &p, cudaStream_t st, int key_lim
     const int rows = min(p.row_chunk, p.T - tau0);
     // prefill (pos 0): keys up to tau0 + rows; general positions: up to key_limit
     const int key_hi = p.require_pos0 ? min(key_limit, tau0 + rows) : key_limit;
-    dim3 g1((key_hi + 63) / 64, (rows + 63) / 64, p.B * p.Hkv);
-    rows_score_kernel<T, DI><<<g1, 256, 0, st>>>(p, tau0, rows);
+    if constexpr (sizeof(T) == 2) {
+      e = launch_rows_score_tc(p, st, tau0, rows, key_hi);      // tensor cores (tcgen05)
+      if (e != cudaSuccess) return e;
+    } else {
+      dim3 g1((key_hi + 63) / 64, (rows + 63) / 64, p.B * p.Hkv);   // fp32: CUDA cores, exact products
+      rows_score_kernel<T, DI><<<g1, 256, 0, st>>>(p, tau0, rows);
+    }
     dim3 g2(rows, p.B * p.Hkv);
     rows_select_kernel<NT><<<g2, NT, p.select_smem, st>>>(p, tau0, rows);
     e = cudaGetLastError();
