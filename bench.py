@@ -350,12 +350,52 @@ def run_lisa(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args, rank, world):
+    """Timing of the causal prefill workload (16384 tokens, 1.5B shape): not
+    the headline metric; used for the prefill kernels' measurements."""
+    import torch
+    from hybrid_linear_top_b200 import lisa as L
+    cfg = get_config("prefill_1p5b_16k")
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    rng = make_rng(cfg.seed, 0)
+    st = gen_step(cfg, rng, cfg.T)
+    tb = lambda z: torch.from_numpy(np.ascontiguousarray(z)).to("cuda", torch.bfloat16)
+    tf = lambda z: torch.from_numpy(np.ascontiguousarray(z)).to("cuda", torch.float32)
+    x = dict(q=tb(st.q), k=tb(st.k), v=tb(st.v), kidx=tb(st.kidx), qidx=tb(st.qidx), w=tf(st.w), lam=tf(st.lam))
+    lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.T, L.LISA_BF16)
+    ws = L.alloc_workspace(lay, cfg.T, L.LISA_OP_PREFILL)
+    out = torch.empty(cfg.B, cfg.T, cfg.Hq, cfg.d, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(cfg.B, cfg.T, cfg.Hkv, cfg.M, dtype=torch.int32, device="cuda")
+
+    def step():
+        L.lisa_prefill(lay, cfg.T, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], out, idx, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if int(lay.err_word.item()) != 0:
+        raise RuntimeError(f"device-side checks flagged the prefill (err word {int(lay.err_word.item())})")
+    if rank == 0:
+        print(json.dumps({"metric": "LISA prefill tokens/s @16K, M=256", "value": cfg.T * cfg.B / (ms / 1e3),
+                          "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                          "config": {"workload": "prefill_1p5b_16k", "T": cfg.T, "M": cfg.M}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "prefill_1p5b_16k"])
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -372,6 +412,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload == "prefill_1p5b_16k":
+            run_prefill(args, rank, world)
         else:
             run_lisa(args, rank, world)
     finally:

@@ -89,6 +89,12 @@ cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, in
 // bf16 indexer scores of rows [tau0, tau0 + rows) of the pass on the tensor cores.
 cudaError_t launch_rows_score_tc(const RowsParams &p, cudaStream_t st, int tau0, int rows, int key_hi);
 cudaError_t launch_prefill_linear(const RowsParams &p, int dtype, cudaStream_t st);
+// bf16, d = 128: the chunked linear attention on the tensor cores (chunks of 128).
+cudaError_t launch_prefill_linear_tc(const RowsParams &p, cudaStream_t st);
+// Pieces shared by both chunked paths (d = 128): exclusive prefix of the chunk
+// increments dS over chunks of `chunk` tokens, and S_T = S_0 + total.
+cudaError_t launch_lin_prefix(const RowsParams &p, cudaStream_t st, int chunk);
+cudaError_t launch_lin_state(const RowsParams &p, cudaStream_t st);
 cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st);
 
 }  // namespace lisa

@@ -64,14 +64,15 @@ __global__ void __launch_bounds__(256) lin_dS_kernel(RowsParams p) {
     for (int bb = 0; bb < kB; ++bb) dst[(ti * kB + a) * D + tj * kB + bb] = acc[a][bb];
 }
 
-// grid (D*D/256, B*Hkv): exclusive prefix over chunks, in place; total -> Ptot
+// grid (D*D/256, B*Hkv): exclusive prefix over the chunks of `chunk` tokens,
+// in place; total -> Ptot
 template <int D>
-__global__ void __launch_bounds__(256) lin_prefix_kernel(RowsParams p) {
+__global__ void __launch_bounds__(256) lin_prefix_kernel(RowsParams p, int chunk) {
   const int e = blockIdx.x * 256 + threadIdx.x;
   const int bg = blockIdx.y;
   const int b = bg / p.Hkv;
   if (p.pos[b] != 0) return;
-  const int nc = (p.T + kLinChunk - 1) / kLinChunk;
+  const int nc = (p.T + chunk - 1) / chunk;
   float *base = p.dS + (size_t)bg * nc * D * D + e;
   float run = 0.f;
   constexpr int kBatch = 16;
@@ -218,15 +219,31 @@ static cudaError_t prefill_linear_t(const RowsParams &p, cudaStream_t st) {
   if ((e = prepare_kernel(lin_prefix_kernel<D>)) != cudaSuccess) return e;
   if ((e = prepare_kernel(lin_state_kernel<D>)) != cudaSuccess) return e;
   lin_dS_kernel<T, D><<<dim3(nc, p.B * p.Hkv), 256, smem1, st>>>(p);
-  lin_prefix_kernel<D><<<dim3(D * D / 256, p.B * p.Hkv), 256, 0, st>>>(p);
+  lin_prefix_kernel<D><<<dim3(D * D / 256, p.B * p.Hkv), 256, 0, st>>>(p, C);
   lin_out_kernel<T, D><<<dim3(nc, p.Hq, p.B), 256, smem3, st>>>(p);
   lin_state_kernel<D><<<dim3(D * D / 256, p.Hq, p.B), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
+cudaError_t launch_lin_prefix(const RowsParams &p, cudaStream_t st, int chunk) {
+  if (p.D != 128) return cudaErrorInvalidValue;
+  cudaError_t e = prepare_kernel(lin_prefix_kernel<128>);
+  if (e != cudaSuccess) return e;
+  lin_prefix_kernel<128><<<dim3(128 * 128 / 256, p.B * p.Hkv), 256, 0, st>>>(p, chunk);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lin_state(const RowsParams &p, cudaStream_t st) {
+  if (p.D != 128) return cudaErrorInvalidValue;
+  cudaError_t e = prepare_kernel(lin_state_kernel<128>);
+  if (e != cudaSuccess) return e;
+  lin_state_kernel<128><<<dim3(128 * 128 / 256, p.Hq, p.B), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prefill_linear(const RowsParams &p, int dtype, cudaStream_t st) {
   if (dtype == LISA_BF16) {
-    if (p.D == 128) return prefill_linear_t<__nv_bfloat16, 128>(p, st);
+    if (p.D == 128) return launch_prefill_linear_tc(p, st);
     if (p.D == 64) return prefill_linear_t<__nv_bfloat16, 64>(p, st);
   } else {
     if (p.D == 128) return prefill_linear_t<float, 128>(p, st);

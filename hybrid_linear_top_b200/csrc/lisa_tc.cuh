@@ -34,13 +34,34 @@ __device__ __forceinline__ void fence_async_shared() {
 }
 
 // ---------------------------------------------------------------- descriptors
-// Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D, M x N.
-__host__ __device__ constexpr uint32_t tc_idesc_bf16(int M, int N) {
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M x N; A / B
+// K-major unless a_mn / b_mn (then MN-major).
+__host__ __device__ constexpr uint32_t tc_idesc_bf16(int M, int N, bool a_mn = false, bool b_mn = false) {
   return (1u << 4)                       // D format: f32
          | (1u << 7)                     // A format: bf16
          | (1u << 10)                    // B format: bf16
+         | ((a_mn ? 1u : 0u) << 15)      // A major
+         | ((b_mn ? 1u : 0u) << 16)      // B major
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Shared-memory matrix descriptor of an MN-major operand with a 128-byte
+// swizzle: each 128-byte row holds 64 consecutive M (or N) elements of one K
+// index, 8 rows form a 1024-byte group (groups 1024 bytes apart), and the
+// next 64 M / N elements start `lbo_bytes` further.  +2048 bytes = +16 in K.
+__device__ __forceinline__ uint64_t tc_sdesc_mnmajor(uint32_t smem_addr, uint32_t lbo_bytes) {
+  const uint64_t start = (smem_addr & 0x3FFFFu) >> 4;
+  return start | ((uint64_t)(lbo_bytes >> 4) << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Byte offset of element (row, col) of a [rows][128] bf16 tile stored as two
+// 128-byte-swizzled halves of 64 columns (`half_bytes` apart) -- the layout
+// TMA writes with a {64, rows} box and the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int col, uint32_t half_bytes) {
+  const int half = col >> 6, cc = col & 63;
+  return (uint32_t)half * half_bytes + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+         (uint32_t)((((cc >> 3) ^ (row & 7)) << 4) + (cc & 7) * 2);
 }
 
 // Shared-memory matrix descriptor of a K-major operand whose rows are
@@ -83,6 +104,16 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t *r) {
 }
 __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 4-D tiled TMA load, coordinates from the innermost.
+__device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int c0, int c1, int c2, int c3,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // 3-D tiled TMA load, coordinates {innermost, middle, outer}.
