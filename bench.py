@@ -187,10 +187,11 @@ def cpu_baseline_sample(seconds=10.0):
 class Instance:
     """One independent layer at 16384 cached tokens, with its step inputs."""
 
-    def __init__(self, L, cfg, torch, seed, exact=None):
+    def __init__(self, L, cfg, torch, seed, exact=None, split=0):
         dev = "cuda"
         bf = torch.bfloat16
-        self.lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.L, L.LISA_BF16)
+        self.lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.L, L.LISA_BF16,
+                                    decode_split=split)
         n = cfg.L - 1
         if exact is not None:
             lay_np, st = exact
@@ -241,7 +242,7 @@ def run_lisa(args, rank, world):
 
     rng = make_rng(cfg.seed, 0)
     exact = (gen_layer(cfg, rng, cfg.L - 1), gen_step(cfg, rng, 1))
-    inst = [Instance(L, cfg, torch, 1000 * rank + i, exact if i == 0 else None) for i in range(R)]
+    inst = [Instance(L, cfg, torch, 1000 * rank + i, exact if i == 0 else None, args.split) for i in range(R)]
     ws = L.alloc_workspace(inst[0].lay, 1, L.LISA_OP_DECODE)
     torch.cuda.synchronize()
 
@@ -252,17 +253,33 @@ def run_lisa(args, rank, world):
         for i in range(args.warmup):
             inst[i % R].step(L, ws, stream)
     stream.synchronize()
-    rot = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(rot, stream=stream):
-        for i in range(R):
-            inst[i].step(L, ws, stream)
+    S = max(1, min(args.streams, R))
+    side = [torch.cuda.Stream() for _ in range(S)]
+
+    def capture(n):
+        # steps of instance i go to chain i % S; the S chains are independent
+        # (distinct layers) and join at the end of the graph
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            if S == 1:
+                for i in range(n):
+                    inst[i].step(L, ws, stream)
+            else:
+                fork = torch.cuda.Event()
+                fork.record(stream)
+                for s_ in side:
+                    s_.wait_event(fork)
+                for i in range(n):
+                    inst[i].step(L, ws, side[i % S])
+                for s_ in side:
+                    j = torch.cuda.Event()
+                    j.record(s_)
+                    stream.wait_event(j)
+        return g
+
+    rot = capture(R)
     n_rot, n_tail = divmod(args.steps, R)
-    tail = None
-    if n_tail:
-        tail = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(tail, stream=stream):
-            for i in range(n_tail):
-                inst[i].step(L, ws, stream)
+    tail = capture(n_tail) if n_tail else None
     for _ in range(2):
         rot.replay()
     torch.cuda.synchronize()
@@ -335,7 +352,7 @@ def run_lisa(args, rank, world):
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/sqrt(dim) caches and inputs; fp32 state ~ N(0,1))",
         "config": {"workload": WORKLOAD, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "HI": cfg.HI,
-                   "dI": cfg.dI, "M": cfg.M, "L": cfg.L, "instances": R,
+                   "dI": cfg.dI, "M": cfg.M, "L": cfg.L, "instances": R, "concurrent_chains": S,
                    "l2": "inputs larger than L2: rotation over instances touching "
                          f"{R * step_bytes / 2 ** 20:.0f} MiB (L2 {l2 / 2 ** 20:.0f} MiB)",
                    "parallelism": f"replicas x{world}"},
@@ -397,6 +414,8 @@ def main():
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "prefill_1p5b_16k"])
     ap.add_argument("--instances", type=int, default=0)
+    ap.add_argument("--streams", type=int, default=1)
+    ap.add_argument("--split", type=int, default=0, choices=[0, 4, 8, 16])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -36,7 +36,6 @@ size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int round4(int x) { return (x + 3) & ~3; }
 
-constexpr int kDecodeKeysCap = 32768;   // order keys staged in shared memory (1024-thread select)
 constexpr int kRowsKeysCap = 16384;     // same, for the 256-thread row select
 constexpr int kCandCap = 4096;          // threshold-bucket candidates kept in shared memory
 constexpr int kRowChunk = 2048;         // query rows scored per pass on the row path
@@ -57,6 +56,8 @@ lisa_status check_layer(const lisa_layer *L) {
   if (L->dI != 32 && L->dI != 64) return fail(LISA_ERR_UNSUPPORTED, "dI=%d not in {32,64}", L->dI);
   if (L->M % 32 || L->M < 32 || L->M > 1024) return fail(LISA_ERR_UNSUPPORTED, "M=%d not a multiple of 32 in [32,1024]", L->M);
   if ((long long)L->B * L->Hkv > 65535) return fail(LISA_ERR_UNSUPPORTED, "B*Hkv=%lld > 65535", (long long)L->B * L->Hkv);
+  if (L->decode_split != 0 && L->decode_split != 4 && L->decode_split != 8 && L->decode_split != 16)
+    return fail(LISA_ERR_INVALID_ARG, "decode_split=%d not in {0, 4, 8, 16}", L->decode_split);
   return LISA_OK;
 }
 
@@ -263,6 +264,7 @@ lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, 
   memset(&p, 0, sizeof(p));
   p.B = L->B; p.Hq = L->Hq; p.Hkv = L->Hkv; p.G = L->Hq / L->Hkv; p.HI = L->HI; p.R = L->HI / L->Hkv;
   p.D = L->d; p.DI = L->dI; p.M = L->M; p.L_max = L->L_max; p.fuse_append = fuse_append ? 1 : 0;
+  p.split_req = L->decode_split;
   p.scale = (float)(1.0 / sqrt((double)L->d));
   p.k_cache = L->k_cache; p.v_cache = L->v_cache; p.kidx_cache = L->kidx_cache;
   p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;

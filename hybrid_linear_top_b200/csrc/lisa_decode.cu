@@ -1,5 +1,5 @@
 // LISA decode step on sm_100a: one kernel, one thread-block cluster of NC CTAs
-// (NC = 16, or 8 where 16 cannot be scheduled) per (sequence b, KV head g).
+// (NC = 16, 8 or 4; see the launcher) per (sequence b, KV head g).
 //
 // Method: arXiv 2607.19358 (LISA).  Abstract: a Lightning Indexer keeps the
 // top-M tokens of the context for a sparse softmax attention, a linear
@@ -9,8 +9,9 @@
 //
 // Work of one cluster (CTA rank r of NC):
 //   1. stream its contiguous slice of the (b, g) indexer-key cache through a
-//      4-stage TMA ring and score every key, keeping 32-bit order keys in
-//      shared memory.  bf16: 2-D tiled TMA with a 64/128-byte swizzle and warp
+//      TMA ring and score every key, keeping 32-bit order keys in
+//      shared memory (NC = 16: 4 stages of 32 KB; NC <= 8: 2 stages, so two
+//      CTAs fit one SM).  bf16: 2-D tiled TMA with a 64/128-byte swizzle and warp
 //      tensor-core MMAs (keys x indexer heads); fp32: 1-D bulk copies and one
 //      thread per key on the CUDA cores.  Meanwhile the columns
 //      [r*d/NC, (r+1)*d/NC) of the linear state of the G query heads are
@@ -18,8 +19,10 @@
 //   2. exact top-M: every CTA takes the smallest of kl group maxima of its
 //      keys; if enough CTAs hold kl keys, the smallest of those values over
 //      the cluster is <= the M-th largest key, so only keys at or above it go
-//      to CTA 0, which selects exactly among them and emits the ascending
-//      index list.  When too many keys pass, a cluster-wide radix select
+//      to CTA 0 (each rank's in position order, in a segment of its own).
+//      CTA 0 finds the M-th key exactly with 1024-bin range histograms of the
+//      candidates and emits the ascending index list by an ordered
+//      compaction.  When a segment overflows, a cluster-wide radix select
 //      (histograms summed over distributed shared memory) runs instead;
 //   3. gather M/NC of the selected K/V rows, partial softmax for the G heads;
 //   4. merge the NC partials for its own column slice, apply the gate, store.
@@ -36,7 +39,7 @@ namespace cg = cooperative_groups;
 namespace lisa {
 
 constexpr int kDecThreads = 256;
-constexpr int kStages = 4;
+constexpr int kStages = 4;        // ring stages at most (the launcher picks 2 or 4)
 constexpr int kStageBytes = 32768;
 constexpr int kCandCap = 4096;   // candidate (key, position) pairs CTA 0 can hold
 
@@ -48,7 +51,7 @@ struct ScoreGeom {
 };
 
 struct DecLayout {
-  int region0, cand_key, cand_pos, gtb, eqb;
+  int region0, cand_key, cand_pos;
   int keys, hist, tot, misc, sel, qs, qi, ks, vs, part, pml, olin, logit, sidx, bars, total;
 };
 
@@ -57,24 +60,21 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // Byte offsets of the dynamic shared-memory carve-up, relative to a
 // 1024-byte aligned base (host and device agree; `total` includes the slack
 // needed to align the base).  region0 holds, one after the other in time: the
-// TMA ring (scoring), the candidate lists and position bitmaps (selection, in
-// CTA 0), and the gathered K / V rows (attention).
+// TMA ring (scoring), the candidate segments (selection, in CTA 0), and the
+// gathered K / V rows (attention).
 __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, int G, int D, int DI, int esize,
-                                                int NC) {
+                                                int NC, int stages = kStages) {
   DecLayout L;
   const int rpc = M / NC;
   const int kv = 2 * rpc * (D * esize + 16);
-  const int nw = (L_max + 31) / 32;
-  const int ring = kStages * kStageBytes;
-  const int sel_bytes = 8 * kCandCap + 2 * align16(nw * 4);
+  const int ring = stages * kStageBytes;
+  const int sel_bytes = 8 * kCandCap;
   int r0 = ring > kv ? ring : kv;
   r0 = r0 > sel_bytes ? r0 : sel_bytes;
   int off = 0;
   L.region0 = off; off += align16(r0);
   L.cand_key = L.region0;
   L.cand_pos = L.region0 + 4 * kCandCap;
-  L.gtb = L.region0 + 8 * kCandCap;
-  L.eqb = L.gtb + align16(nw * 4);
   L.keys = off; off += align16(kpc_max * 4);
   L.hist = off; off += 8 * 256 * 4;
   L.tot = off; off += 256 * 4;
@@ -130,43 +130,47 @@ __device__ __forceinline__ void dec_find_bucket(const uint32_t *tot, uint32_t *m
   }
 }
 
-// CTA-wide: the top 8*passes bits of the k-th largest of keys[0..cnt)
-// (1 <= k <= cnt), lower bits zero -- a lower bound of that key, exact when
-// passes == 4.  Histograms are kept per warp (hw[8][256]) so no warp-level
-// matching is needed.  All kDecThreads threads call it; uses tot[256] and
-// misc[0..1].
-__device__ uint32_t cta_kth_prefix(const uint32_t *keys, int cnt, uint32_t k, int passes, uint32_t *hw,
-                                   uint32_t *tot, uint32_t *misc) {
-  const int tid = threadIdx.x, warp = tid >> 5;
-  uint32_t prefix = 0, pmask = 0, rem = k;
-  for (int pass = 0; pass < passes; ++pass) {
-    const int shift = 24 - 8 * pass;
-    __syncthreads();                       // readers of the previous pass are done
-    for (int i = tid; i < 8 * 256; i += kDecThreads) hw[i] = 0;
-    if (tid == 0) misc[0] = 0xFFFFFFFFu;
-    __syncthreads();
-    for (int j = tid; j < cnt; j += kDecThreads) {
-      const uint32_t u = keys[j];
-      if ((u & pmask) == prefix) atomicAdd(&hw[warp * 256 + ((u >> shift) & 255u)], 1u);
-    }
-    __syncthreads();
-    {
-      uint32_t s = 0;
+// CTA-wide (kDecThreads = 256 threads, 4 bins each): the bin of fh[0..1024)
+// (higher bin = larger keys) that holds the rem-th largest key, counting from
+// the top.  misc[0] = bin (0xFFFFFFFF if the counts hold fewer than rem keys),
+// misc[1] = keys in higher bins, misc[2] = keys in the bin; misc[3] is zeroed.
+// Uses misc[8..15].  Ends with a barrier.
+__device__ void dec_find_bin1024(const uint32_t *fh, uint32_t rem, uint32_t *misc) {
+  static_assert(kDecThreads * 4 == 1024, "four bins per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b0 = 1023 - 4 * tid;
+  const uint32_t c0 = fh[b0], c1 = fh[b0 - 1], c2 = fh[b0 - 2], c3 = fh[b0 - 3];
+  const uint32_t c = c0 + c1 + c2 + c3;
+  uint32_t inc = c;
 #pragma unroll
-      for (int w8 = 0; w8 < 8; ++w8) s += hw[w8 * 256 + tid];
-      tot[tid] = s;
-    }
-    __syncthreads();
-    dec_find_bucket(tot, misc, rem);
-    __syncthreads();
-    const uint32_t dig = misc[0];
-    if (dig > 255u) break;                 // counts inconsistent (cannot happen); keep the bound found so far
-    rem -= misc[1];
-    prefix |= dig << shift;
-    pmask |= 255u << shift;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) misc[8 + warp] = inc;
+  if (tid == 0) {
+    misc[0] = 0xFFFFFFFFu;
+    misc[3] = 0;
   }
   __syncthreads();
-  return prefix;
+  uint32_t off = 0;
+#pragma unroll
+  for (int w8 = 0; w8 < kDecThreads / 32; ++w8) off += w8 < warp ? misc[8 + w8] : 0u;
+  const uint32_t exc = off + inc - c;
+  if (exc < rem && rem <= exc + c) {
+    const uint32_t cc[4] = {c0, c1, c2, c3};
+    uint32_t cum = exc;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (cum < rem && rem <= cum + cc[j]) {
+        misc[0] = (uint32_t)(b0 - j);
+        misc[1] = cum;
+        misc[2] = cc[j];
+      }
+      cum += cc[j];
+    }
+  }
+  __syncthreads();
 }
 
 // CTA-wide exclusive prefix sums of two counters, plus their totals.
@@ -204,7 +208,7 @@ __device__ __forceinline__ void cta_scan2(uint32_t a, uint32_t b, uint32_t &ea, 
 }
 
 template <typename T, int D, int DI, int NC>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 : 1)
     decode_cluster_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   using SG = ScoreGeom<T, DI>;
@@ -215,6 +219,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   constexpr int COLS = D / NC;                   // state / output columns of this CTA
   constexpr int QPR = COLS / 4;                  // float4 per state row slice
   constexpr int ITER = (D * QPR + kDecThreads - 1) / kDecThreads;
+  constexpr int HP = (16 / ITER) < 8 ? (16 / ITER < 1 ? 1 : 16 / ITER) : 8;   // state heads held in registers at once
   constexpr int ROWB = D * (int)sizeof(T);       // K / V row bytes
   constexpr int RS = ROWB + 16;                  // padded K / V row stride in shared memory
   constexpr int SL = ROWB / 16;                  // 16-byte slices per K / V row
@@ -229,7 +234,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // 1024-byte aligned base: the swizzled TMA tiles depend on address bits 4..9
   unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC);
+  const int NS = p.stages;
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC, NS);
   unsigned char *ring = smem + lay.region0;
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem + lay.keys);
   uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist);
@@ -268,16 +274,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // ---------------------------------------------------------------- TMA prologue
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % kStages
+  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS
     const int s_lo = k0 + i * SUB;
     const int s_hi = min(k1, s_lo + SUB);
     const int ncopy = max(0, min(s_hi, t) - s_lo);   // row t comes from the argument
-    uint64_t *bar = &bars[i % kStages];
-    unsigned char *dst = ring + (i % kStages) * kStageBytes;
+    uint64_t *bar = &bars[i % NS];
+    unsigned char *dst = ring + (i % NS) * kStageBytes;
     if (ncopy > 0) {
       if constexpr (SG::kMma) {
         mbar_arrive_expect_tx(bar, (uint32_t)(SUB * RB));   // the whole box lands, out-of-range rows zero
@@ -291,16 +297,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
   };
   if (tid == 0)
-    for (int i = 0; i < min(kStages, nsub); ++i) issue(i);
+    for (int i = 0; i < min(NS, nsub); ++i) issue(i);
 
   // ---------------------------------------------------------------- early loads
-  // state slab of the first (up to) 8 query heads: in flight during scoring
+  // state slab of the first (up to) HP query heads: in flight during scoring
   const int c0s = rank * COLS;
   const int cq = tid % QPR;                // same float4 column for every row this thread visits
-  const int gA = min(G, 8);
-  float4 sv[8][ITER];
+  const int gA = min(G, HP);
+  float4 sv[HP][ITER];
 #pragma unroll
-  for (int hh = 0; hh < 8; ++hh) {
+  for (int hh = 0; hh < HP; ++hh) {
     if (hh >= gA) continue;
     const float *S = p.state + ((size_t)b * p.Hq + g * G + hh) * D * D;
 #pragma unroll
@@ -351,8 +357,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // ---------------------------------------------------------------- indexer scores
   for (int i = 0; i < nsub; ++i) {
-    const int stage = i % kStages;
-    if (!mbar_wait_bounded(&bars[stage], (uint32_t)((i / kStages) & 1)) && tid == 0)
+    const int stage = i % NS;
+    if (!mbar_wait_bounded(&bars[stage], (uint32_t)((i / NS) & 1)) && tid == 0)
       set_err(p.err_word, LISA_DEVERR_TIMEOUT);
     const int s_lo = k0 + i * SUB;
     const int nk = min(k1, s_lo + SUB) - s_lo;
@@ -415,7 +421,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
     }
     __syncthreads();   // every thread is done with this stage
-    if (tid == 0 && i + kStages < nsub) issue(i + kStages);
+    if (tid == 0 && i + NS < nsub) issue(i + NS);
   }
   // the new token's score, from the argument row (its cache row may be stale)
   if (t >= k0 && t < k1 && warp == 0) {
@@ -436,12 +442,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     float vj[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) vj[j] = vs[c0s + cq * 4 + j];
-    float *red = logit;                  // scratch [8 heads][8 warps][COLS]
-    for (int h0 = 0; h0 < G; h0 += 8) {
-      const int hn = min(8, G - h0);
-      if (h0 > 0) {                      // heads beyond the first 8 are loaded now
+    float *red = logit;                  // scratch [HP heads][8 warps][COLS]
+    for (int h0 = 0; h0 < G; h0 += HP) {
+      const int hn = min(HP, G - h0);
+      if (h0 > 0) {                      // heads beyond the first HP are loaded now
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
+        for (int hh = 0; hh < HP; ++hh) {
           if (hh >= hn) continue;
           const float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
 #pragma unroll
@@ -454,7 +460,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       __syncthreads();                   // red is free
 #pragma unroll
-      for (int hh = 0; hh < 8; ++hh) {
+      for (int hh = 0; hh < HP; ++hh) {
         if (hh >= hn) continue;
         float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
         const float *qh = qs + (h0 + hh) * D;
@@ -507,8 +513,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   // ---------------------------------------------------------------- top-M
   int *sel0 = cluster.map_shared_rank(sel, 0);
   if (n > M) {
+    constexpr int SEG = kCandCap / NC;                  // candidate slots of each rank in CTA 0
+    uint32_t *fh = hist + 1024;                         // CTA 0: 1024-bin histogram of candidate keys
+    uint32_t *segp = tot + 64;                          // CTA 0: exclusive prefix of the segment sizes
+    uint32_t *misc0 = cluster.map_shared_rank(misc, 0);
     // (a) theta = the smallest of kl group maxima of this CTA's keys (groups:
     //     positions j = g (mod kl)); at least kl of its keys are >= theta.
+    //     Also the largest key, for the histogram range.
     int kl = 1;
     while (kl < (M + NC - 1) / NC) kl <<= 1;
     int covered = 0;
@@ -516,118 +527,206 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int cr = min(n, (r + 1) * kpc) - min(n, r * kpc);
       if (cr >= kl) covered += kl;
     }
-    uint32_t theta = 0xFFFFFFFFu;                       // neutral for the minimum
-    if (cnt >= kl) {
+    {
       uint32_t m = 0;
       for (int j = tid; j < cnt; j += kDecThreads) m = max(m, keys[j]);
       tot[tid] = m;                                     // thread tid holds group tid % kl
+      if (rank == 0)
+        for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
       __syncthreads();
-      if (tid < kl) {
+      if (cnt >= kl && tid < kl) {
         uint32_t gm = 0;
         for (int j = tid; j < kDecThreads; j += kl) gm = max(gm, tot[j]);
         hist[tid] = gm;
       }
       __syncthreads();
       if (warp == 0) {
-        uint32_t mn = 0xFFFFFFFFu;
-        for (int j = lane; j < kl; j += 32) mn = min(mn, hist[j]);
+        uint32_t mn = 0xFFFFFFFFu, mx = 0;              // 0xFFFFFFFF: neutral for the minimum
+        if (cnt >= kl)
+          for (int j = lane; j < kl; j += 32) mn = min(mn, hist[j]);
+        for (int j = lane; j < kDecThreads; j += 32) mx = max(mx, tot[j]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        theta = mn;
+        for (int o = 16; o > 0; o >>= 1) {
+          mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        if (lane == 0) {
+          misc[4] = mn;
+          misc[6] = mx;
+        }
       }
-    }
-    if (tid == 0) {
-      misc[4] = theta;
-      if (rank == 0) misc[5] = 0;                       // candidate counter in CTA 0
     }
     cluster.sync();                                     // bounds published, every ring is free
-    uint32_t lb = 0;
-    if (covered >= M) {
-      lb = 0xFFFFFFFFu;
-#pragma unroll
-      for (int r = 0; r < NC; ++r) lb = min(lb, cluster.map_shared_rank(misc, r)[4]);
-    }
-    // (b) keys >= lb go to CTA 0 (unordered): one slot reservation per warp
-    uint32_t *cnt0 = cluster.map_shared_rank(misc, 0) + 5;
-    uint32_t *ckey0 = cluster.map_shared_rank(reinterpret_cast<uint32_t *>(smem + lay.cand_key), 0);
-    int *cpos0 = cluster.map_shared_rank(reinterpret_cast<int *>(smem + lay.cand_pos), 0);
+    uint32_t lb = 0, hi = 0;
     {
-      const int iters = (cnt + kDecThreads - 1) / kDecThreads;
-      const unsigned lt = (1u << lane) - 1u;
-      uint32_t wc = 0;
-      for (int it = 0; it < iters; ++it) {
-        const int j = tid + it * kDecThreads;
-        wc += __popc(__ballot_sync(0xffffffffu, j < cnt && keys[j] >= lb));
+      uint32_t mn = 0xFFFFFFFFu;
+#pragma unroll
+      for (int r = 0; r < NC; ++r) {
+        const uint32_t *mr = cluster.map_shared_rank(misc, r);
+        mn = min(mn, mr[4]);
+        hi = max(hi, mr[6]);
       }
-      uint32_t off = 0;
-      if (lane == 0 && wc) off = atomicAdd(cnt0, wc);
-      off = __shfl_sync(0xffffffffu, off, 0);
-      for (int it = 0; it < iters; ++it) {
-        const int j = tid + it * kDecThreads;
-        const bool act = j < cnt && keys[j] >= lb;
-        const unsigned am = __ballot_sync(0xffffffffu, act);
-        if (act) {
-          const uint32_t slot = off + __popc(am & lt);
-          if (slot < (uint32_t)kCandCap) {
-            ckey0[slot] = keys[j];
-            cpos0[slot] = k0 + j;
+      if (covered >= M) lb = mn;
+    }
+    // (b) keys >= lb go, in position order, to this rank's segment of CTA 0's
+    //     candidate list; segment sizes to misc0[48 + rank]
+    {
+      uint32_t *ck = cluster.map_shared_rank(reinterpret_cast<uint32_t *>(smem + lay.cand_key), 0) + rank * SEG;
+      int *cp = cluster.map_shared_rank(reinterpret_cast<int *>(smem + lay.cand_pos), 0) + rank * SEG;
+      const int cw = (((cnt + 7) / 8) + 31) & ~31;      // contiguous keys per warp
+      const int j0 = min(cnt, warp * cw), j1 = min(cnt, j0 + cw);
+      uint32_t wc = 0;
+      for (int base = j0; base < j1; base += 32) {
+        const int j = base + lane;
+        wc += __popc(__ballot_sync(0xffffffffu, j < j1 && keys[j] >= lb));
+      }
+      if (lane == 0) misc[24 + warp] = wc;
+      __syncthreads();
+      uint32_t off = 0, total = 0;
+#pragma unroll
+      for (int w8 = 0; w8 < kDecThreads / 32; ++w8) {
+        const uint32_t c = misc[24 + w8];
+        off += w8 < warp ? c : 0u;
+        total += c;
+      }
+      if (tid == 0) misc0[48 + rank] = total;
+      if (total <= (uint32_t)SEG) {
+        const unsigned lt = (1u << lane) - 1u;
+        for (int base = j0; base < j1; base += 32) {
+          const int j = base + lane;
+          const bool act = j < j1 && keys[j] >= lb;
+          const unsigned am = __ballot_sync(0xffffffffu, act);
+          if (act) {
+            const uint32_t o = off + __popc(am & lt);
+            ck[o] = keys[j];
+            cp[o] = k0 + j;
           }
+          off += __popc(am);
         }
-        off += __popc(am);
       }
     }
     cluster.sync();                                     // candidates complete
-    const uint32_t n_c = *cnt0;
-    if (n_c <= (uint32_t)kCandCap) {
+    bool fits = true;                                   // the same answer in every CTA
+#pragma unroll
+    for (int r = 0; r < NC; ++r) fits = fits && misc0[48 + r] <= (uint32_t)SEG;
+    if (fits) {
       if (rank == 0) {
-        // (c) CTA 0: exact M-th key among the candidates, then the selected
-        //     positions in ascending order through two position bitmaps
+        // (c) CTA 0: exact M-th key among the candidates (range histograms of
+        //     1024 bins over [lb, hi], narrowed until one bin holds <= 32 keys
+        //     or a single key value), then the ascending index list by an
+        //     ordered compaction of the candidates
         const uint32_t *ck = reinterpret_cast<const uint32_t *>(smem + lay.cand_key);
         const int *cp = reinterpret_cast<const int *>(smem + lay.cand_pos);
-        uint32_t *gtb = reinterpret_cast<uint32_t *>(smem + lay.gtb);
-        uint32_t *eqb = reinterpret_cast<uint32_t *>(smem + lay.eqb);
-        const uint32_t kstar = cta_kth_prefix(ck, (int)n_c, (uint32_t)M, 4, hist, tot, misc);
-        const int nw = (n + 31) >> 5;
-        for (int i = tid; i < nw; i += kDecThreads) {
-          gtb[i] = 0;
-          eqb[i] = 0;
-        }
-        __syncthreads();
-        for (int j = tid; j < (int)n_c; j += kDecThreads) {
-          const uint32_t u = ck[j];
-          const int pos = cp[j];
-          if (pos < 0 || pos >= n) {
-            set_err(p.err_word, LISA_DEVERR_CHECK);
-            continue;
+        if (warp == 0) {
+          const uint32_t v = lane < NC ? misc[48 + lane] : 0u;
+          uint32_t inc = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
           }
-          if (u > kstar) atomicOr(&gtb[pos >> 5], 1u << (pos & 31));
-          else if (u == kstar) atomicOr(&eqb[pos >> 5], 1u << (pos & 31));
+          if (lane < NC) segp[lane + 1] = inc;
+          if (lane == 0) segp[0] = 0;
         }
-        // each thread owns a run of bitmap words, in position order
-        const int wpt = (nw + kDecThreads - 1) / kDecThreads;
-        const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
         __syncthreads();
-        uint32_t cgt = 0, ceq = 0;
-        for (int w = w0; w < w1; ++w) {
-          cgt += __popc(gtb[w]);
-          ceq += __popc(eqb[w]);
+        const uint32_t n_c = segp[NC];
+        const uint32_t per = (n_c + kDecThreads - 1) / kDecThreads;
+        const uint32_t c_lo = min(n_c, (uint32_t)tid * per), c_hi = min(n_c, c_lo + per);
+        int r_lo = 0;
+#pragma unroll
+        for (int r = 1; r < NC; ++r) r_lo += segp[r] <= c_lo ? 1 : 0;
+        // candidates c_lo .. c_hi-1 of the concatenation, in order: f(slot)
+        auto for_run = [&](auto &&f) {
+          int r = r_lo;
+          for (uint32_t c = c_lo; c < c_hi; ++c) {
+            while (c >= segp[r + 1]) ++r;
+            f(r * SEG + (int)(c - segp[r]));
+          }
+        };
+        uint32_t lbx = lb, ubx = hi, rem = (uint32_t)M, kstar = 0, need_eq = 0;
+        uint32_t shx = (hi - lb) < 1024u ? 0u : (uint32_t)(32 - __clz(hi - lb)) - 10u;
+        bool found = false;
+#pragma unroll 1
+        for (int iter = 0; iter < 4 && !found; ++iter) {
+          if (iter > 0) {
+            for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
+            __syncthreads();
+          }
+          for_run([&](int slot) {
+            const uint32_t u = ck[slot];
+            if (u >= lbx && u <= ubx) atomicAdd(&fh[(u - lbx) >> shx], 1u);
+          });
+          __syncthreads();
+          dec_find_bin1024(fh, rem, misc);              // misc[0..2]; zeroes misc[3]
+          const uint32_t bin = misc[0];
+          if (bin > 1023u) break;                       // counts inconsistent: cannot happen
+          rem -= misc[1];
+          const uint32_t cb = misc[2];
+          const uint32_t blo = lbx + (bin << shx);
+          if (shx == 0) {                               // the bin is one key value
+            kstar = blo;
+            need_eq = rem;
+            found = true;
+          } else if (cb <= 32) {                        // rank the bin's keys in one warp
+            for_run([&](int slot) {
+              const uint32_t u = ck[slot];
+              if (u >= blo && u <= ubx && ((u - lbx) >> shx) == bin) {
+                const uint32_t s = atomicAdd(&misc[3], 1u);
+                if (s < 32) tot[s] = u;
+              }
+            });
+            __syncthreads();
+            if (warp == 0) {
+              const uint32_t x = lane < (int)cb ? tot[lane] : 0u;
+              uint32_t gt = 0, ge = 0;
+              for (int j = 0; j < (int)cb; ++j) {
+                const uint32_t y = __shfl_sync(0xffffffffu, x, j);
+                gt += y > x ? 1u : 0u;
+                ge += y >= x ? 1u : 0u;
+              }
+              if (lane < (int)cb && gt < rem && rem <= ge) {   // lanes holding the rem-th key agree
+                misc[5] = x;
+                misc[7] = rem - gt;
+              }
+            }
+            __syncthreads();
+            kstar = misc[5];
+            need_eq = misc[7];
+            found = true;
+          } else {                                      // narrow to the bin
+            const unsigned long long top = (unsigned long long)blo + (1ull << shx) - 1ull;
+            lbx = blo;
+            ubx = top < ubx ? (uint32_t)top : ubx;
+            shx = shx > 10u ? shx - 10u : 0u;
+          }
+          __syncthreads();                              // misc and the histogram are reused
         }
-        uint32_t eg, ee, tg, te;
-        cta_scan2(cgt, ceq, eg, ee, tg, te, misc);
-        const uint32_t need_eq = (uint32_t)M - tg;      // keys equal to K* still to take
-        for (int w = w0; w < w1; ++w) {
-          const uint32_t gb = gtb[w], eb = eqb[w];
-          uint32_t bits = gb | eb;
-          while (bits) {
-            const int bpos = __ffs(bits) - 1;
-            bits &= bits - 1;
-            const int pos = (w << 5) + bpos;
-            if ((gb >> bpos) & 1u) {
+        if (!found) {
+          if (tid == 0) set_err(p.err_word, LISA_DEVERR_CHECK);
+          for (int j = tid; j < M; j += kDecThreads) sel[j] = -1;
+        } else {
+          uint32_t cgt = 0, ceq = 0;
+          for_run([&](int slot) {
+            const uint32_t u = ck[slot];
+            cgt += u > kstar ? 1u : 0u;
+            ceq += u == kstar ? 1u : 0u;
+          });
+          uint32_t eg, ee, tg, te;
+          cta_scan2(cgt, ceq, eg, ee, tg, te, misc);
+          if (tid == 0 && (tg + need_eq != (uint32_t)M || te < need_eq)) set_err(p.err_word, LISA_DEVERR_CHECK);
+          for_run([&](int slot) {
+            const uint32_t u = ck[slot];
+            const int pos = cp[slot];
+            if (pos < 0 || pos >= n) {
+              set_err(p.err_word, LISA_DEVERR_CHECK);
+              return;
+            }
+            if (u > kstar) {
               const uint32_t o = eg + min(ee, need_eq);
               if (o < (uint32_t)M) sel[o] = pos;
               else set_err(p.err_word, LISA_DEVERR_CHECK);
               ++eg;
-            } else {
+            } else if (u == kstar) {
               if (ee < need_eq) {
                 const uint32_t o = eg + ee;
                 if (o < (uint32_t)M) sel[o] = pos;
@@ -635,7 +734,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
               }
               ++ee;
             }
-          }
+          });
         }
       }
     } else {
@@ -869,7 +968,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 template <typename T, int D, int DI, int NC>
 static cudaError_t launch_cluster_t(const DecodeParams &p, const CUtensorMap &kmap, cudaStream_t st) {
   auto kern = decode_cluster_kernel<T, D, DI, NC>;
-  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), NC);
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), NC, p.stages);
   cudaError_t e = prepare_kernel(kern, lay.total);
   if (e != cudaSuccess) return e;
   if (NC > 8) {
@@ -925,24 +1024,46 @@ static int pick_cluster(const DecodeParams &p) {
 
 template <typename T, int D, int DI>
 static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
-  // the cluster size depends on the device and the shared-memory footprint: cache per (device, footprint)
+  // whether 16-CTA clusters can be scheduled depends on the device and the
+  // shared-memory footprint: cache per (device, footprint)
   static int cache_dev[8] = {-1, -1, -1, -1, -1, -1, -1, -1};
-  static int cache_key[8], cache_nc[8];
+  static int cache_key[8], cache_ok16[8], cache_sms[8];
   static int next = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   const int key = p.L_max * 2 + (p.M << 20) + (p.G << 28);
-  int nc = 0;
+  int ok16 = -1, sms = 0;
   for (int i = 0; i < 8; ++i)
-    if (cache_dev[i] == dev && cache_key[i] == key) nc = cache_nc[i];
-  if (!nc) {
-    nc = pick_cluster<T, D, DI>(p);
+    if (cache_dev[i] == dev && cache_key[i] == key) {
+      ok16 = cache_ok16[i];
+      sms = cache_sms[i];
+    }
+  if (ok16 < 0) {
+    ok16 = pick_cluster<T, D, DI>(p) == 16 ? 1 : 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      sms = 148;
+    }
     const int slot = next++ & 7;
     cache_dev[slot] = dev;
     cache_key[slot] = key;
-    cache_nc[slot] = nc;
+    cache_ok16[slot] = ok16;
+    cache_sms[slot] = sms;
   }
+  // CTAs per (sequence, KV head): 16 keeps one small step short; with many
+  // (sequence, KV head) pairs in the launch, fewer CTAs per pair (two per SM)
+  // spend less SM time per step.
+  int nc = p.split_req;
+  if (nc == 0) {
+    const int pairs = p.B * p.Hkv;
+    nc = pairs * 16 <= sms ? 16 : pairs * 8 <= 2 * sms ? 8 : 4;
+  }
+  if (nc == 16 && !ok16) nc = 8;
+  if (nc == 4 && dec_layout((((p.L_max + 3) / 4) + 31) & ~31, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), 4, 2).total >
+                     227 * 1024)
+    nc = 8;
   p.nc = nc;
+  p.stages = nc == 16 ? 4 : 2;          // two CTAs per SM fit the smaller ring
   p.kpc_max = (((p.L_max + nc - 1) / nc) + 31) & ~31;
   CUtensorMap kmap;
   memset(&kmap, 0, sizeof(kmap));
@@ -953,6 +1074,7 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   if (nc == 16) return launch_cluster_t<T, D, DI, 16>(p, kmap, st);
+  if (nc == 4) return launch_cluster_t<T, D, DI, 4>(p, kmap, st);
   return launch_cluster_t<T, D, DI, 8>(p, kmap, st);
 }
 

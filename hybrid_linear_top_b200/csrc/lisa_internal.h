@@ -51,7 +51,9 @@ struct DecodeParams {
   void *out;
   int *idx_out;
   // launch geometry (filled by the launcher)
+  int split_req;                        // requested CTAs per (b, g): 0 (library's choice), 4, 8, 16
   int nc;                               // CTAs per cluster
+  int stages;                           // TMA ring stages (2 or 4)
   int kpc_max;                          // order keys per CTA, upper bound
 };
 

@@ -49,6 +49,7 @@ class LisaLayerC(ctypes.Structure):
         ("dtype", ctypes.c_int),
         ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("kidx_cache", ctypes.c_void_p),
         ("state", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("err_word", ctypes.c_void_p),
+        ("decode_split", ctypes.c_int),
     ]
 
 
@@ -131,17 +132,19 @@ class Layer:
 
     k_cache, v_cache [B, Hkv, L_max, d]; kidx_cache [B, Hkv, L_max, dI] in the
     storage dtype; state [B, Hq, d, d] fp32; pos [B] int32; err_word [1] int32
-    (all on one CUDA device)."""
+    (all on one CUDA device).  decode_split: CTAs per (sequence, KV head) of
+    the decode step (0 = the library's choice, or 4, 8, 16)."""
 
     def __init__(self, B, Hq, Hkv, d, HI, dI, M, L_max, dtype, k_cache, v_cache, kidx_cache, state, pos,
-                 err_word=None):
+                 err_word=None, decode_split=0):
         self.B, self.Hq, self.Hkv, self.d, self.HI, self.dI, self.M, self.L_max = B, Hq, Hkv, d, HI, dI, M, L_max
         self.dtype = dtype
         self.k_cache, self.v_cache, self.kidx_cache = k_cache, v_cache, kidx_cache
         self.state, self.pos, self.err_word = state, pos, err_word
+        self.decode_split = decode_split
 
     @classmethod
-    def allocate(cls, B, Hq, Hkv, d, HI, dI, M, L_max, dtype=LISA_BF16, device="cuda"):
+    def allocate(cls, B, Hq, Hkv, d, HI, dI, M, L_max, dtype=LISA_BF16, device="cuda", decode_split=0):
         tdt = TORCH_DTYPE[dtype]
         return cls(B, Hq, Hkv, d, HI, dI, M, L_max, dtype,
                    torch.zeros(B, Hkv, L_max, d, dtype=tdt, device=device),
@@ -149,13 +152,13 @@ class Layer:
                    torch.zeros(B, Hkv, L_max, dI, dtype=tdt, device=device),
                    torch.zeros(B, Hq, d, d, dtype=torch.float32, device=device),
                    torch.zeros(B, dtype=torch.int32, device=device),
-                   torch.zeros(1, dtype=torch.int32, device=device))
+                   torch.zeros(1, dtype=torch.int32, device=device), decode_split)
 
     def c_struct(self):
         return LisaLayerC(
             self.B, self.Hq, self.Hkv, self.d, self.HI, self.dI, self.M, self.L_max, self.dtype,
             _ptr(self.k_cache), _ptr(self.v_cache), _ptr(self.kidx_cache), _ptr(self.state), _ptr(self.pos),
-            _ptr(self.err_word),
+            _ptr(self.err_word), int(self.decode_split),
         )
 
     @property

@@ -97,6 +97,14 @@ typedef struct {
   const int *pos;    /* [B] device: position of the first new token of this call
                         (= tokens already cached) */
   int *err_word;     /* device int or NULL: LISA_DEVERR_* bits are ORed in */
+  int decode_split;  /* CTAs that share one (sequence, KV head) in lisa_decode_step:
+                        0 = the library's choice (16 when all of them fit on the
+                        device at once, else 8 or 4), or 4, 8, 16 (16 falls back
+                        to 8 where 16-CTA clusters cannot be scheduled, 4 to 8
+                        where its shared memory would not fit).  16 gives the
+                        shortest single step; 4 the least SM time per step when
+                        many steps run concurrently.  Results do not depend on it
+                        beyond float summation order.  Other calls ignore it. */
 } lisa_layer;
 
 /*

@@ -33,11 +33,12 @@ def f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def make_layer(L, cfg, L_max, layer_np=None, n_rows=0, poison=True, device="cuda"):
+def make_layer(L, cfg, L_max, layer_np=None, n_rows=0, poison=True, device="cuda", decode_split=0):
     """Allocate a lisa Layer; copy rows [0, n_rows) of the generated caches and
     S_0; fill the unused cache rows with NaN so stray reads show up."""
     lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, L_max,
-                           L.LISA_BF16 if cfg.dtype == "bf16" else L.LISA_FP32, device=device)
+                           L.LISA_BF16 if cfg.dtype == "bf16" else L.LISA_FP32, device=device,
+                           decode_split=decode_split)
     if poison:
         lay.k_cache.fill_(float("nan"))
         lay.v_cache.fill_(float("nan"))

@@ -21,11 +21,12 @@ def _replace(cfg, **kw):
 
 
 def run_decode(cfg, layer_np, step, pos, L_max, fuse_append=True, pre_append=False, exact_sets=False,
-               n_rows=None, reps=1):
-    """Run one decode step on the GPU and check it against the oracle."""
+               n_rows=None, reps=1, split=0):
+    """Run one decode step on the GPU and check it against the oracle
+    (split: CTAs per (sequence, KV head), 0 = the library's choice)."""
     B = cfg.B
     n_rows = int(pos.max()) if n_rows is None else n_rows
-    lay = make_layer(L, cfg, L_max, layer_np, n_rows=n_rows)
+    lay = make_layer(L, cfg, L_max, layer_np, n_rows=n_rows, decode_split=split)
     # rows >= pos[b] of a shorter sequence must not be read: poison them
     for b in range(B):
         lay.k_cache[b, :, int(pos[b]):] = float("nan")
@@ -72,36 +73,41 @@ def run_decode(cfg, layer_np, step, pos, L_max, fuse_append=True, pre_append=Fal
     return dict(ndiff=ndiff, errs=errs, lay=lay)
 
 
-def test_decode_1p5b_16k():
-    """Full-size single-layer decode step at 16384 cached tokens."""
+@pytest.mark.parametrize("split", [0, 4, 8, 16])
+def test_decode_1p5b_16k(split):
+    """Full-size single-layer decode step at 16384 cached tokens, for every
+    CTA split of a (sequence, KV head)."""
     cfg = get_config("decode_1p5b_16k")
     rng = make_rng(cfg.seed, 0)
     lay = gen_layer(cfg, rng, cfg.L - 1)
     step = gen_step(cfg, rng, 1)
     pos = decode_positions(cfg)
-    run_decode(cfg, lay, step, pos, cfg.L_max)
+    run_decode(cfg, lay, step, pos, cfg.L_max, split=split)
 
 
-def test_decode_7b_ragged_batch():
-    """B=32 ragged lengths in [4096, 16384]."""
+@pytest.mark.parametrize("split", [0, 16])
+def test_decode_7b_ragged_batch(split):
+    """B=32 ragged lengths in [4096, 16384] (the library's choice is 4 CTAs per
+    (sequence, KV head) here)."""
     cfg = get_config("ragged_7b_b32")
     rng = make_rng(cfg.seed, 0)
     lengths = gen_lengths(cfg, rng)
     lay = gen_layer(cfg, rng, cfg.L_hi - 1)
     step = gen_step(cfg, rng, 1)
     pos = decode_positions(cfg, lengths=lengths)
-    run_decode(cfg, lay, step, pos, cfg.L_max, n_rows=cfg.L_hi - 1)
+    run_decode(cfg, lay, step, pos, cfg.L_max, n_rows=cfg.L_hi - 1, split=split)
 
 
+@pytest.mark.parametrize("split", [0, 4])
 @pytest.mark.parametrize("L_ctx", [1, 2, 100, 255, 256, 257, 300, 4097])
-def test_decode_short_prefixes(L_ctx):
+def test_decode_short_prefixes(L_ctx, split):
     """Prefixes around M (all kept, exactly M, M+1) and t = 0."""
     cfg = _replace(get_config("decode_1p5b_16k"), B=2)
     rng = make_rng(100 + L_ctx, 0)
     lay = gen_layer(cfg, rng, 4096)
     step = gen_step(cfg, rng, 1)
     pos = np.array([L_ctx - 1, max(0, L_ctx // 2 - 1)], dtype=np.int64)
-    run_decode(cfg, lay, step, pos, 4200, n_rows=4096)
+    run_decode(cfg, lay, step, pos, 4200, n_rows=4096, split=split)
 
 
 def test_decode_twice_reuses_workspace():
@@ -112,7 +118,8 @@ def test_decode_twice_reuses_workspace():
     run_decode(cfg, lay, step, np.array([2999]), 3000, reps=3)
 
 
-def test_decode_exact_ties_integer_inputs():
+@pytest.mark.parametrize("split", [0, 4, 8])
+def test_decode_exact_ties_integer_inputs(split):
     """Small-integer indexer inputs make exact score ties (exactly representable
     in bf16 and summed exactly in fp32): the set must equal the oracle's with no
     borderline exemption (tie -> lower position)."""
@@ -125,7 +132,7 @@ def test_decode_exact_ties_integer_inputs():
     step.kidx = ir.integers(-1, 2, size=step.kidx.shape).astype(np.float32)
     step.qidx = ir.integers(-1, 2, size=step.qidx.shape).astype(np.float32)
     step.w = ir.integers(0, 3, size=step.w.shape).astype(np.float32)
-    res = run_decode(cfg, lay, step, np.array([4999, 3000]), 5000, exact_sets=True)
+    res = run_decode(cfg, lay, step, np.array([4999, 3000]), 5000, exact_sets=True, split=split)
     assert res["ndiff"] == 0
 
 
@@ -230,8 +237,9 @@ def test_decode_graph_replays_are_stable():
     torch.cuda.synchronize()
 
 
+@pytest.mark.parametrize("split", [0, 4, 8])
 @pytest.mark.parametrize("L_ctx", [16384, 3000])
-def test_decode_all_scores_equal(L_ctx):
+def test_decode_all_scores_equal(L_ctx, split):
     """w = 0 makes every score 0: the first M positions must be selected (the
     tie rule), and at 16384 tokens every key passes the candidate bound, which
     exercises the cluster-wide radix path."""
@@ -240,5 +248,5 @@ def test_decode_all_scores_equal(L_ctx):
     lay = gen_layer(cfg, rng, L_ctx - 1)
     step = gen_step(cfg, rng, 1)
     step.w = np.zeros_like(step.w)
-    res = run_decode(cfg, lay, step, np.array([L_ctx - 1]), L_ctx, exact_sets=True)
+    res = run_decode(cfg, lay, step, np.array([L_ctx - 1]), L_ctx, exact_sets=True, split=split)
     assert res["ndiff"] == 0
