@@ -5,11 +5,17 @@ Workload: the Qwen2.5-1.5B-shaped single-layer decode step (B=1, 12 query /
 One step = one lisa_decode_step call: indexer over all 16384 keys, top-M,
 sparse attention, linear-state update and gate.
 
-The timed region replays a CUDA graph of K steps that rotates over R
-independent layer instances whose touched bytes exceed 4x the L2 size, so the
-traffic is HBM traffic.  value = tokens/s over all ranks (B tokens per step).
+The timed region replays CUDA graphs of exactly K steps that rotate over R
+independent layer instances whose touched bytes exceed 4x the L2 size (so
+the traffic is HBM traffic), in S concurrent chains (instance i in chain
+i mod S; steps of different instances are independent, like the layers of
+independent sequences).  value = tokens/s over all ranks (B tokens per
+step).  Also reported: the latency of one step run alone
+(latency_us_one_step) and the end-to-end rate with every step's inputs
+copied from pinned host memory and its output copied back (e2e).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lisa|reference]
+                  [--streams S] [--split 0|4|8|16] [--workload prefill_1p5b_16k]
 
 --impl reference times the fp64 CPU oracle on the host cores (bounded
 sample), the only reference this method has.
@@ -18,6 +24,9 @@ sample), the only reference this method has.
 import argparse
 import json
 import os
+
+# hardware work queues for the concurrent chains (read when CUDA starts)
+os.environ.setdefault("CUDA_DEVICE_MAX_CONNECTIONS", "32")
 import statistics
 import subprocess
 import sys
@@ -34,6 +43,10 @@ from lisa_inputs.gen import decode_positions  # noqa: E402
 
 METRIC = "LISA decode-attn tokens/s @16K ctx, M=256; % of HBM roofline"
 WORKLOAD = "decode_1p5b_16k"
+# DRAM bytes (read + write) of one decode launch from an ncu capture of this
+# kernel on this workload, by CTA split (the ncu summary under profiles/);
+# None where no capture of the current kernel exists.
+DECODE_TRAFFIC = {4: 5346816, 8: None, 16: None, 0: None}
 
 
 def algorithmic_bytes(cfg, L, esize=2):
@@ -184,8 +197,19 @@ def cpu_baseline_sample(seconds=10.0):
 
 
 # ---------------------------------------------------------------- lisa arm
+# packed per-step inputs of one instance: (name, elements per sequence, bf16?)
+def _input_layout(cfg):
+    return [("q", cfg.Hq * cfg.d, True), ("k", cfg.Hkv * cfg.d, True), ("v", cfg.Hkv * cfg.d, True),
+            ("kidx", cfg.Hkv * cfg.dI, True), ("qidx", cfg.HI * cfg.dI, True), ("w", cfg.HI, False),
+            ("lam", cfg.Hq, False)]
+
+
 class Instance:
-    """One independent layer at 16384 cached tokens, with its step inputs."""
+    """One independent layer at 16384 cached tokens, with its step inputs.
+
+    The step inputs live in one device buffer (16-byte aligned segments) so
+    that the end-to-end run can refill them with a single host-to-device copy
+    per step."""
 
     def __init__(self, L, cfg, torch, seed, exact=None, split=0):
         dev = "cuda"
@@ -193,6 +217,19 @@ class Instance:
         self.lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.L, L.LISA_BF16,
                                     decode_split=split)
         n = cfg.L - 1
+        segs, off = {}, 0
+        for name, nel, is_bf in _input_layout(cfg):
+            nb = cfg.B * nel * (2 if is_bf else 4)
+            segs[name] = (off, nb, is_bf)
+            off += (nb + 15) // 16 * 16
+        self.in_bytes = off
+        self.inbuf = torch.zeros(off, dtype=torch.uint8, device=dev)
+        shapes = {"q": (cfg.B, cfg.Hq, cfg.d), "k": (cfg.B, cfg.Hkv, cfg.d), "v": (cfg.B, cfg.Hkv, cfg.d),
+                  "kidx": (cfg.B, cfg.Hkv, cfg.dI), "qidx": (cfg.B, cfg.HI, cfg.dI), "w": (cfg.B, cfg.HI),
+                  "lam": (cfg.B, cfg.Hq)}
+        for name, (o, nb, is_bf) in segs.items():
+            view = self.inbuf[o:o + nb].view(bf if is_bf else torch.float32).view(shapes[name])
+            setattr(self, name, view)
         if exact is not None:
             lay_np, st = exact
             tb = lambda z: torch.from_numpy(np.ascontiguousarray(z)).to(dev, bf)
@@ -202,9 +239,10 @@ class Instance:
             self.lay.kidx_cache[:, :, :n] = tb(lay_np.kidx_cache)
             self.lay.state.copy_(tf(lay_np.S0))
             s0 = lambda z: z[:, 0]
-            self.q, self.k, self.v = tb(s0(st.q)), tb(s0(st.k)), tb(s0(st.v))
-            self.kidx, self.qidx = tb(s0(st.kidx)), tb(s0(st.qidx))
-            self.w, self.lam = tf(s0(st.w)), tf(s0(st.lam))
+            for name in ("q", "k", "v", "kidx", "qidx"):
+                getattr(self, name).copy_(tb(s0(getattr(st, name))))
+            self.w.copy_(tf(s0(st.w)))
+            self.lam.copy_(tf(s0(st.lam)))
         else:
             g = torch.Generator(device=dev)
             g.manual_seed(seed)
@@ -213,18 +251,67 @@ class Instance:
             self.lay.v_cache[:, :, :n] = rn((cfg.B, cfg.Hkv, n, cfg.d), cfg.d)
             self.lay.kidx_cache[:, :, :n] = rn((cfg.B, cfg.Hkv, n, cfg.dI), cfg.dI)
             self.lay.state.copy_(torch.randn(self.lay.state.shape, generator=g, device=dev))
-            self.q, self.k, self.v = (rn((cfg.B, cfg.Hq, cfg.d), cfg.d), rn((cfg.B, cfg.Hkv, cfg.d), cfg.d),
-                                      rn((cfg.B, cfg.Hkv, cfg.d), cfg.d))
-            self.kidx, self.qidx = rn((cfg.B, cfg.Hkv, cfg.dI), cfg.dI), rn((cfg.B, cfg.HI, cfg.dI), cfg.dI)
-            self.w = torch.rand((cfg.B, cfg.HI), generator=g, device=dev)
-            self.lam = torch.randn((cfg.B, cfg.Hq), generator=g, device=dev)
+            for name in ("q", "k", "v"):
+                getattr(self, name).copy_(rn(shapes[name], cfg.d))
+            self.kidx.copy_(rn(shapes["kidx"], cfg.dI))
+            self.qidx.copy_(rn(shapes["qidx"], cfg.dI))
+            self.w.copy_(torch.rand(shapes["w"], generator=g, device=dev))
+            self.lam.copy_(torch.randn(shapes["lam"], generator=g, device=dev))
         self.lay.pos.fill_(n)
         self.out = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=bf, device=dev)
         self.idx = torch.empty(cfg.B, cfg.Hkv, cfg.M, dtype=torch.int32, device=dev)
+        self.host_in = None
 
     def step(self, L, ws, stream=None):
         L.lisa_decode_step(self.lay, self.q, self.k, self.v, self.kidx, self.qidx, self.w, self.lam, 1, self.out,
                            self.idx, ws, stream)
+
+    def step_e2e(self, L, ws, stream):
+        """Host -> device copy of the step's inputs, the decode call, and the
+        output back to host memory (pinned buffers)."""
+        self.inbuf.copy_(self.host_in, non_blocking=True)
+        L.lisa_decode_step(self.lay, self.q, self.k, self.v, self.kidx, self.qidx, self.w, self.lam, 1, self.out,
+                           None, ws, stream)
+        self.host_out.copy_(self.out, non_blocking=True)
+
+
+def _capture(torch, stream, chains, items, fn):
+    """CUDA graph of fn(item, chain stream) over items; item i goes to chain
+    i % len(chains); the chains are independent and join at the end."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        if len(chains) == 1:
+            for it in items:
+                fn(it, stream)
+        else:
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            for s_ in chains:
+                s_.wait_event(fork)
+            for i, it in enumerate(items):
+                fn(it, chains[i % len(chains)])
+            for s_ in chains:
+                j = torch.cuda.Event()
+                j.record(s_)
+                stream.wait_event(j)
+    return g
+
+
+def _timed_replays(torch, stream, graphs, barrier=None):
+    """Device time (ms) of replaying `graphs` once each, in order."""
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for g in graphs:
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    return e0.elapsed_time(e1)
 
 
 def run_lisa(args, rank, world):
@@ -239,6 +326,7 @@ def run_lisa(args, rank, world):
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
     step_bytes = algorithmic_bytes(cfg, cfg.L)
     R = max(args.instances, int(np.ceil(4 * l2 / step_bytes)))
+    barrier = dist.barrier if world > 1 else None
 
     rng = make_rng(cfg.seed, 0)
     exact = (gen_layer(cfg, rng, cfg.L - 1), gen_step(cfg, rng, 1))
@@ -247,105 +335,76 @@ def run_lisa(args, rank, world):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
-    # warm-up (eager launches), then capture one rotation (R steps) and the
-    # K mod R tail as CUDA graphs; the timed region replays them for exactly K steps
+    S = max(1, min(args.streams, R))
+    chains = [torch.cuda.Stream() for _ in range(S)]
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             inst[i % R].step(L, ws, stream)
     stream.synchronize()
-    S = max(1, min(args.streams, R))
-    side = [torch.cuda.Stream() for _ in range(S)]
 
-    def capture(n):
-        # steps of instance i go to chain i % S; the S chains are independent
-        # (distinct layers) and join at the end of the graph
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            if S == 1:
-                for i in range(n):
-                    inst[i].step(L, ws, stream)
-            else:
-                fork = torch.cuda.Event()
-                fork.record(stream)
-                for s_ in side:
-                    s_.wait_event(fork)
-                for i in range(n):
-                    inst[i].step(L, ws, side[i % S])
-                for s_ in side:
-                    j = torch.cuda.Event()
-                    j.record(s_)
-                    stream.wait_event(j)
-        return g
-
-    rot = capture(R)
+    # ---- headline: exactly K steps, rotating over the R instances in S chains
     n_rot, n_tail = divmod(args.steps, R)
-    tail = capture(n_tail) if n_tail else None
+    run = lambda x, s_: x.step(L, ws, s_)
+    rot = _capture(torch, stream, chains, inst, run)
+    tail = _capture(torch, stream, chains, inst[:n_tail], run) if n_tail else None
     for _ in range(2):
         rot.replay()
     torch.cuda.synchronize()
-
     clk = ClockSampler(local)
     clk.start()
     time.sleep(0.2)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(n_rot):
-            rot.replay()
-        if tail is not None:
-            tail.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
+    ms = _timed_replays(torch, stream, [rot] * n_rot + ([tail] if tail else []), barrier)
     t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
-    ms = e0.elapsed_time(e1)
     clk.stop()
     if world > 1:
         t = torch.tensor([ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    steps_total = args.steps
-    ms_per_step = ms / steps_total
-    value = world * steps_total * cfg.B / (ms / 1e3)
+    ms_per_step = ms / args.steps
+    value = world * args.steps * cfg.B / (ms / 1e3)
+
+    # ---- one step at a time: the latency of a single decode step (one chain,
+    #      the library's CTA split for one sequence)
+    splits = [x.lay.decode_split for x in inst]
+    for x in inst:
+        x.lay.decode_split = 0
+    lat_steps = min(args.steps, 20 * R)
+    one = _capture(torch, stream, chains[:1], inst[:R] * (lat_steps // R), run)
+    one.replay()
+    lat_ms = _timed_replays(torch, stream, [one], barrier)
+    lat_us = lat_ms * 1e3 / (lat_steps // R * R)
+    for x, sp in zip(inst, splits):
+        x.lay.decode_split = sp
+    del one
 
     bad = [i for i, x in enumerate(inst) if int(x.lay.err_word.item()) != 0]
     if bad:
         raise RuntimeError(f"device-side checks flagged instances {bad[:8]} "
                            f"(err words {[int(inst[i].lay.err_word.item()) for i in bad[:8]]})")
 
-    # ---- end to end through the public call: pinned host inputs in, output out
-    host = {k: getattr(inst[0], k).cpu().pin_memory() for k in ["q", "k", "v", "kidx", "qidx", "w", "lam"]}
-    out_h = torch.empty_like(inst[0].out, device="cpu").pin_memory()
-    dev_in = {k: torch.empty_like(getattr(inst[0], k)) for k in host}
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size()
-    n_e2e = max(20, min(2000, args.steps))
-    with torch.cuda.stream(stream):
-        for it in range(n_e2e + 5):
-            if it == 5:
-                torch.cuda.synchronize()
-                t0 = time.perf_counter()
-            for k2 in host:
-                dev_in[k2].copy_(host[k2], non_blocking=True)
-            L.lisa_decode_step(inst[0].lay, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["kidx"], dev_in["qidx"],
-                               dev_in["w"], dev_in["lam"], 1, inst[0].out, None, ws, stream)
-            out_h.copy_(inst[0].out, non_blocking=True)
-            stream.synchronize()
-    e2e_s = (time.perf_counter() - t0) / n_e2e
-    e2e_val = world * cfg.B / e2e_s
+    # ---- end to end through the public call: every step copies its inputs
+    #      from pinned host memory and its output back (same chains)
+    for x in inst:
+        x.host_in = x.inbuf.cpu().pin_memory()
+        x.host_out = torch.empty(x.out.shape, dtype=x.out.dtype).pin_memory()
+    h2d = inst[0].in_bytes
+    d2h = inst[0].out.numel() * inst[0].out.element_size()
+    run_e2e = lambda x, s_: x.step_e2e(L, ws, s_)
+    rot_e = _capture(torch, stream, chains, inst, run_e2e)
+    rot_e.replay()
+    n_e = max(1, min(n_rot, 200))
+    e2e_ms = _timed_replays(torch, stream, [rot_e] * n_e, barrier)
+    e2e_val = world * n_e * R * cfg.B / (e2e_ms / 1e3)
+    del rot_e
 
-    # ---- parity of instance 0 (exact seeded inputs) against the oracle, small check
     peak, peak_kind = load_peaks()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     if rank != 0:
         return
     cpu = cpu_baseline_sample(args.cpu_seconds) if world == 1 and not args.no_cpu_baseline else None
     clocks = clk.summary(t_wall0, t_wall1)
+    split_used = args.split or "library"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -353,15 +412,19 @@ def run_lisa(args, rank, world):
         "data": "synthetic (seeded N(0,1)/sqrt(dim) caches and inputs; fp32 state ~ N(0,1))",
         "config": {"workload": WORKLOAD, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "d": cfg.d, "HI": cfg.HI,
                    "dI": cfg.dI, "M": cfg.M, "L": cfg.L, "instances": R, "concurrent_chains": S,
+                   "decode_split": split_used,
                    "l2": "inputs larger than L2: rotation over instances touching "
                          f"{R * step_bytes / 2 ** 20:.0f} MiB (L2 {l2 / 2 ** 20:.0f} MiB)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": "decode_cluster_kernel (whole decode step)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": step_bytes, "traffic": None},
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": step_bytes,
+                     "time_per_launch": "timed region / steps (steady state of the concurrent chains)",
+                     "traffic": DECODE_TRAFFIC.get(args.split)},
+        "latency_us_one_step": lat_us,
         "clocks": clocks,
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": steps_total,
+        "gpu_launches": args.steps,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -414,8 +477,8 @@ def main():
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "prefill_1p5b_16k"])
     ap.add_argument("--instances", type=int, default=0)
-    ap.add_argument("--streams", type=int, default=1)
-    ap.add_argument("--split", type=int, default=0, choices=[0, 4, 8, 16])
+    ap.add_argument("--streams", type=int, default=32)
+    ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
