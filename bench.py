@@ -325,7 +325,9 @@ def run_lisa(args, rank, world):
     props = torch.cuda.get_device_properties(local)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
     step_bytes = algorithmic_bytes(cfg, cfg.L)
-    R = max(args.instances, int(np.ceil(4 * l2 / step_bytes)))
+    S = max(1, args.streams)
+    R = max(args.instances, int(np.ceil(4 * l2 / step_bytes)), S)
+    R = -(-R // S) * S                  # each instance stays in one chain: S divides R
     barrier = dist.barrier if world > 1 else None
 
     rng = make_rng(cfg.seed, 0)
@@ -335,18 +337,21 @@ def run_lisa(args, rank, world):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
-    S = max(1, min(args.streams, R))
     chains = [torch.cuda.Stream() for _ in range(S)]
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             inst[i % R].step(L, ws, stream)
     stream.synchronize()
 
-    # ---- headline: exactly K steps, rotating over the R instances in S chains
-    n_rot, n_tail = divmod(args.steps, R)
+    # ---- headline: exactly K steps, rotating over the R instances in S chains;
+    #      one graph holds several rotations so that the chains stay full
+    #      between replays (each replay ends with a join of the chains)
+    per_graph = R * max(1, -(-2048 // R))
+    per_graph = min(per_graph, max(R, args.steps // R * R))
+    n_rot, n_tail = divmod(args.steps, per_graph)
     run = lambda x, s_: x.step(L, ws, s_)
-    rot = _capture(torch, stream, chains, inst, run)
-    tail = _capture(torch, stream, chains, inst[:n_tail], run) if n_tail else None
+    rot = _capture(torch, stream, chains, [inst[i % R] for i in range(per_graph)], run)
+    tail = _capture(torch, stream, chains, [inst[i % R] for i in range(n_tail)], run) if n_tail else None
     for _ in range(2):
         rot.replay()
     torch.cuda.synchronize()
@@ -391,11 +396,11 @@ def run_lisa(args, rank, world):
     h2d = inst[0].in_bytes
     d2h = inst[0].out.numel() * inst[0].out.element_size()
     run_e2e = lambda x, s_: x.step_e2e(L, ws, s_)
-    rot_e = _capture(torch, stream, chains, inst, run_e2e)
+    rot_e = _capture(torch, stream, chains, [inst[i % R] for i in range(per_graph)], run_e2e)
     rot_e.replay()
-    n_e = max(1, min(n_rot, 200))
+    n_e = max(1, min(n_rot, 20))
     e2e_ms = _timed_replays(torch, stream, [rot_e] * n_e, barrier)
-    e2e_val = world * n_e * R * cfg.B / (e2e_ms / 1e3)
+    e2e_val = world * n_e * per_graph * cfg.B / (e2e_ms / 1e3)
     del rot_e
 
     peak, peak_kind = load_peaks()
@@ -472,7 +477,7 @@ def run_prefill(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--steps", type=int, default=200000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "prefill_1p5b_16k"])

@@ -278,10 +278,15 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS
+  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS, and sub-chunk i + NS -> L2
     const int s_lo = k0 + i * SUB;
     const int s_hi = min(k1, s_lo + SUB);
     const int ncopy = max(0, min(s_hi, t) - s_lo);   // row t comes from the argument
+    {
+      const int p_lo = s_lo + NS * SUB;
+      const int np = max(0, min(min(k1, p_lo + SUB), t) - p_lo);
+      if (np > 0) bulk_prefetch_l2(kidx_cache + (size_t)p_lo * DI, (uint32_t)(np * RB));
+    }
     uint64_t *bar = &bars[i % NS];
     unsigned char *dst = ring + (i % NS) * kStageBytes;
     if (ncopy > 0) {
@@ -298,7 +303,6 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   };
   if (tid == 0)
     for (int i = 0; i < min(NS, nsub); ++i) issue(i);
-
   // ---------------------------------------------------------------- early loads
   // state slab of the first (up to) HP query heads: in flight during scoring
   const int c0s = rank * COLS;
@@ -315,6 +319,9 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       if (idx < D * QPR) sv[hh][it] = *reinterpret_cast<const float4 *>(S + (size_t)(idx / QPR) * D + c0s + cq * 4);
     }
   }
+  // heads beyond the first HP: their slab rows requested into L2 now
+  for (int i = tid; i < (G - gA) * D; i += kDecThreads)
+    prefetch_l2(p.state + ((size_t)b * p.Hq + g * G + gA + i / D) * D * D + (size_t)(i % D) * D + c0s);
   const T *qin = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + g * G) * D;
   for (int i = tid; i < G * D; i += kDecThreads) qs[i] = Dt<T>::to_f(qin[i]);
   const T *kin = reinterpret_cast<const T *>(p.k) + (size_t)bg * D;
