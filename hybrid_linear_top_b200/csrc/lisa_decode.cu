@@ -40,13 +40,14 @@ namespace lisa {
 
 constexpr int kDecThreads = 256;
 constexpr int kStages = 4;        // ring stages at most (the launcher picks 2 or 4)
-constexpr int kStageBytes = 32768;
+constexpr int kStageBytes = 32768;  // ring stage size at most (the launcher picks 16 or 32 KB)
 constexpr int kCandCap = 4096;   // candidate (key, position) pairs CTA 0 can hold
 
 template <typename T, int DI>
 struct ScoreGeom {
   static constexpr int RB = DI * (int)sizeof(T);                              // key row bytes
-  static constexpr int SUB = (kStageBytes / RB) < 256 ? kStageBytes / RB : 256; // keys per ring stage
+  // keys per ring stage of `stage_bytes`
+  static __host__ __device__ int sub(int stage_bytes) { return (stage_bytes / RB) < 256 ? stage_bytes / RB : 256; }
   static constexpr bool kMma = sizeof(T) == 2;                                // bf16: swizzled tiles + MMA
 };
 
@@ -63,11 +64,11 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // TMA ring (scoring), the candidate segments (selection, in CTA 0), and the
 // gathered K / V rows (attention).
 __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, int G, int D, int DI, int esize,
-                                                int NC, int stages = kStages) {
+                                                int NC, int stages = kStages, int stage_bytes = kStageBytes) {
   DecLayout L;
   const int rpc = M / NC;
   const int kv = 2 * rpc * (D * esize + 16);
-  const int ring = stages * kStageBytes;
+  const int ring = stages * stage_bytes;
   const int sel_bytes = 8 * kCandCap;
   int r0 = ring > kv ? ring : kv;
   r0 = r0 > sel_bytes ? r0 : sel_bytes;
@@ -213,7 +214,6 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   using SG = ScoreGeom<T, DI>;
   constexpr int RB = SG::RB;                     // indexer-key row bytes
-  constexpr int SUB = SG::SUB;                   // keys per ring stage
   constexpr int NCH = RB / 16;                   // 16-byte chunks per key row
   constexpr int VEC = 16 / (int)sizeof(T);       // elements per chunk
   constexpr int COLS = D / NC;                   // state / output columns of this CTA
@@ -235,7 +235,9 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   // 1024-byte aligned base: the swizzled TMA tiles depend on address bits 4..9
   unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const int NS = p.stages;
-  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC, NS);
+  const int SUB = p.stage_keys;                  // keys per ring stage
+  const int STB = SUB * RB;                      // bytes per ring stage
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC, NS, STB);
   unsigned char *ring = smem + lay.region0;
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem + lay.keys);
   uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist);
@@ -288,7 +290,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       if (np > 0) bulk_prefetch_l2(kidx_cache + (size_t)p_lo * DI, (uint32_t)(np * RB));
     }
     uint64_t *bar = &bars[i % NS];
-    unsigned char *dst = ring + (i % NS) * kStageBytes;
+    unsigned char *dst = ring + (i % NS) * STB;
     if (ncopy > 0) {
       if constexpr (SG::kMma) {
         mbar_arrive_expect_tx(bar, (uint32_t)(SUB * RB));   // the whole box lands, out-of-range rows zero
@@ -369,7 +371,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       set_err(p.err_word, LISA_DEVERR_TIMEOUT);
     const int s_lo = k0 + i * SUB;
     const int nk = min(k1, s_lo + SUB) - s_lo;
-    const unsigned char *st = ring + stage * kStageBytes;
+    const unsigned char *st = ring + stage * STB;
     if constexpr (SG::kMma) {
       // tiles of 16 keys; A = keys (row-major, swizzled by TMA), B = queries
       const uint32_t st_u32 = smem_u32(st);
@@ -893,27 +895,59 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     }
   }
   __syncthreads();
-  // logits[hh][r] = q_h . k_r / sqrt(d)
-  for (int i = tid; i < G * rpc; i += kDecThreads) {
-    const int hh = i / rpc, r = i % rpc;
-    float l = -INFINITY;
-    if (sidx[r] >= 0) {
-      const float *qh = qs + hh * D;
-      const unsigned char *kr = kvs + r * RS;
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll 4
-      for (int sl = 0; sl < SL; ++sl) {
-        float x[VEC];
-        Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(kr + sl * 16), x);
+  // bf16 with whole 16-row k-steps: both products on the tensor cores (warp
+  // MMAs; query heads are the 16 rows of the A operand)
+  const bool mma_attn = SG::kMma && (rpc % 16) == 0;
+  if (mma_attn) {
+    // logits[hh][r] = q_h . k_r / sqrt(d): A = q (heads x d), B = K rows (d x rows)
+    const int g4 = lane >> 2, t2 = (lane & 3) * 2;
+    const uint32_t kvs_u32 = smem_u32(kvs);
+    for (int nt = warp; nt < rpc / 8; nt += kDecThreads / 32) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < VEC; j += 2) {
-          a0 = fmaf(qh[sl * VEC + j], x[j], a0);
-          a1 = fmaf(qh[sl * VEC + j + 1], x[j + 1], a1);
+      for (int ks2 = 0; ks2 < D / 32; ++ks2) {
+        uint32_t bk[4];
+        ldmatrix_x4(kvs_u32 + (nt * 8 + (lane & 7)) * RS + ks2 * 64 + (lane >> 3) * 16, bk[0], bk[1], bk[2], bk[3]);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int k0q = (2 * ks2 + h2) * 16 + t2;
+          uint32_t a[4];
+          a[0] = g4 < G ? pack_bf16(qs[g4 * D + k0q], qs[g4 * D + k0q + 1]) : 0u;
+          a[1] = g4 + 8 < G ? pack_bf16(qs[(g4 + 8) * D + k0q], qs[(g4 + 8) * D + k0q + 1]) : 0u;
+          a[2] = g4 < G ? pack_bf16(qs[g4 * D + k0q + 8], qs[g4 * D + k0q + 9]) : 0u;
+          a[3] = g4 + 8 < G ? pack_bf16(qs[(g4 + 8) * D + k0q + 8], qs[(g4 + 8) * D + k0q + 9]) : 0u;
+          mma_16816_bf16(c, a, bk + 2 * h2);
         }
       }
-      l = (a0 + a1) * p.scale;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int hh = g4 + (j >> 1) * 8, r = nt * 8 + t2 + (j & 1);
+        if (hh < G) logit[hh * rpc + r] = sidx[r] >= 0 ? c[j] * p.scale : -INFINITY;
+      }
     }
-    logit[hh * rpc + r] = l;
+  } else {
+    // logits[hh][r] = q_h . k_r / sqrt(d)
+    for (int i = tid; i < G * rpc; i += kDecThreads) {
+      const int hh = i / rpc, r = i % rpc;
+      float l = -INFINITY;
+      if (sidx[r] >= 0) {
+        const float *qh = qs + hh * D;
+        const unsigned char *kr = kvs + r * RS;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+        for (int sl = 0; sl < SL; ++sl) {
+          float x[VEC];
+          Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(kr + sl * 16), x);
+#pragma unroll
+          for (int j = 0; j < VEC; j += 2) {
+            a0 = fmaf(qh[sl * VEC + j], x[j], a0);
+            a1 = fmaf(qh[sl * VEC + j + 1], x[j + 1], a1);
+          }
+        }
+        l = (a0 + a1) * p.scale;
+      }
+      logit[hh * rpc + r] = l;
+    }
   }
   __syncthreads();
   // per head: local max and sum of exponentials over this CTA's rows
@@ -935,14 +969,60 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     }
   }
   __syncthreads();
-  // part[hh][d] = sum_r e[hh][r] v_r[d]
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    const int hh = i / D, d = i % D;
-    const float *e = logit + hh * rpc;
-    const T *vcol = reinterpret_cast<const T *>(kvs + rpc * RS) + d;
-    float a = 0.f;
-    for (int r = 0; r < rpc; ++r) a = fmaf(e[r], Dt<T>::to_f(vcol[(size_t)r * (RS / sizeof(T))]), a);
-    part[i] = a;
+  if (mma_attn) {
+    // part[hh][d] = sum_r e[hh][r] v_r[d]: A = e (heads x rows) as bf16 hi + lo
+    // pairs, B = V rows (rows x d) through transposing matrix loads
+    const int g4 = lane >> 2, t2 = (lane & 3) * 2;
+    const uint32_t v_u32 = smem_u32(kvs + rpc * RS);
+    for (int np = warp; np < D / 16; np += kDecThreads / 32) {     // pairs of 8-column tiles
+      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int ks = 0; ks < rpc / 16; ++ks) {
+        uint32_t bv[4];
+        const int m = lane >> 3;
+        ldmatrix_x4_trans(v_u32 + (ks * 16 + (m & 1) * 8 + (lane & 7)) * RS + (np * 16 + (m >> 1) * 8) * 2, bv[0],
+                          bv[1], bv[2], bv[3]);
+        float e[8];
+        const int r0 = ks * 16 + t2;
+        e[0] = g4 < G ? logit[g4 * rpc + r0] : 0.f;
+        e[1] = g4 < G ? logit[g4 * rpc + r0 + 1] : 0.f;
+        e[2] = g4 + 8 < G ? logit[(g4 + 8) * rpc + r0] : 0.f;
+        e[3] = g4 + 8 < G ? logit[(g4 + 8) * rpc + r0 + 1] : 0.f;
+        e[4] = g4 < G ? logit[g4 * rpc + r0 + 8] : 0.f;
+        e[5] = g4 < G ? logit[g4 * rpc + r0 + 9] : 0.f;
+        e[6] = g4 + 8 < G ? logit[(g4 + 8) * rpc + r0 + 8] : 0.f;
+        e[7] = g4 + 8 < G ? logit[(g4 + 8) * rpc + r0 + 9] : 0.f;
+        uint32_t ahi[4], alo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          ahi[j] = pack_bf16(e[2 * j], e[2 * j + 1]);
+          const float h0 = __bfloat162float(__float2bfloat16_rn(e[2 * j]));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(e[2 * j + 1]));
+          alo[j] = pack_bf16(e[2 * j] - h0, e[2 * j + 1] - h1);
+        }
+        mma_16816_bf16(c0, ahi, bv);
+        mma_16816_bf16(c0, alo, bv);
+        mma_16816_bf16(c1, ahi, bv + 2);
+        mma_16816_bf16(c1, alo, bv + 2);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int hh = g4 + (j >> 1) * 8, d = np * 16 + t2 + (j & 1);
+        if (hh < G) {
+          part[hh * D + d] = c0[j];
+          part[hh * D + d + 8] = c1[j];
+        }
+      }
+    }
+  } else {
+    // part[hh][d] = sum_r e[hh][r] v_r[d]
+    for (int i = tid; i < G * D; i += kDecThreads) {
+      const int hh = i / D, d = i % D;
+      const float *e = logit + hh * rpc;
+      const T *vcol = reinterpret_cast<const T *>(kvs + rpc * RS) + d;
+      float a = 0.f;
+      for (int r = 0; r < rpc; ++r) a = fmaf(e[r], Dt<T>::to_f(vcol[(size_t)r * (RS / sizeof(T))]), a);
+      part[i] = a;
+    }
   }
   cluster.sync();                            // all partials of the cluster are ready
 
@@ -975,7 +1055,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
 template <typename T, int D, int DI, int NC>
 static cudaError_t launch_cluster_t(const DecodeParams &p, const CUtensorMap &kmap, cudaStream_t st) {
   auto kern = decode_cluster_kernel<T, D, DI, NC>;
-  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), NC, p.stages);
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), NC, p.stages,
+                                   p.stage_keys * ScoreGeom<T, DI>::RB);
   cudaError_t e = prepare_kernel(kern, lay.total);
   if (e != cudaSuccess) return e;
   if (NC > 8) {
@@ -1070,14 +1151,16 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
                      227 * 1024)
     nc = 8;
   p.nc = nc;
-  p.stages = nc == 16 ? 4 : 2;          // two CTAs per SM fit the smaller ring
+  // 16 CTAs: 4 stages of 32 KB; fewer: 2 stages, so two CTAs fit one SM
+  p.stages = nc == 16 ? 4 : 2;
+  p.stage_keys = ScoreGeom<T, DI>::sub(32768);
   p.kpc_max = (((p.L_max + nc - 1) / nc) + 31) & ~31;
   CUtensorMap kmap;
   memset(&kmap, 0, sizeof(kmap));
   if (ScoreGeom<T, DI>::kMma) {
     using SG = ScoreGeom<T, DI>;
     if (!make_tmap_2d(&kmap, p.kidx_cache, (int)sizeof(T), (unsigned long long)DI,
-                      (unsigned long long)p.B * p.Hkv * p.L_max, (unsigned long long)SG::RB, DI, SG::SUB, SG::RB))
+                      (unsigned long long)p.B * p.Hkv * p.L_max, (unsigned long long)SG::RB, DI, p.stage_keys, SG::RB))
       return cudaErrorInvalidValue;
   }
   if (nc == 16) return launch_cluster_t<T, D, DI, 16>(p, kmap, st);

@@ -53,7 +53,8 @@ struct DecodeParams {
   // launch geometry (filled by the launcher)
   int split_req;                        // requested CTAs per (b, g): 0 (library's choice), 4, 8, 16
   int nc;                               // CTAs per cluster
-  int stages;                           // TMA ring stages (2 or 4)
+  int stages;                           // TMA ring stages
+  int stage_keys;                       // keys per ring stage
   int kpc_max;                          // order keys per CTA, upper bound
 };
 
