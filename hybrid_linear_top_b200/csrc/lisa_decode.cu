@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   if (tid == 0)
     for (int i = 0; i < min(NS, nsub); ++i) issue(i);
   // ---------------------------------------------------------------- early loads
-  // state slab of the first (up to) HP query heads: in flight during scoring
+  // state slab of the first (up to) HP query heads
   const int c0s = rank * COLS;
   const int cq = tid % QPR;                // same float4 column for every row this thread visits
   const int gA = min(G, HP);
@@ -363,6 +363,80 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     for (int i = tid; i < DI; i += kDecThreads) kic[i] = kidx_new[i];
   }
   __syncthreads();
+
+  // ---------------------------------------------------------------- linear state
+  // S_h <- S_h + k^T v on columns [c0s, c0s + COLS); o_lin[h][c] = sum_i q_h[i] S_h[i][c].
+  // Runs while the first key stages are in flight.
+  {
+    float vj[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) vj[j] = vs[c0s + cq * 4 + j];
+    float *red = logit;                  // scratch [HP heads][8 warps][COLS]
+    for (int h0 = 0; h0 < G; h0 += HP) {
+      const int hn = min(HP, G - h0);
+      if (h0 > 0) {                      // heads beyond the first HP are loaded now
+#pragma unroll
+        for (int hh = 0; hh < HP; ++hh) {
+          if (hh >= hn) continue;
+          const float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
+#pragma unroll
+          for (int it = 0; it < ITER; ++it) {
+            const int idx = tid + it * kDecThreads;
+            if (idx < D * QPR)
+              sv[hh][it] = *reinterpret_cast<const float4 *>(S + (size_t)(idx / QPR) * D + c0s + cq * 4);
+          }
+        }
+      }
+      __syncthreads();                   // red is free
+#pragma unroll
+      for (int hh = 0; hh < HP; ++hh) {
+        if (hh >= hn) continue;
+        float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
+        const float *qh = qs + (h0 + hh) * D;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int it = 0; it < ITER; ++it) {
+          const int idx = tid + it * kDecThreads;
+          if (idx < D * QPR) {
+            const int i = idx / QPR;
+            const float ki = ks[i], qi = qh[i];
+            float4 sn = sv[hh][it];
+            sn.x = fmaf(ki, vj[0], sn.x);
+            sn.y = fmaf(ki, vj[1], sn.y);
+            sn.z = fmaf(ki, vj[2], sn.z);
+            sn.w = fmaf(ki, vj[3], sn.w);
+            *reinterpret_cast<float4 *>(S + (size_t)i * D + c0s + cq * 4) = sn;
+            a0 = fmaf(qi, sn.x, a0);
+            a1 = fmaf(qi, sn.y, a1);
+            a2 = fmaf(qi, sn.z, a2);
+            a3 = fmaf(qi, sn.w, a3);
+          }
+        }
+#pragma unroll
+        for (int o = QPR; o < 32; o <<= 1) {
+          a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+          a3 += __shfl_xor_sync(0xffffffffu, a3, o);
+        }
+        if (lane < QPR) {
+          float *rw = red + (hh * 8 + warp) * COLS + lane * 4;
+          rw[0] = a0;
+          rw[1] = a1;
+          rw[2] = a2;
+          rw[3] = a3;
+        }
+      }
+      __syncthreads();
+      for (int i = tid; i < hn * COLS; i += kDecThreads) {
+        const int hh = i / COLS, c = i % COLS;
+        float o = 0.f;
+#pragma unroll
+        for (int w8 = 0; w8 < 8; ++w8) o += red[(hh * 8 + w8) * COLS + c];
+        olin[(h0 + hh) * COLS + c] = o;
+      }
+    }
+  }
 
   // ---------------------------------------------------------------- indexer scores
   for (int i = 0; i < nsub; ++i) {
@@ -445,78 +519,6 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     if (lane == 0) keys[t - k0] = score_key(score);
   }
 
-  // ---------------------------------------------------------------- linear state
-  // S_h <- S_h + k^T v on columns [c0s, c0s + COLS); o_lin[h][c] = sum_i q_h[i] S_h[i][c]
-  {
-    float vj[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) vj[j] = vs[c0s + cq * 4 + j];
-    float *red = logit;                  // scratch [HP heads][8 warps][COLS]
-    for (int h0 = 0; h0 < G; h0 += HP) {
-      const int hn = min(HP, G - h0);
-      if (h0 > 0) {                      // heads beyond the first HP are loaded now
-#pragma unroll
-        for (int hh = 0; hh < HP; ++hh) {
-          if (hh >= hn) continue;
-          const float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
-#pragma unroll
-          for (int it = 0; it < ITER; ++it) {
-            const int idx = tid + it * kDecThreads;
-            if (idx < D * QPR)
-              sv[hh][it] = *reinterpret_cast<const float4 *>(S + (size_t)(idx / QPR) * D + c0s + cq * 4);
-          }
-        }
-      }
-      __syncthreads();                   // red is free
-#pragma unroll
-      for (int hh = 0; hh < HP; ++hh) {
-        if (hh >= hn) continue;
-        float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
-        const float *qh = qs + (h0 + hh) * D;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int it = 0; it < ITER; ++it) {
-          const int idx = tid + it * kDecThreads;
-          if (idx < D * QPR) {
-            const int i = idx / QPR;
-            const float ki = ks[i], qi = qh[i];
-            float4 sn = sv[hh][it];
-            sn.x = fmaf(ki, vj[0], sn.x);
-            sn.y = fmaf(ki, vj[1], sn.y);
-            sn.z = fmaf(ki, vj[2], sn.z);
-            sn.w = fmaf(ki, vj[3], sn.w);
-            *reinterpret_cast<float4 *>(S + (size_t)i * D + c0s + cq * 4) = sn;
-            a0 = fmaf(qi, sn.x, a0);
-            a1 = fmaf(qi, sn.y, a1);
-            a2 = fmaf(qi, sn.z, a2);
-            a3 = fmaf(qi, sn.w, a3);
-          }
-        }
-#pragma unroll
-        for (int o = QPR; o < 32; o <<= 1) {
-          a0 += __shfl_xor_sync(0xffffffffu, a0, o);
-          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
-          a3 += __shfl_xor_sync(0xffffffffu, a3, o);
-        }
-        if (lane < QPR) {
-          float *rw = red + (hh * 8 + warp) * COLS + lane * 4;
-          rw[0] = a0;
-          rw[1] = a1;
-          rw[2] = a2;
-          rw[3] = a3;
-        }
-      }
-      __syncthreads();
-      for (int i = tid; i < hn * COLS; i += kDecThreads) {
-        const int hh = i / COLS, c = i % COLS;
-        float o = 0.f;
-#pragma unroll
-        for (int w8 = 0; w8 < 8; ++w8) o += red[(hh * 8 + w8) * COLS + c];
-        olin[(h0 + hh) * COLS + c] = o;
-      }
-    }
-  }
   __syncthreads();
 
   // ---------------------------------------------------------------- top-M

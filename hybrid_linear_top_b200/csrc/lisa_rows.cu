@@ -6,6 +6,7 @@
 // attention, gated with a linear branch) and the gptget.net digest's method
 // section (ReLU dot-product indexer); exact formulas as stated in lisa.h.
 #include "lisa_internal.h"
+#include "lisa_common.cuh"
 #include "lisa_select.cuh"
 
 namespace lisa {
@@ -318,9 +319,252 @@ __global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
   }
 }
 
+// ------------------------------------------------------------ bf16 on warp MMAs
+// grid (T, B*Hkv); 4 warps.  Warp w owns selected rows [w*M/4, (w+1)*M/4) of
+// the (b, tau, g) list, in tiles of 16 rows staged by cp.async (two stages per
+// warp), flash-attention style: S = Q K^T with the G query heads as the 16 rows
+// of the A operand, online softmax in registers, O += P V with P as bf16
+// hi + lo pairs.  The 4 warps' (max, sum, O) are merged through shared memory,
+// then the gate mixes in o_lin.
+constexpr int kAttnWarps = 4;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int D>
+constexpr int attn_mma_smem() {
+  // per warp: 2 stages x (K, V) x 16 rows x (2D + 16) bytes; the merge reuses it
+  return kAttnWarps * 2 * 2 * 16 * (2 * D + 16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(RowsParams p) {
+  extern __shared__ __align__(16) unsigned char s_att[];
+  constexpr int RS = 2 * D + 16;                 // padded row stride (bytes)
+  constexpr int TILE = 16 * RS;                  // one 16-row K or V tile
+  constexpr int NT = D / 8;                      // 8-column output tiles
+  const int tau = blockIdx.x, bg = blockIdx.y;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  if (!rows_pos_ok(p, b)) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = p.G;
+  const int g4 = lane >> 2, t2 = (lane & 3) * 2;
+  const int RW = p.M / kAttnWarps;               // rows of this warp (a multiple of 16)
+  const int t_abs = p.pos[b] + tau;
+  unsigned char *wbuf = s_att + warp * 4 * TILE; // [stage][K | V]
+  const uint32_t wbuf_u32 = smem_u32(wbuf);
+  const int *idx = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M + warp * RW;
+  const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(p.k_cache) + (size_t)bg * p.L_max * D;
+  const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(p.v_cache) + (size_t)bg * p.L_max * D;
+
+  // A fragments of q (heads = rows, padded to 16), for every 16-wide k-step
+  uint32_t qa[D / 16][4];
+  {
+    const uint32_t *q32 = reinterpret_cast<const uint32_t *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
+                                                             (((size_t)b * p.T + tau) * p.Hq + g * G) * D);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const int k0 = ks * 16 + t2;
+      qa[ks][0] = g4 < G ? q32[(g4 * D + k0) >> 1] : 0u;
+      qa[ks][1] = g4 + 8 < G ? q32[((g4 + 8) * D + k0) >> 1] : 0u;
+      qa[ks][2] = g4 < G ? q32[(g4 * D + k0 + 8) >> 1] : 0u;
+      qa[ks][3] = g4 + 8 < G ? q32[((g4 + 8) * D + k0 + 8) >> 1] : 0u;
+    }
+  }
+  // rows of tile i: positions (or -1), lanes 0..15 hold one each
+  auto tile_pos = [&](int i) {
+    int s = -1;
+    if (lane < 16) {
+      s = idx[i * 16 + lane];
+      if (s < -1 || s > t_abs) {
+        set_err(p.err_word, LISA_DEVERR_CHECK);
+        s = -1;
+      }
+    }
+    return s;
+  };
+  auto stage_tile = [&](int i, int my_pos) {   // cp.async 16 rows of K and V into stage i & 1
+    const uint32_t kdst = wbuf_u32 + (i & 1) * 2 * TILE, vdst = kdst + TILE;
+    constexpr int CH = 2 * D / 16;               // 16-byte chunks per row
+#pragma unroll
+    for (int c = lane; c < 16 * CH; c += 32) {
+      const int r = c / CH, ch = c % CH;
+      const int s = __shfl_sync(0xffffffffu, my_pos, r);
+      const size_t off = (size_t)(s < 0 ? 0 : s) * D + ch * 8;
+      cp_async16(kdst + r * RS + ch * 16, kc + off, s >= 0);
+      cp_async16(vdst + r * RS + ch * 16, vc + off, s >= 0);
+    }
+    cp_async_commit();
+  };
+
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads g4 and g4 + 8
+  float o[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+
+  const int ntiles = RW / 16;
+  int pos_cur = tile_pos(0);
+  const bool any0 = __any_sync(0xffffffffu, lane < 16 && pos_cur >= 0);
+  int nvalid = any0 ? ntiles : 0;
+  if (nvalid) stage_tile(0, pos_cur);
+  for (int i = 0; i < nvalid; ++i) {
+    int pos_next = -1;
+    bool more = false;
+    if (i + 1 < ntiles) {
+      pos_next = tile_pos(i + 1);
+      more = __any_sync(0xffffffffu, lane < 16 && pos_next >= 0);
+    }
+    if (more) {
+      stage_tile(i + 1, pos_next);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+      nvalid = i + 1;                              // the list is -1 padded at its end
+    }
+    __syncwarp();
+    const uint32_t kt = wbuf_u32 + (i & 1) * 2 * TILE, vt = kt + TILE;
+    // S = Q K^T for 16 rows (two 8-row n-tiles)
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int ks2 = 0; ks2 < D / 32; ++ks2) {
+        uint32_t bk[4];
+        ldmatrix_x4(kt + (nt * 8 + (lane & 7)) * RS + ks2 * 64 + (lane >> 3) * 16, bk[0], bk[1], bk[2], bk[3]);
+        mma_16816_bf16(sc[nt], qa[2 * ks2], bk);
+        mma_16816_bf16(sc[nt], qa[2 * ks2 + 1], bk + 2);
+      }
+    }
+    // scale, mask, online softmax (rows g4 and g4 + 8; a quad holds 16 columns)
+    float mt0 = -INFINITY, mt1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = nt * 8 + t2 + (j & 1);
+        const int s = __shfl_sync(0xffffffffu, pos_cur, r);
+        const float x = s >= 0 ? sc[nt][j] * p.scale : -INFINITY;
+        sc[nt][j] = x;
+        if (j < 2) mt0 = fmaxf(mt0, x);
+        else mt1 = fmaxf(mt1, x);
+      }
+    mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 1));
+    mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 2));
+    mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 1));
+    mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 2));
+    const float mn0 = fmaxf(m0, mt0), mn1 = fmaxf(m1, mt1);
+    const float f0 = m0 == -INFINITY ? 0.f : expf(m0 - mn0);
+    const float f1 = m1 == -INFINITY ? 0.f : expf(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    float e[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float mm = j < 2 ? mn0 : mn1;
+        e[nt][j] = sc[nt][j] == -INFINITY ? 0.f : expf(sc[nt][j] - mm);
+      }
+    l0 = l0 * f0 + e[0][0] + e[0][1] + e[1][0] + e[1][1];
+    l1 = l1 * f1 + e[0][2] + e[0][3] + e[1][2] + e[1][3];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      o[j][0] *= f0;
+      o[j][1] *= f0;
+      o[j][2] *= f1;
+      o[j][3] *= f1;
+    }
+    // P as the A operand of a 16-row k-step: hi + lo bf16 pairs
+    uint32_t ph[4], pl[4];
+    {
+      const float pv[4][2] = {{e[0][0], e[0][1]}, {e[0][2], e[0][3]}, {e[1][0], e[1][1]}, {e[1][2], e[1][3]}};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        ph[j] = pack_bf16(pv[j][0], pv[j][1]);
+        const float h0 = __bfloat162float(__float2bfloat16_rn(pv[j][0]));
+        const float h1 = __bfloat162float(__float2bfloat16_rn(pv[j][1]));
+        pl[j] = pack_bf16(pv[j][0] - h0, pv[j][1] - h1);
+      }
+    }
+    // O += P V
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+      uint32_t bv[4];
+      const int mm = lane >> 3;
+      ldmatrix_x4_trans(vt + ((mm & 1) * 8 + (lane & 7)) * RS + (np * 16 + (mm >> 1) * 8) * 2, bv[0], bv[1], bv[2],
+                        bv[3]);
+      mma_16816_bf16(o[2 * np], ph, bv);
+      mma_16816_bf16(o[2 * np], pl, bv);
+      mma_16816_bf16(o[2 * np + 1], ph, bv + 2);
+      mma_16816_bf16(o[2 * np + 1], pl, bv + 2);
+    }
+    __syncwarp();                                  // this stage may be refilled next
+    pos_cur = pos_next;
+  }
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+
+  // merge the warps: [warp][16 heads] max and sum, [warp][16][D] O
+  __syncthreads();
+  float *s_ml = reinterpret_cast<float *>(s_att);                 // [4][16][2]
+  float *s_o = s_ml + kAttnWarps * 32;                            // [4][16][D]
+  if ((lane & 3) == 0) {
+    s_ml[(warp * 16 + g4) * 2] = m0;
+    s_ml[(warp * 16 + g4) * 2 + 1] = l0;
+    s_ml[(warp * 16 + g4 + 8) * 2] = m1;
+    s_ml[(warp * 16 + g4 + 8) * 2 + 1] = l1;
+  }
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int d = j * 8 + t2;
+    s_o[(warp * 16 + g4) * D + d] = o[j][0];
+    s_o[(warp * 16 + g4) * D + d + 1] = o[j][1];
+    s_o[(warp * 16 + g4 + 8) * D + d] = o[j][2];
+    s_o[(warp * 16 + g4 + 8) * D + d + 1] = o[j][3];
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kAttnWarps * 32) {
+    const int hh = i / D, d = i % D;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) mx = fmaxf(mx, s_ml[(w * 16 + hh) * 2]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) {
+      const float mw = s_ml[(w * 16 + hh) * 2];
+      if (mw == -INFINITY) continue;
+      const float f = expf(mw - mx);
+      num = fmaf(f, s_o[(w * 16 + hh) * D + d], num);
+      den = fmaf(f, s_ml[(w * 16 + hh) * 2 + 1], den);
+    }
+    const size_t row = ((size_t)b * p.T + tau) * p.Hq + g * G + hh;
+    const float gam = 1.f / (1.f + expf(-p.gate[row]));
+    const float o_lin = p.olin[row * D + d];
+    reinterpret_cast<__nv_bfloat16 *>(p.out)[row * D + d] = __float2bfloat16_rn(gam * (num / den) + (1.f - gam) * o_lin);
+  }
+}
+
 cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st) {
   dim3 grid(p.T, p.B * p.Hkv);
   cudaError_t e;
+  if (dtype == LISA_BF16 && p.M % (16 * kAttnWarps) == 0) {
+    if (p.D == 128) {
+      constexpr int smem = attn_mma_smem<128>();
+      if ((e = prepare_kernel(prefill_attend_mma_kernel<128>, smem)) != cudaSuccess) return e;
+      prefill_attend_mma_kernel<128><<<grid, kAttnWarps * 32, smem, st>>>(p);
+    } else {
+      constexpr int smem = attn_mma_smem<64>();
+      if ((e = prepare_kernel(prefill_attend_mma_kernel<64>, smem)) != cudaSuccess) return e;
+      prefill_attend_mma_kernel<64><<<grid, kAttnWarps * 32, smem, st>>>(p);
+    }
+    return cudaGetLastError();
+  }
   if (dtype == LISA_BF16) {
     if (p.D == 128) {
       if ((e = prepare_kernel(prefill_attend_kernel<__nv_bfloat16, 128>)) != cudaSuccess) return e;
