@@ -114,7 +114,7 @@ void set_select_smem(lisa::RowsParams &r, int n_max) {
   const int cap = n_max < kRowsKeysCap ? n_max : kRowsKeysCap;
   r.smem_keys_cap = (cap + 3) & ~3;
   r.cand_cap = kCandCap;
-  r.select_smem = (size_t)(r.smem_keys_cap + r.cand_cap) * 4;
+  r.select_smem = (size_t)(r.smem_keys_cap + 2 * r.cand_cap) * 4;   // keys, candidate keys and positions
 }
 
 }  // namespace

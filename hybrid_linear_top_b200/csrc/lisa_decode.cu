@@ -33,6 +33,7 @@
 
 #include "lisa_internal.h"
 #include "lisa_common.cuh"
+#include "lisa_select.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -129,83 +130,6 @@ __device__ __forceinline__ void dec_find_bucket(const uint32_t *tot, uint32_t *m
       }
     }
   }
-}
-
-// CTA-wide (kDecThreads = 256 threads, 4 bins each): the bin of fh[0..1024)
-// (higher bin = larger keys) that holds the rem-th largest key, counting from
-// the top.  misc[0] = bin (0xFFFFFFFF if the counts hold fewer than rem keys),
-// misc[1] = keys in higher bins, misc[2] = keys in the bin; misc[3] is zeroed.
-// Uses misc[8..15].  Ends with a barrier.
-__device__ void dec_find_bin1024(const uint32_t *fh, uint32_t rem, uint32_t *misc) {
-  static_assert(kDecThreads * 4 == 1024, "four bins per thread");
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b0 = 1023 - 4 * tid;
-  const uint32_t c0 = fh[b0], c1 = fh[b0 - 1], c2 = fh[b0 - 2], c3 = fh[b0 - 3];
-  const uint32_t c = c0 + c1 + c2 + c3;
-  uint32_t inc = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
-  }
-  if (lane == 31) misc[8 + warp] = inc;
-  if (tid == 0) {
-    misc[0] = 0xFFFFFFFFu;
-    misc[3] = 0;
-  }
-  __syncthreads();
-  uint32_t off = 0;
-#pragma unroll
-  for (int w8 = 0; w8 < kDecThreads / 32; ++w8) off += w8 < warp ? misc[8 + w8] : 0u;
-  const uint32_t exc = off + inc - c;
-  if (exc < rem && rem <= exc + c) {
-    const uint32_t cc[4] = {c0, c1, c2, c3};
-    uint32_t cum = exc;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (cum < rem && rem <= cum + cc[j]) {
-        misc[0] = (uint32_t)(b0 - j);
-        misc[1] = cum;
-        misc[2] = cc[j];
-      }
-      cum += cc[j];
-    }
-  }
-  __syncthreads();
-}
-
-// CTA-wide exclusive prefix sums of two counters, plus their totals.
-__device__ __forceinline__ void cta_scan2(uint32_t a, uint32_t b, uint32_t &ea, uint32_t &eb, uint32_t &ta,
-                                          uint32_t &tb, uint32_t *misc) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t ia = a, ib = b;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o);
-    if (lane >= o) {
-      ia += ya;
-      ib += yb;
-    }
-  }
-  __syncthreads();
-  if (lane == 31) {
-    misc[32 + warp] = ia;
-    misc[40 + warp] = ib;
-  }
-  __syncthreads();
-  uint32_t wa = 0, wb = 0;
-  ta = 0;
-  tb = 0;
-  for (int w8 = 0; w8 < kDecThreads / 32; ++w8) {
-    if (w8 < warp) {
-      wa += misc[32 + w8];
-      wb += misc[40 + w8];
-    }
-    ta += misc[32 + w8];
-    tb += misc[40 + w8];
-  }
-  ea = wa + ia - a;
-  eb = wb + ib - b;
 }
 
 template <typename T, int D, int DI, int NC>
@@ -668,7 +592,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
             if (u >= lbx && u <= ubx) atomicAdd(&fh[(u - lbx) >> shx], 1u);
           });
           __syncthreads();
-          dec_find_bin1024(fh, rem, misc);              // misc[0..2]; zeroes misc[3]
+          find_bin1024<kDecThreads>(fh, rem, misc);     // misc[0..2]; zeroes misc[3]
           const uint32_t bin = misc[0];
           if (bin > 1023u) break;                       // counts inconsistent: cannot happen
           rem -= misc[1];
@@ -723,7 +647,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
             ceq += u == kstar ? 1u : 0u;
           });
           uint32_t eg, ee, tg, te;
-          cta_scan2(cgt, ceq, eg, ee, tg, te, misc);
+          cta_scan2<kDecThreads>(cgt, ceq, eg, ee, tg, te, misc);
           if (tid == 0 && (tg + need_eq != (uint32_t)M || te < need_eq)) set_err(p.err_word, LISA_DEVERR_CHECK);
           for_run([&](int slot) {
             const uint32_t u = ck[slot];

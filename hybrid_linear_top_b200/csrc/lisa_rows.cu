@@ -170,6 +170,18 @@ __global__ void __launch_bounds__(NT) rows_select_kernel(RowsParams p, int tau0,
     cand = s_dyn + p.smem_keys_cap;
   }
   int *out = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M;
+  if (keys == s_dyn && n >= 8 * NT) {
+    // long rows: a bound from every thread's 4 largest keys, then an exact
+    // select among the few keys above it
+    __shared__ BoundedShared bsm;
+    const int r = block_topm_bounded<NT>(keys, n, p.M, out, bsm, cand, reinterpret_cast<int *>(cand + p.cand_cap),
+                                         p.cand_cap);
+    if (r == 1) return;
+    if (r < 0) {
+      if (threadIdx.x == 0) set_err(p.err_word, LISA_DEVERR_CHECK);
+      return;
+    }
+  }
   if (!block_topm<NT>(keys, n, p.M, out, sm, cand, p.cand_cap) && threadIdx.x == 0)
     set_err(p.err_word, LISA_DEVERR_CHECK);
 }

@@ -218,4 +218,278 @@ __device__ bool block_topm(const uint32_t *keys, int n, int M, int *out, TopmSha
   return !__syncthreads_or(bad);
 }
 
+
+// ---------------------------------------------------------------- range-histogram select helpers
+// CTA-wide (NT = 256 threads, 4 bins each): the bin of fh[0..1024) (higher bin
+// = larger keys) that holds the rem-th largest key, counting from the top.
+// misc[0] = bin (0xFFFFFFFF if the counts hold fewer than rem keys), misc[1] =
+// keys in higher bins, misc[2] = keys in the bin; misc[3] is zeroed.  Uses
+// misc[8..15].  Ends with a barrier.
+template <int NT>
+__device__ void find_bin1024(const uint32_t *fh, uint32_t rem, uint32_t *misc) {
+  static_assert(NT * 4 == 1024, "four bins per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b0 = 1023 - 4 * tid;
+  const uint32_t c0 = fh[b0], c1 = fh[b0 - 1], c2 = fh[b0 - 2], c3 = fh[b0 - 3];
+  const uint32_t c = c0 + c1 + c2 + c3;
+  uint32_t inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) misc[8 + warp] = inc;
+  if (tid == 0) {
+    misc[0] = 0xFFFFFFFFu;
+    misc[3] = 0;
+  }
+  __syncthreads();
+  uint32_t off = 0;
+#pragma unroll
+  for (int w8 = 0; w8 < NT / 32; ++w8) off += w8 < warp ? misc[8 + w8] : 0u;
+  const uint32_t exc = off + inc - c;
+  if (exc < rem && rem <= exc + c) {
+    const uint32_t cc[4] = {c0, c1, c2, c3};
+    uint32_t cum = exc;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (cum < rem && rem <= cum + cc[j]) {
+        misc[0] = (uint32_t)(b0 - j);
+        misc[1] = cum;
+        misc[2] = cc[j];
+      }
+      cum += cc[j];
+    }
+  }
+  __syncthreads();
+}
+
+// CTA-wide exclusive prefix sums of two counters, plus their totals.  Uses
+// misc[32..47].
+template <int NT>
+__device__ __forceinline__ void cta_scan2(uint32_t a, uint32_t b, uint32_t &ea, uint32_t &eb, uint32_t &ta,
+                                          uint32_t &tb, uint32_t *misc) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += ya;
+      ib += yb;
+    }
+  }
+  __syncthreads();
+  if (lane == 31) {
+    misc[32 + warp] = ia;
+    misc[40 + warp] = ib;
+  }
+  __syncthreads();
+  uint32_t wa = 0, wb = 0;
+  ta = 0;
+  tb = 0;
+  for (int w8 = 0; w8 < NT / 32; ++w8) {
+    if (w8 < warp) {
+      wa += misc[32 + w8];
+      wb += misc[40 + w8];
+    }
+    ta += misc[32 + w8];
+    tb += misc[40 + w8];
+  }
+  ea = wa + ia - a;
+  eb = wb + ib - b;
+}
+
+// Exact M-th largest key K* among keys ck[0..nc) that all lie in [lo, hi]:
+// 1024-bin range histograms narrowed until one bin holds <= 32 keys (ranked
+// in one warp) or is a single value.  Writes K* and need_eq = how many keys
+// equal to K* the top M takes; returns false if the counts are inconsistent.
+// fh: 1024 words of shared scratch; misc: 64 words.  All NT threads call it.
+template <int NT>
+__device__ bool range_kth(const uint32_t *ck, int nc, uint32_t lo, uint32_t hi, uint32_t M, uint32_t *fh,
+                          uint32_t *misc, uint32_t *members, uint32_t &kstar, uint32_t &need_eq) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t lbx = lo, ubx = hi, rem = M;
+  uint32_t shx = (hi - lo) < 1024u ? 0u : (uint32_t)(32 - __clz(hi - lo)) - 10u;
+#pragma unroll 1
+  for (int iter = 0; iter < 4; ++iter) {
+    for (int i = tid; i < 1024; i += NT) fh[i] = 0;
+    __syncthreads();
+    for (int j = tid; j < nc; j += NT) {
+      const uint32_t u = ck[j];
+      if (u >= lbx && u <= ubx) atomicAdd(&fh[(u - lbx) >> shx], 1u);
+    }
+    __syncthreads();
+    find_bin1024<NT>(fh, rem, misc);
+    const uint32_t bin = misc[0];
+    if (bin > 1023u) return false;
+    rem -= misc[1];
+    const uint32_t cb = misc[2];
+    const uint32_t blo = lbx + (bin << shx);
+    if (shx == 0) {
+      kstar = blo;
+      need_eq = rem;
+      return true;
+    }
+    if (cb <= 32) {
+      for (int j = tid; j < nc; j += NT) {
+        const uint32_t u = ck[j];
+        if (u >= blo && u <= ubx && ((u - lbx) >> shx) == bin) {
+          const uint32_t s = atomicAdd(&misc[3], 1u);
+          if (s < 32) members[s] = u;
+        }
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t x = lane < (int)cb ? members[lane] : 0u;
+        uint32_t gt = 0, ge = 0;
+        for (int j = 0; j < (int)cb; ++j) {
+          const uint32_t y = __shfl_sync(0xffffffffu, x, j);
+          gt += y > x ? 1u : 0u;
+          ge += y >= x ? 1u : 0u;
+        }
+        if (lane < (int)cb && gt < rem && rem <= ge) {
+          misc[5] = x;
+          misc[7] = rem - gt;
+        }
+      }
+      __syncthreads();
+      kstar = misc[5];
+      need_eq = misc[7];
+      __syncthreads();
+      return true;
+    }
+    const unsigned long long top = (unsigned long long)blo + (1ull << shx) - 1ull;
+    lbx = blo;
+    ubx = top < ubx ? (uint32_t)top : ubx;
+    shx = shx > 10u ? shx - 10u : 0u;
+    __syncthreads();
+  }
+  return false;
+}
+
+struct BoundedShared {
+  uint32_t fh[1024];
+  uint32_t misc[64];
+  uint32_t members[32];
+};
+
+// Top-M of keys[0..n) (shared memory, n > M, n >= 8 * NT) through a bound:
+// every thread keeps the 4 largest of its keys; the bin holding the M-th
+// largest of those 4 * NT values gives lb with at least M keys >= lb; the keys
+// >= lb are compacted in position order into (ck, cp); the exact K* among them
+// and an ordered compaction emit the ascending index list.
+// Returns 1 when done, 0 when more than cap keys pass the bound (nothing
+// written; the caller selects another way), -1 on an internal check failure.
+template <int NT>
+__device__ int block_topm_bounded(const uint32_t *keys, int n, int M, int *out, BoundedShared &sm, uint32_t *ck,
+                                  int *cp, int cap) {
+  static_assert(NT == 256, "256 threads");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // (1) the 4 largest keys of each thread
+  uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
+  for (int i = tid; i < n; i += NT) {
+    uint32_t u = keys[i];
+    if (u > t3) {
+      t3 = u;
+      if (t3 > t2) { const uint32_t x = t2; t2 = t3; t3 = x; }
+      if (t2 > t1) { const uint32_t x = t1; t1 = t2; t2 = x; }
+      if (t1 > t0) { const uint32_t x = t0; t0 = t1; t1 = x; }
+    }
+  }
+  // range of those values
+  uint32_t vmin = t3, vmax = t0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  }
+  if (lane == 0) {
+    sm.misc[16 + warp] = vmin;
+    sm.misc[24 + warp] = vmax;
+  }
+  for (int i = tid; i < 1024; i += NT) sm.fh[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int w8 = 0; w8 < NT / 32; ++w8) {
+    vmin = min(vmin, sm.misc[16 + w8]);
+    vmax = max(vmax, sm.misc[24 + w8]);
+  }
+  // (2) lb = lower edge of the bin of the M-th largest of the 4 * NT values
+  const uint32_t sh = (vmax - vmin) < 1024u ? 0u : (uint32_t)(32 - __clz(vmax - vmin)) - 10u;
+  atomicAdd(&sm.fh[(t0 - vmin) >> sh], 1u);
+  atomicAdd(&sm.fh[(t1 - vmin) >> sh], 1u);
+  atomicAdd(&sm.fh[(t2 - vmin) >> sh], 1u);
+  atomicAdd(&sm.fh[(t3 - vmin) >> sh], 1u);
+  __syncthreads();
+  find_bin1024<NT>(sm.fh, (uint32_t)M, sm.misc);
+  if (sm.misc[0] > 1023u) return -1;
+  const uint32_t lb = vmin + (sm.misc[0] << sh);
+  // (3) keys >= lb in position order: warp w owns a contiguous run
+  const int cw = (((n + 7) / 8) + 31) & ~31;
+  const int j0 = min(n, warp * cw), j1 = min(n, j0 + cw);
+  uint32_t wc = 0;
+  for (int base = j0; base < j1; base += 32) {
+    const int j = base + lane;
+    wc += __popc(__ballot_sync(0xffffffffu, j < j1 && keys[j] >= lb));
+  }
+  if (lane == 0) sm.misc[48 + warp] = wc;
+  __syncthreads();
+  uint32_t off = 0, nc = 0;
+#pragma unroll
+  for (int w8 = 0; w8 < NT / 32; ++w8) {
+    const uint32_t c = sm.misc[48 + w8];
+    off += w8 < warp ? c : 0u;
+    nc += c;
+  }
+  if (nc > (uint32_t)cap) return 0;               // the same answer in every thread
+  {
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = j0; base < j1; base += 32) {
+      const int j = base + lane;
+      const bool act = j < j1 && keys[j] >= lb;
+      const unsigned am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t o = off + __popc(am & lt);
+        ck[o] = keys[j];
+        cp[o] = j;
+      }
+      off += __popc(am);
+    }
+  }
+  __syncthreads();
+  // (4) exact K* among the candidates
+  uint32_t kstar = 0, need_eq = 0;
+  if (!range_kth<NT>(ck, (int)nc, lb, vmax, (uint32_t)M, sm.fh, sm.misc, sm.members, kstar, need_eq)) return -1;
+  // (5) ordered emission from the candidate list: thread-contiguous runs
+  const int per = ((int)nc + NT - 1) / NT;
+  const int c0 = min((int)nc, tid * per), c1 = min((int)nc, c0 + per);
+  uint32_t cgt = 0, ceq = 0;
+  for (int c = c0; c < c1; ++c) {
+    const uint32_t u = ck[c];
+    cgt += u > kstar ? 1u : 0u;
+    ceq += u == kstar ? 1u : 0u;
+  }
+  uint32_t eg, ee, tg, te;
+  cta_scan2<NT>(cgt, ceq, eg, ee, tg, te, sm.misc);
+  bool bad = tg + need_eq != (uint32_t)M || te < need_eq;
+  for (int c = c0; c < c1; ++c) {
+    const uint32_t u = ck[c];
+    if (u > kstar) {
+      const uint32_t o = eg + min(ee, need_eq);
+      if (o < (uint32_t)M) out[o] = cp[c];
+      else bad = true;
+      ++eg;
+    } else if (u == kstar) {
+      if (ee < need_eq) {
+        const uint32_t o = eg + ee;
+        if (o < (uint32_t)M) out[o] = cp[c];
+        else bad = true;
+      }
+      ++ee;
+    }
+  }
+  return __syncthreads_or(bad) ? -1 : 1;
+}
+
 }  // namespace lisa
