@@ -452,43 +452,63 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     uint32_t *fh = hist + 1024;                         // CTA 0: 1024-bin histogram of candidate keys
     uint32_t *segp = tot + 64;                          // CTA 0: exclusive prefix of the segment sizes
     uint32_t *misc0 = cluster.map_shared_rank(misc, 0);
-    // (a) theta = the smallest of kl group maxima of this CTA's keys (groups:
-    //     positions j = g (mod kl)); at least kl of its keys are >= theta.
-    //     Also the largest key, for the histogram range.
-    int kl = 1;
-    while (kl < (M + NC - 1) / NC) kl <<= 1;
+    // (a) theta: every thread keeps the 4 largest of its keys; the lower edge
+    //     of the 1024-bin range-histogram bin that holds the kl-th largest of
+    //     those values has at least kl of this CTA's keys at or above it.
+    //     Also the largest key, for the range of the exact select.
+    const int kl = (M + NC - 1) / NC;
     int covered = 0;
     for (int r = 0; r < NC; ++r) {
       const int cr = min(n, (r + 1) * kpc) - min(n, r * kpc);
       if (cr >= kl) covered += kl;
     }
     {
-      uint32_t m = 0;
-      for (int j = tid; j < cnt; j += kDecThreads) m = max(m, keys[j]);
-      tot[tid] = m;                                     // thread tid holds group tid % kl
-      if (rank == 0)
-        for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
-      __syncthreads();
-      if (cnt >= kl && tid < kl) {
-        uint32_t gm = 0;
-        for (int j = tid; j < kDecThreads; j += kl) gm = max(gm, tot[j]);
-        hist[tid] = gm;
+      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
+      int kt = 0;
+      for (int j = tid; j < cnt; j += kDecThreads) {
+        const uint32_t u = keys[j];
+        ++kt;
+        if (kt > 4 && u <= t3) continue;
+        t3 = u;
+        if (t3 > t2) { const uint32_t x = t2; t2 = t3; t3 = x; }
+        if (t2 > t1) { const uint32_t x = t1; t1 = t2; t2 = x; }
+        if (t1 > t0) { const uint32_t x = t0; t0 = t1; t1 = x; }
       }
-      __syncthreads();
-      if (warp == 0) {
-        uint32_t mn = 0xFFFFFFFFu, mx = 0;              // 0xFFFFFFFF: neutral for the minimum
-        if (cnt >= kl)
-          for (int j = lane; j < kl; j += 32) mn = min(mn, hist[j]);
-        for (int j = lane; j < kDecThreads; j += 32) mx = max(mx, tot[j]);
+      kt = min(kt, 4);
+      // smallest and largest of the kept values (0xFFFFFFFF / 0 where a thread kept none)
+      uint32_t vmin = kt == 0 ? 0xFFFFFFFFu : kt == 1 ? t0 : kt == 2 ? t1 : kt == 3 ? t2 : t3;
+      uint32_t vmax = t0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        if (lane == 0) {
-          misc[4] = mn;
-          misc[6] = mx;
-        }
+      for (int o = 16; o > 0; o >>= 1) {
+        vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+        vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      }
+      if (lane == 0) {
+        tot[warp] = vmin;
+        tot[8 + warp] = vmax;
+      }
+      for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int w8 = 0; w8 < kDecThreads / 32; ++w8) {
+        vmin = min(vmin, tot[w8]);
+        vmax = max(vmax, tot[8 + w8]);
+      }
+      uint32_t theta = 0xFFFFFFFFu;                     // neutral for the minimum
+      if (cnt >= kl) {                                  // uniform in the CTA
+        const uint32_t sh = (vmax - vmin) < 1024u ? 0u : (uint32_t)(32 - __clz(vmax - vmin)) - 10u;
+        if (kt > 0) atomicAdd(&fh[(t0 - vmin) >> sh], 1u);
+        if (kt > 1) atomicAdd(&fh[(t1 - vmin) >> sh], 1u);
+        if (kt > 2) atomicAdd(&fh[(t2 - vmin) >> sh], 1u);
+        if (kt > 3) atomicAdd(&fh[(t3 - vmin) >> sh], 1u);
+        __syncthreads();
+        find_bin1024<kDecThreads>(fh, (uint32_t)kl, misc);
+        if (misc[0] <= 1023u) theta = vmin + (misc[0] << sh);
+        else theta = 0;                                 // counts inconsistent: no bound from this CTA
+      }
+      if (tid == 0) {
+        misc[4] = theta;
+        misc[6] = vmax;
       }
     }
     cluster.sync();                                     // bounds published, every ring is free
@@ -583,10 +603,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         bool found = false;
 #pragma unroll 1
         for (int iter = 0; iter < 4 && !found; ++iter) {
-          if (iter > 0) {
-            for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
-            __syncthreads();
-          }
+          for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
+          __syncthreads();
           for_run([&](int slot) {
             const uint32_t u = ck[slot];
             if (u >= lbx && u <= ubx) atomicAdd(&fh[(u - lbx) >> shx], 1u);
