@@ -555,6 +555,16 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
             const uint32_t o = off + __popc(am & lt);
             ck[o] = keys[j];
             cp[o] = k0 + j;
+            if (k0 + j != t) {                        // a likely selected row: K and V into L2 now
+              const size_t row = ((size_t)bg * p.L_max + k0 + j) * D;
+              const char *kr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.k_cache) + row);
+              const char *vr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.v_cache) + row);
+#pragma unroll
+              for (int c = 0; c < ROWB; c += 128) {
+                prefetch_l2(kr + c);
+                prefetch_l2(vr + c);
+              }
+            }
           }
           off += __popc(am);
         }
