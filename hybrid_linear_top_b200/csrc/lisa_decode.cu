@@ -179,56 +179,19 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   int *sidx = reinterpret_cast<int *>(smem + lay.sidx);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
 
-  // Everything read below may have been written by the previous kernel.
-  grid_dep_wait();
-  grid_dep_launch();
-
-  const int t = p.pos[b];
-  if (t < 0 || t >= p.L_max) {  // same value in every CTA of the cluster: all leave together
-    if (rank == 0 && tid == 0) set_err(p.err_word, LISA_DEVERR_POS);
-    return;
-  }
-  const int n = t + 1;
-  const int kpc = (((n + NC - 1) / NC) + 31) & ~31;
-  const int k0 = min(n, rank * kpc);
-  const int k1 = min(n, k0 + kpc);
-  const int cnt = k1 - k0;
-  const int nsub = (cnt + SUB - 1) / SUB;
-
-  const T *kidx_cache = reinterpret_cast<const T *>(p.kidx_cache) + (size_t)bg * p.L_max * DI;
-  const T *kidx_new = reinterpret_cast<const T *>(p.kidx) + (size_t)bg * DI;
-
-  // ---------------------------------------------------------------- TMA prologue
+  // barrier init touches shared memory only: before the wait on the previous kernel
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
-  __syncthreads();
-  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS, and sub-chunk i + NS -> L2
-    const int s_lo = k0 + i * SUB;
-    const int s_hi = min(k1, s_lo + SUB);
-    const int ncopy = max(0, min(s_hi, t) - s_lo);   // row t comes from the argument
-    {
-      const int p_lo = s_lo + NS * SUB;
-      const int np = max(0, min(min(k1, p_lo + SUB), t) - p_lo);
-      if (np > 0) bulk_prefetch_l2(kidx_cache + (size_t)p_lo * DI, (uint32_t)(np * RB));
-    }
-    uint64_t *bar = &bars[i % NS];
-    unsigned char *dst = ring + (i % NS) * STB;
-    if (ncopy > 0) {
-      if constexpr (SG::kMma) {
-        mbar_arrive_expect_tx(bar, (uint32_t)(SUB * RB));   // the whole box lands, out-of-range rows zero
-        tma_load_2d(dst, &kmap, 0, bg * p.L_max + s_lo, bar);
-      } else {
-        mbar_arrive_expect_tx(bar, (uint32_t)(ncopy * RB));
-        bulk_g2s(dst, kidx_cache + (size_t)s_lo * DI, (uint32_t)(ncopy * RB), bar);
-      }
-    } else {
-      mbar_arrive(bar);
-    }
-  };
-  if (tid == 0)
-    for (int i = 0; i < min(NS, nsub); ++i) issue(i);
+  // Everything read below may have been written by the previous kernel.
+  grid_dep_wait();
+  grid_dep_launch();
+
+  const int t = p.pos[b];                  // in flight while the loads below are issued
+  const T *kidx_cache = reinterpret_cast<const T *>(p.kidx_cache) + (size_t)bg * p.L_max * DI;
+  const T *kidx_new = reinterpret_cast<const T *>(p.kidx) + (size_t)bg * DI;
+
   // ---------------------------------------------------------------- early loads
   // state slab of the first (up to) HP query heads
   const int c0s = rank * COLS;
@@ -274,6 +237,43 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     if (kc < R) wq0 = p.w[(size_t)b * p.HI + g * R + kc];
     if (kc + 1 < R) wq1 = p.w[(size_t)b * p.HI + g * R + kc + 1];
   }
+  if (t < 0 || t >= p.L_max) {  // same value in every CTA of the cluster: all leave together
+    if (rank == 0 && tid == 0) set_err(p.err_word, LISA_DEVERR_POS);
+    return;
+  }
+  const int n = t + 1;
+  const int kpc = (((n + NC - 1) / NC) + 31) & ~31;
+  const int k0 = min(n, rank * kpc);
+  const int k1 = min(n, k0 + kpc);
+  const int cnt = k1 - k0;
+  const int nsub = (cnt + SUB - 1) / SUB;
+
+  // ---------------------------------------------------------------- TMA ring
+  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS, and sub-chunk i + NS -> L2
+    const int s_lo = k0 + i * SUB;
+    const int s_hi = min(k1, s_lo + SUB);
+    const int ncopy = max(0, min(s_hi, t) - s_lo);   // row t comes from the argument
+    {
+      const int p_lo = s_lo + NS * SUB;
+      const int np = max(0, min(min(k1, p_lo + SUB), t) - p_lo);
+      if (np > 0) bulk_prefetch_l2(kidx_cache + (size_t)p_lo * DI, (uint32_t)(np * RB));
+    }
+    uint64_t *bar = &bars[i % NS];
+    unsigned char *dst = ring + (i % NS) * STB;
+    if (ncopy > 0) {
+      if constexpr (SG::kMma) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(SUB * RB));   // the whole box lands, out-of-range rows zero
+        tma_load_2d(dst, &kmap, 0, bg * p.L_max + s_lo, bar);
+      } else {
+        mbar_arrive_expect_tx(bar, (uint32_t)(ncopy * RB));
+        bulk_g2s(dst, kidx_cache + (size_t)s_lo * DI, (uint32_t)(ncopy * RB), bar);
+      }
+    } else {
+      mbar_arrive(bar);
+    }
+  };
+  if (tid == 0)
+    for (int i = 0; i < min(NS, nsub); ++i) issue(i);
   // append the new token (row t) from the CTA whose key slice holds it
   if (p.fuse_append && t >= k0 && t < k1) {
     const size_t row = (size_t)bg * p.L_max + t;
