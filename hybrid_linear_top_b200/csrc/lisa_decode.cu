@@ -514,12 +514,18 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     cluster.sync();                                     // bounds published, every ring is free
     uint32_t lb = 0, hi = 0;
     {
+      // lane r of every warp reads rank r's bound and maximum (one remote
+      // load per lane, not per thread and rank)
       uint32_t mn = 0xFFFFFFFFu;
+      if (lane < NC) {
+        const uint32_t *mr = cluster.map_shared_rank(misc, lane);
+        mn = mr[4];
+        hi = mr[6];
+      }
 #pragma unroll
-      for (int r = 0; r < NC; ++r) {
-        const uint32_t *mr = cluster.map_shared_rank(misc, r);
-        mn = min(mn, mr[4]);
-        hi = max(hi, mr[6]);
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
       }
       if (covered >= M) lb = mn;
     }
@@ -571,9 +577,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       }
     }
     cluster.sync();                                     // candidates complete
-    bool fits = true;                                   // the same answer in every CTA
-#pragma unroll
-    for (int r = 0; r < NC; ++r) fits = fits && misc0[48 + r] <= (uint32_t)SEG;
+    // the same answer in every CTA: lane r of every warp checks rank r's segment
+    const bool fits = __all_sync(0xffffffffu, lane >= NC || misc0[48 + lane] <= (uint32_t)SEG);
     if (fits) {
       if (rank == 0) {
         // (c) CTA 0: exact M-th key among the candidates (range histograms of
@@ -981,20 +986,23 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   cluster.sync();                            // all partials of the cluster are ready
 
   // ---------------------------------------------------------------- merge + gate, columns of this CTA
+  // every rank's (max, sum) per head, copied once into this CTA
+  float *pml_all = reinterpret_cast<float *>(hist);     // [NC][2G]
+  for (int i = tid; i < NC * 2 * G; i += kDecThreads) pml_all[i] = cluster.map_shared_rank(pml, i / (2 * G))[i % (2 * G)];
+  __syncthreads();
   for (int i = tid; i < G * COLS; i += kDecThreads) {
     const int hh = i / COLS, c = i % COLS, d = c0s + c;
     float mx = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < NC; ++r) mx = fmaxf(mx, cluster.map_shared_rank(pml, r)[2 * hh]);
+    for (int r = 0; r < NC; ++r) mx = fmaxf(mx, pml_all[r * 2 * G + 2 * hh]);
     float num = 0.f, den = 0.f;
 #pragma unroll
     for (int r = 0; r < NC; ++r) {
-      const float *pr = cluster.map_shared_rank(pml, r);
-      const float mr = pr[2 * hh];
+      const float mr = pml_all[r * 2 * G + 2 * hh];
       if (mr == -INFINITY) continue;
       const float f = expf(mr - mx);
       num = fmaf(f, cluster.map_shared_rank(part, r)[hh * D + d], num);
-      den = fmaf(f, pr[2 * hh + 1], den);
+      den = fmaf(f, pml_all[r * 2 * G + 2 * hh + 1], den);
     }
     const int h = g * G + hh;
     const float o_sp = num / den;
