@@ -561,22 +561,26 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
             const uint32_t o = off + __popc(am & lt);
             ck[o] = keys[j];
             cp[o] = k0 + j;
-            if (k0 + j != t) {                        // a likely selected row: K and V into L2 now
-              const size_t row = ((size_t)bg * p.L_max + k0 + j) * D;
-              const char *kr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.k_cache) + row);
-              const char *vr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.v_cache) + row);
-#pragma unroll
-              for (int c = 0; c < ROWB; c += 128) {
-                prefetch_l2(kr + c);
-                prefetch_l2(vr + c);
-              }
-            }
           }
           off += __popc(am);
         }
       }
     }
     cluster.sync();                                     // candidates complete
+    // this CTA's candidates are likely selected: their K and V rows into L2
+    // while CTA 0 selects (after the barrier, which need not wait for them)
+    for (int j = tid; j < cnt; j += kDecThreads) {
+      if (keys[j] >= lb && k0 + j != t) {
+        const size_t row = ((size_t)bg * p.L_max + k0 + j) * D;
+        const char *kr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.k_cache) + row);
+        const char *vr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.v_cache) + row);
+#pragma unroll
+        for (int c = 0; c < ROWB; c += 128) {
+          prefetch_l2(kr + c);
+          prefetch_l2(vr + c);
+        }
+      }
+    }
     // the same answer in every CTA: lane r of every warp checks rank r's segment
     const bool fits = __all_sync(0xffffffffu, lane >= NC || misc0[48 + lane] <= (uint32_t)SEG);
     if (fits) {
