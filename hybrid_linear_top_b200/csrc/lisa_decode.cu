@@ -841,21 +841,21 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   }
   __syncthreads();
   {
+    // every 16-byte piece in flight at once (asynchronous copies; rows of
+    // unselected slots are zero-filled)
     const T *kc = reinterpret_cast<const T *>(p.k_cache) + (size_t)bg * p.L_max * D;
     const T *vc = reinterpret_cast<const T *>(p.v_cache) + (size_t)bg * p.L_max * D;
+    const uint32_t kvs_base = smem_u32(kvs);
     for (int i = tid; i < rpc * SL; i += kDecThreads) {
       const int r = i / SL, sl = i % SL;
       const int s = sidx[r];
-      uint4 uk = make_uint4(0, 0, 0, 0), uv = make_uint4(0, 0, 0, 0);
-      if (s >= 0) {
-        const T *kr = (s == t) ? kin : kc + (size_t)s * D;
-        const T *vr = (s == t) ? vin : vc + (size_t)s * D;
-        uk = *reinterpret_cast<const uint4 *>(kr + sl * VEC);
-        uv = *reinterpret_cast<const uint4 *>(vr + sl * VEC);
-      }
-      *reinterpret_cast<uint4 *>(kvs + r * RS + sl * 16) = uk;
-      *reinterpret_cast<uint4 *>(kvs + (rpc + r) * RS + sl * 16) = uv;
+      const T *kr = (s == t) ? kin : kc + (size_t)(s < 0 ? 0 : s) * D;
+      const T *vr = (s == t) ? vin : vc + (size_t)(s < 0 ? 0 : s) * D;
+      cp_async16(kvs_base + r * RS + sl * 16, kr + sl * VEC, s >= 0);
+      cp_async16(kvs_base + (rpc + r) * RS + sl * 16, vr + sl * VEC, s >= 0);
     }
+    cp_async_commit();
+    cp_async_wait_all();
   }
   __syncthreads();
   // bf16 with whole 16-row k-steps: both products on the tensor cores (warp

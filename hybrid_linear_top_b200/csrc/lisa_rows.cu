@@ -340,12 +340,6 @@ __global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
 // then the gate mixes in o_lin.
 constexpr int kAttnWarps = 4;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int D>
 constexpr int attn_mma_smem() {
