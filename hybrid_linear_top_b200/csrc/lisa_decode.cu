@@ -25,7 +25,8 @@
 //      compaction.  When a segment overflows, a cluster-wide radix select
 //      (histograms summed over distributed shared memory) runs instead;
 //   3. gather M/NC of the selected K/V rows, partial softmax for the G heads;
-//   4. merge the NC partials for its own column slice, apply the gate, store.
+//   4. every rank writes its partials of CTA r's columns into CTA r; after
+//      one barrier each CTA merges its column slice, applies the gate, stores.
 // Only cluster barriers synchronise; nothing leaves the cluster but the
 // outputs, the state and the appended cache row.
 #include <cooperative_groups.h>
@@ -53,7 +54,7 @@ struct ScoreGeom {
 };
 
 struct DecLayout {
-  int region0, cand_key, cand_pos;
+  int region0, cand_key, cand_pos, pin;
   int keys, hist, tot, misc, sel, qs, qi, ks, vs, part, pml, olin, logit, sidx, bars, total;
 };
 
@@ -63,7 +64,8 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // 1024-byte aligned base (host and device agree; `total` includes the slack
 // needed to align the base).  region0 holds, one after the other in time: the
 // TMA ring (scoring), the candidate segments (selection, in CTA 0), and the
-// gathered K / V rows (attention).
+// gathered K / V rows (attention) followed by the partials that every rank
+// writes for this CTA's output columns (merge).
 __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, int G, int D, int DI, int esize,
                                                 int NC, int stages = kStages, int stage_bytes = kStageBytes) {
   DecLayout L;
@@ -71,12 +73,14 @@ __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, i
   const int kv = 2 * rpc * (D * esize + 16);
   const int ring = stages * stage_bytes;
   const int sel_bytes = 8 * kCandCap;
-  int r0 = ring > kv ? ring : kv;
+  const int kvp = align16(kv) + G * D * 4 + NC * 2 * G * 4;   // + [NC][G][D/NC] partials, [NC][2G] statistics
+  int r0 = ring > kvp ? ring : kvp;
   r0 = r0 > sel_bytes ? r0 : sel_bytes;
   int off = 0;
   L.region0 = off; off += align16(r0);
   L.cand_key = L.region0;
   L.cand_pos = L.region0 + 4 * kCandCap;
+  L.pin = L.region0 + align16(kv);
   L.keys = off; off += align16(kpc_max * 4);
   L.hist = off; off += 8 * 256 * 4;
   L.tot = off; off += 256 * 4;
@@ -987,34 +991,48 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       part[i] = a;
     }
   }
-  cluster.sync();                            // all partials of the cluster are ready
-
   // ---------------------------------------------------------------- merge + gate, columns of this CTA
-  // every rank's (max, sum) per head, copied once into this CTA
-  float *pml_all = reinterpret_cast<float *>(hist);     // [NC][2G]
-  for (int i = tid; i < NC * 2 * G; i += kDecThreads) pml_all[i] = cluster.map_shared_rank(pml, i / (2 * G))[i % (2 * G)];
-  __syncthreads();
-  for (int i = tid; i < G * COLS; i += kDecThreads) {
-    const int hh = i / COLS, c = i % COLS, d = c0s + c;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int r = 0; r < NC; ++r) mx = fmaxf(mx, pml_all[r * 2 * G + 2 * hh]);
-    float num = 0.f, den = 0.f;
-#pragma unroll
-    for (int r = 0; r < NC; ++r) {
-      const float mr = pml_all[r * 2 * G + 2 * hh];
-      if (mr == -INFINITY) continue;
-      const float f = expf(mr - mx);
-      num = fmaf(f, cluster.map_shared_rank(part, r)[hh * D + d], num);
-      den = fmaf(f, pml_all[r * 2 * G + 2 * hh + 1], den);
+  // each rank writes its partials of the columns [r*D/NC, (r+1)*D/NC) and its
+  // softmax statistics into CTA r; after one barrier every CTA merges from its
+  // own shared memory and nobody reads another CTA's memory again
+  {
+    __syncthreads();                           // part and pml are complete
+    for (int i = tid; i < G * D; i += kDecThreads) {
+      const int hh = i / D, d = i % D, owner = d / COLS, c = d % COLS;
+      float *pin_o = cluster.map_shared_rank(reinterpret_cast<float *>(smem + lay.pin), owner);
+      pin_o[(rank * G + hh) * COLS + c] = part[i];
     }
-    const int h = g * G + hh;
-    const float o_sp = num / den;
-    const float o_lin = olin[hh * COLS + c];
-    const float gam = 1.f / (1.f + expf(-p.gate[(size_t)b * p.Hq + h]));
-    reinterpret_cast<T *>(p.out)[((size_t)b * p.Hq + h) * D + d] = Dt<T>::from_f(gam * o_sp + (1.f - gam) * o_lin);
+    for (int i = tid; i < NC * 2 * G; i += kDecThreads) {
+      const int owner = i / (2 * G), j = i % (2 * G);
+      float *pin_o = cluster.map_shared_rank(reinterpret_cast<float *>(smem + lay.pin), owner);
+      pin_o[NC * G * COLS + rank * 2 * G + j] = pml[j];
+    }
   }
-  cluster.sync();                            // keep this CTA's shared memory alive for its readers
+  cluster.sync();                            // every partial of this CTA's columns has arrived
+  {
+    const float *pin = reinterpret_cast<const float *>(smem + lay.pin);
+    const float *pml_all = pin + NC * G * COLS;                 // [NC][2G]
+    for (int i = tid; i < G * COLS; i += kDecThreads) {
+      const int hh = i / COLS, c = i % COLS, d = c0s + c;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < NC; ++r) mx = fmaxf(mx, pml_all[r * 2 * G + 2 * hh]);
+      float num = 0.f, den = 0.f;
+#pragma unroll
+      for (int r = 0; r < NC; ++r) {
+        const float mr = pml_all[r * 2 * G + 2 * hh];
+        if (mr == -INFINITY) continue;
+        const float f = expf(mr - mx);
+        num = fmaf(f, pin[(r * G + hh) * COLS + c], num);
+        den = fmaf(f, pml_all[r * 2 * G + 2 * hh + 1], den);
+      }
+      const int h = g * G + hh;
+      const float o_sp = num / den;
+      const float o_lin = olin[hh * COLS + c];
+      const float gam = 1.f / (1.f + expf(-p.gate[(size_t)b * p.Hq + h]));
+      reinterpret_cast<T *>(p.out)[((size_t)b * p.Hq + h) * D + d] = Dt<T>::from_f(gam * o_sp + (1.f - gam) * o_lin);
+    }
+  }
 }
 
 // ============================================================ launcher
