@@ -297,6 +297,23 @@ def _capture(torch, stream, chains, items, fn):
     return g
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (the job's time) when several replicas run."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_rate(units_per_rank, ms, world):
+    """Whole-job units per second: every replica processes units_per_rank in
+    the (max-over-ranks) time ms."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def _timed_replays(torch, stream, graphs, barrier=None):
     """Device time (ms) of replaying `graphs` once each, in order."""
     if barrier:
@@ -362,12 +379,9 @@ def run_lisa(args, rank, world):
     ms = _timed_replays(torch, stream, [rot] * n_rot + ([tail] if tail else []), barrier)
     t_wall1 = time.time()
     clk.stop()
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, "cuda")
     ms_per_step = ms / args.steps
-    value = world * args.steps * cfg.B / (ms / 1e3)
+    value = replica_rate(args.steps * cfg.B, ms, world)
 
     # ---- one step at a time: the latency of a single decode step (one chain,
     #      the library's CTA split for one sequence)
