@@ -9,16 +9,17 @@
 // key tiles of N keys.  Per key tile the R head products Q_r K^T (128 x N,
 // K = dI) are accumulated in tensor memory; the epilogue turns them into
 // sum_r w_r * max(0, .), then into order keys, and stores the causal part
-// (key position <= query position).  Warp roles: warps 0-3 epilogue (one
-// thread per query row = one TMEM lane), warp 4 TMA producer, warp 5 MMA
-// issuer and TMEM owner.  Two accumulator buffers let the MMAs of one tile
-// overlap the epilogue of the previous one.
+// (key position <= query position).  Warp roles: warps 0-3 and 8-11
+// epilogue (one thread per query row = one TMEM lane; warps q and q + 8 take
+// the two halves of a tile's keys), warp 4 TMA producer, warp 5 MMA issuer
+// and TMEM owner.  Two accumulator buffers let the MMAs of one tile overlap
+// the epilogue of the previous one.
 #include "lisa_internal.h"
 #include "lisa_tc.cuh"
 
 namespace lisa {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 384;   // warps 0-3 and 8-11 epilogue, 4 TMA, 5 MMA, 6-7 idle
 constexpr int kTcStages = 4;
 constexpr int kTcKeyTilesPerCta = 8;
 constexpr int kTcRows = 128;
@@ -26,9 +27,15 @@ constexpr int kTcRows = 128;
 // Keys per tile: 2 buffers x R accumulators x N columns fill the 512 TMEM columns.
 __host__ __device__ inline int tc_tile_n(int R) { return R <= 1 ? 256 : R <= 2 ? 128 : R <= 4 ? 64 : 32; }
 
+// Epilogue staging: per epilogue warp 32 rows x 32 keys, rows padded to 36
+// words (16-byte aligned, conflict-free for the row-wise writes and the
+// transposed reads).
+constexpr int kStageRowWords = 36;
+constexpr int kStageWarpWords = 32 * kStageRowWords;
+
 __host__ __device__ inline int tc_smem_bytes(int R, int DI) {
   const int RB = DI * 2;
-  return 1024 + R * kTcRows * RB + kTcStages * tc_tile_n(R) * RB + 256;
+  return 1024 + R * kTcRows * RB + kTcStages * tc_tile_n(R) * RB + 256 + 8 * kStageWarpWords * 4;
 }
 
 template <int DI>
@@ -65,6 +72,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t *acc_full = bars + 1 + 2 * kTcStages;
   uint64_t *acc_empty = bars + 3 + 2 * kTcStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5 + 2 * kTcStages);
+  unsigned char *bars_end = reinterpret_cast<unsigned char *>(bars) + 256;   // staging of the epilogue warps
   constexpr uint32_t kTmemCols = 512;
 
   if (tid == 0) {
@@ -75,7 +83,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4 * 32);
+      mbar_init(&acc_empty[i], 8 * 32);
     }
     fence_mbar_init();
   }
@@ -124,50 +132,73 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_commit(&acc_full[buf]);   // the accumulators of this tile are ready
       }
     }
-  } else {
+  } else if (warp < 4 || warp >= 8) {
     // ------------------------------------------------------------ epilogue: thread = query row
-    const int row = warp * 32 + lane;
+    // Warps q and q + 8 share TMEM lanes 32q..32q+31 (one query row per
+    // thread) and split the key columns of a tile.  Scores of 32 keys per row
+    // are staged in shared memory, then written row-wise: 8 lanes cover 128
+    // contiguous bytes of one row, so a warp store touches 4 rows, not 32.
+    const int qd = warp & 3, hsel = warp >= 8 ? 1 : 0;
+    const int cbeg = N >= 64 ? hsel * (N / 2) : 0;
+    const int cend = N >= 64 ? cbeg + N / 2 : (hsel ? 0 : N);
+    const int row = qd * 32 + lane;
     const int rr = r_lo + row;
     const bool row_ok = rr < r_hi;
-    const int tpos = p0 + tau0 + rr;
     float wr[kMaxR];
 #pragma unroll
     for (int r = 0; r < kMaxR; ++r)
       wr[r] = (row_ok && r < R) ? p.w[((size_t)b * p.T + tau0 + rr) * p.HI + g * R + r] : 0.f;
-    uint32_t *krow = p.keys + ((size_t)bg * p.row_chunk + (row_ok ? rr : 0)) * p.L_keys;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    uint32_t *stg = reinterpret_cast<uint32_t *>(bars_end) + (qd + 4 * hsel) * kStageWarpWords;
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const int wrow = lane >> 3, wcol = (lane & 7) * 4;          // write-out: row within 4, key offset
     for (int it = 0; it < ntiles; ++it) {
       const int buf = it & 1;
       if (!mbar_wait_bounded(&acc_full[buf], (uint32_t)((it >> 1) & 1)) && lane == 0)
         set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+      __syncwarp();
       tc_fence_after();
       const int s0 = (kt0 + it) * N;
-      for (int c = 0; c < N; c += 16) {
-        float acc[16];
+      for (int c = cbeg; c < cend; c += 32) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-#pragma unroll 1
-        for (int r = 0; r < R; ++r) {
-          uint32_t v[16];
-          tc_ld16(tmem + lane_base + (uint32_t)((buf * R + r) * N + c), v);
-          tc_wait_ld();
+        for (int half = 0; half < 2; ++half) {
+          float acc[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[j] = fmaf(wr[r], fmaxf(__uint_as_float(v[j]), 0.f), acc[j]);
+          for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+#pragma unroll
+          for (int r = 0; r < kMaxR; ++r) {
+            if (r >= R) break;
+            uint32_t v[16];
+            tc_ld16(tmem + lane_base + (uint32_t)((buf * R + r) * N + c + 16 * half), v);
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = fmaf(wr[r], fmaxf(__uint_as_float(v[j]), 0.f), acc[j]);
+          }
+          uint4 *sd = reinterpret_cast<uint4 *>(stg + lane * kStageRowWords + 16 * half);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            sd[q] = make_uint4(score_key(acc[4 * q]), score_key(acc[4 * q + 1]), score_key(acc[4 * q + 2]),
+                               score_key(acc[4 * q + 3]));
         }
-        if (row_ok) {
-          const int sc = s0 + c;
-          if (sc + 15 <= tpos) {
-            uint4 *dst = reinterpret_cast<uint4 *>(krow + sc);
+        __syncwarp();
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(score_key(acc[4 * q]), score_key(acc[4 * q + 1]), score_key(acc[4 * q + 2]),
-                                  score_key(acc[4 * q + 3]));
-          } else if (sc <= tpos) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (sc + j <= tpos) krow[sc + j] = score_key(acc[j]);
+        for (int k = 0; k < 8; ++k) {
+          const int rloc = 4 * k + wrow;
+          const int rr2 = r_lo + qd * 32 + rloc;
+          const int sc = s0 + c + wcol;
+          const int tpos2 = p0 + tau0 + rr2;
+          if (rr2 < r_hi && sc <= tpos2) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(stg + rloc * kStageRowWords + wcol);
+            uint32_t *gd = p.keys + ((size_t)bg * p.row_chunk + rr2) * p.L_keys + sc;
+            if (sc + 3 <= tpos2) {
+              *reinterpret_cast<uint4 *>(gd) = v;
+            } else {
+              gd[0] = v.x;
+              if (sc + 1 <= tpos2) gd[1] = v.y;
+              if (sc + 2 <= tpos2) gd[2] = v.z;
+            }
           }
         }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
