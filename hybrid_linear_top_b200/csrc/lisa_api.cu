@@ -36,7 +36,7 @@ size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int round4(int x) { return (x + 3) & ~3; }
 
-constexpr int kRowsKeysCap = 16384;     // same, for the 256-thread row select
+constexpr int kRowsStagedCap = 2048;   // keys of a row staged in shared memory by the row select
 constexpr int kCandCap = 4096;          // threshold-bucket candidates kept in shared memory
 constexpr int kRowChunk = 2048;         // query rows scored per pass on the row path
 constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory a CTA may use on sm_100
@@ -111,7 +111,9 @@ void fill_rows(lisa::RowsParams &r, const lisa_layer *L, int T) {
 }
 
 void set_select_smem(lisa::RowsParams &r, int n_max) {
-  const int cap = n_max < kRowsKeysCap ? n_max : kRowsKeysCap;
+  // rows of up to 2048 keys are staged in shared memory; longer rows are read
+  // from global memory by the bounded select
+  const int cap = n_max < kRowsStagedCap ? n_max : kRowsStagedCap;
   r.smem_keys_cap = (cap + 3) & ~3;
   r.cand_cap = kCandCap;
   r.select_smem = (size_t)(r.smem_keys_cap + 2 * r.cand_cap) * 4;   // keys, candidate keys and positions

@@ -170,9 +170,10 @@ __global__ void __launch_bounds__(NT) rows_select_kernel(RowsParams p, int tau0,
     cand = s_dyn + p.smem_keys_cap;
   }
   int *out = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M;
-  if (keys == s_dyn && n >= 8 * NT) {
-    // long rows: a bound from every thread's 4 largest keys, then an exact
-    // select among the few keys above it
+  if (n >= 8 * NT) {
+    // long rows (read from global memory / L2, not staged, so that several
+    // rows share an SM): a bound from every thread's 4 largest keys, then an
+    // exact select among the few keys above it
     __shared__ BoundedShared bsm;
     const int r = block_topm_bounded<NT>(keys, n, p.M, out, bsm, cand, reinterpret_cast<int *>(cand + p.cand_cap),
                                          p.cand_cap);
