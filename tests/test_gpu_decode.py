@@ -144,14 +144,26 @@ def test_decode_without_fused_append():
     run_decode(cfg, lay, step, np.array([2047, 1000, 5]), 2048, fuse_append=False, pre_append=True)
 
 
+@pytest.mark.parametrize("split", [0, 4, 8])
 @pytest.mark.parametrize("dtype,d,dI", [("bf16", 64, 32), ("bf16", 128, 32), ("bf16", 64, 64),
                                         ("fp32", 64, 32), ("fp32", 128, 64)])
-def test_decode_other_shapes(dtype, d, dI):
+def test_decode_other_shapes(dtype, d, dI, split):
     cfg = _replace(get_config("decode_1p5b_16k"), B=2, Hq=8, Hkv=2, HI=2, d=d, dI=dI, M=64, dtype=dtype, L=1500)
     rng = make_rng(13, 0)
     lay = gen_layer(cfg, rng, 1499)
     step = gen_step(cfg, rng, 1)
-    run_decode(cfg, lay, step, np.array([1499, 700]), 1500)
+    run_decode(cfg, lay, step, np.array([1499, 700]), 1500, split=split)
+
+
+@pytest.mark.parametrize("split", [4, 16])
+def test_decode_largest_groups_and_m(split):
+    """16 query heads and 8 indexer heads per KV head, M = 1024 (the largest
+    supported values)."""
+    cfg = _replace(get_config("decode_1p5b_16k"), B=1, Hq=32, Hkv=2, HI=16, M=1024, L=9000)
+    rng = make_rng(17, 0)
+    lay = gen_layer(cfg, rng, 8999)
+    step = gen_step(cfg, rng, 1)
+    run_decode(cfg, lay, step, np.array([8999]), 9000, split=split)
 
 
 def test_decode_bad_position_sets_error_word():

@@ -149,3 +149,16 @@ def test_indexer_topk_rows_match_prefill_sets():
         sc = oracle.indexer_scores(a(step.qidx[0, t]), a(step.w[0, t]), keys[:, : t + 1])
         for g in range(cfg.Hkv):
             check_set(idx_g[0, t, g], sc[g], cfg.M, t, where=f"t={t} g={g}")
+
+
+@pytest.mark.parametrize("d,dI,HI,Hq,M", [(64, 32, 8, 8, 64), (128, 64, 2, 8, 128), (128, 32, 16, 32, 64)])
+def test_prefill_other_shapes(d, dI, HI, Hq, M):
+    """Other head dims, 1..8 indexer heads per KV head (every tcgen05 tile
+    width), 4..16 query heads per KV head, M below T."""
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=700, B=1, Hq=Hq, Hkv=2, d=d, dI=dI, HI=HI, M=M,
+                              S0="normal")
+    rng = make_rng(300 + d + HI, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = gen_step(cfg, rng, 700)
+    lay, out, idx = gpu_prefill(cfg, layer_np, step, 700, 710)
+    check_prefill(cfg, layer_np, step, lay, out, idx)
