@@ -488,13 +488,160 @@ def run_prefill(args, rank, world):
                           "config": {"workload": "prefill_1p5b_16k", "T": cfg.T, "M": cfg.M}}), flush=True)
 
 
+def _decode_bytes(cfg, L, B=None):
+    """Algorithmic bytes of one decode step of one layer: algorithmic_bytes()
+    per sequence (context L, or the per-sequence lengths L)."""
+    Ls = np.broadcast_to(np.asarray(L), (cfg.B if B is None else B,))
+    return int(sum(algorithmic_bytes(cfg, int(l)) for l in Ls))
+
+
+def _fill_layer(L, lay, cfg, n_rows, g, torch):
+    bf = torch.bfloat16
+    rn = lambda shape, dim: (torch.randn(shape, generator=g, device="cuda") / dim ** 0.5).to(bf)
+    lay.k_cache[:, :, :n_rows] = rn((cfg.B, cfg.Hkv, n_rows, cfg.d), cfg.d)
+    lay.v_cache[:, :, :n_rows] = rn((cfg.B, cfg.Hkv, n_rows, cfg.d), cfg.d)
+    lay.kidx_cache[:, :, :n_rows] = rn((cfg.B, cfg.Hkv, n_rows, cfg.dI), cfg.dI)
+    lay.state.copy_(torch.randn(lay.state.shape, generator=g, device="cuda"))
+
+
+def _step_inputs(cfg, g, torch):
+    bf = torch.bfloat16
+    rn = lambda shape, dim: (torch.randn(shape, generator=g, device="cuda") / dim ** 0.5).to(bf)
+    return dict(q=rn((cfg.B, cfg.Hq, cfg.d), cfg.d), k=rn((cfg.B, cfg.Hkv, cfg.d), cfg.d),
+                v=rn((cfg.B, cfg.Hkv, cfg.d), cfg.d), kidx=rn((cfg.B, cfg.Hkv, cfg.dI), cfg.dI),
+                qidx=rn((cfg.B, cfg.HI, cfg.dI), cfg.dI), w=torch.rand((cfg.B, cfg.HI), generator=g, device="cuda"),
+                lam=torch.randn((cfg.B, cfg.Hq), generator=g, device="cuda"))
+
+
+def _line(rank, metric, value, unit, args, world, ms_per_step, config, roofline, extra=None):
+    if rank != 0:
+        return
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/sqrt(dim) inputs)",
+            "config": config, "roofline": roofline}
+    line.update(extra or {})
+    print(json.dumps(line), flush=True)
+
+
+def run_ragged(args, rank, world):
+    """Qwen2.5-7B-shaped batched decode step: B=32 sequences with context
+    lengths drawn uniformly in [4096, 16384] (one lisa_decode_step call)."""
+    import torch
+    from hybrid_linear_top_b200 import lisa as L
+    from lisa_inputs.gen import gen_lengths
+    cfg = get_config("ragged_7b_b32")
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    lengths = gen_lengths(cfg, make_rng(cfg.seed, 0))
+    step_bytes = _decode_bytes(cfg, lengths)
+    l2 = getattr(torch.cuda.get_device_properties(0), "L2_cache_size", 126 * 2 ** 20)
+    R = max(2, int(np.ceil(4 * l2 / step_bytes)))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 * rank + 3)
+    lays, xs = [], []
+    for _ in range(R):
+        lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.L_max, L.LISA_BF16,
+                               decode_split=args.split)
+        _fill_layer(L, lay, cfg, cfg.L_max - 1, g, torch)
+        lay.pos.copy_(torch.from_numpy((lengths - 1).astype(np.int32)))
+        lays.append(lay)
+        xs.append(_step_inputs(cfg, g, torch))
+    out = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def one(i, s_):
+        x = xs[i % R]
+        L.lisa_decode_step(lays[i % R], x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, out,
+                           None, None, s_)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            one(i, stream)
+    n_graph = min(args.steps, 64 * R)
+    gr = _capture(torch, stream, [stream], list(range(n_graph)), one)
+    reps, tail_n = divmod(args.steps, n_graph)
+    tail = _capture(torch, stream, [stream], list(range(tail_n)), one) if tail_n else None
+    gr.replay()
+    ms = _timed_replays(torch, stream, [gr] * reps + ([tail] if tail else []))
+    ms = max_over_ranks(ms, world, "cuda")
+    if any(int(l.err_word.item()) for l in lays):
+        raise RuntimeError("device-side checks flagged the ragged decode")
+    peak, kind = load_peaks()
+    per = ms / args.steps
+    achieved = step_bytes / (per * 1e-3) / 1e9
+    _line(rank, "LISA decode tokens/s, 7B shape, B=32 ragged 4K-16K, M=256", replica_rate(args.steps * cfg.B, ms, world),
+          "tokens/s", args, world, per,
+          {"workload": "ragged_7b_b32", "B": cfg.B, "L_range": [cfg.L_lo, cfg.L_hi], "M": cfg.M, "instances": R,
+           "decode_split": args.split or "library", "parallelism": f"replicas x{world}"},
+          {"bound": "hbm", "kernel": "decode_cluster_kernel", "achieved": achieved, "peak": peak, "unit": "GB/s",
+           "frac": achieved / peak, "peak_kind": kind, "algorithmic_bytes_per_launch": step_bytes, "traffic": None})
+
+
+def run_longcot(args, rank, world):
+    """Qwen2.5-7B-shaped long chain of thought: 28 independent layers, B=8,
+    16384 prefilled rows, 1024 sequential decode steps per layer (each
+    appending its token); the layers run as 28 concurrent chains."""
+    import torch
+    from hybrid_linear_top_b200 import lisa as L
+    cfg = get_config("longcot_7b_28l")
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    n_steps = cfg.n_decode
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 * rank + 4)
+    lays, pools = [], []
+    for _ in range(cfg.layers):
+        lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.L_max, L.LISA_BF16,
+                               decode_split=args.split)
+        _fill_layer(L, lay, cfg, cfg.L, g, torch)
+        lays.append(lay)
+        pools.append([_step_inputs(cfg, g, torch) for _ in range(4)])     # step inputs cycle over 4 draws
+    # pos of step n = L + n for every sequence: one 16-byte aligned row per step
+    pos_all = (torch.arange(n_steps, device="cuda", dtype=torch.int32)[:, None] + cfg.L).repeat(1, cfg.B).contiguous()
+    out = torch.empty(cfg.layers, cfg.B, cfg.Hq, cfg.d, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.Stream()
+    chains = [torch.cuda.Stream() for _ in range(cfg.layers)]
+
+    def one(item, s_):
+        l, n = item
+        lay = lays[l]
+        lay.pos = pos_all[n]
+        x = pools[l][n % 4]
+        L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, out[l], None,
+                           None, s_)
+
+    block = 64
+    graphs = []
+    for n0 in range(0, n_steps, block):
+        items = [(l, n) for n in range(n0, min(n_steps, n0 + block)) for l in range(cfg.layers)]
+        graphs.append(_capture(torch, stream, chains, items, one))
+    # warm-up: one pass over a few steps (rewrites the same rows the timed pass writes)
+    graphs[0].replay()
+    torch.cuda.synchronize()
+    ms = _timed_replays(torch, stream, graphs)
+    ms = max_over_ranks(ms, world, "cuda")
+    if any(int(l.err_word.item()) for l in lays):
+        raise RuntimeError("device-side checks flagged the long-CoT decode")
+    total_bytes = cfg.layers * sum(_decode_bytes(cfg, cfg.L + n + 1) for n in range(n_steps))
+    peak, kind = load_peaks()
+    achieved = total_bytes / (ms * 1e-3) / 1e9
+    _line(rank, "LISA long-CoT decode tokens/s, 7B shape, 28 layers, B=8, 16K->17K, M=256",
+          replica_rate(cfg.B * n_steps, ms, world), "tokens/s", args, world, ms / n_steps,
+          {"workload": "longcot_7b_28l", "B": cfg.B, "layers": cfg.layers, "steps": n_steps, "L0": cfg.L,
+           "decode_split": args.split or "library", "concurrent_chains": cfg.layers,
+           "parallelism": f"replicas x{world}"},
+          {"bound": "hbm", "kernel": "decode_cluster_kernel", "achieved": achieved, "peak": peak, "unit": "GB/s",
+           "frac": achieved / peak, "peak_kind": kind, "algorithmic_bytes_total": total_bytes, "traffic": None},
+          {"note": "steps = sequential decode steps of every layer; value = B x steps / time of the whole stack"})
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "prefill_1p5b_16k"])
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l"])
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--streams", type=int, default=32)
     ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16])
@@ -502,6 +649,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.steps is None:
+        args.steps = {WORKLOAD: 200000, "prefill_1p5b_16k": 20, "ragged_7b_b32": 2000,
+                      "longcot_7b_28l": 1024}[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if world > 1:
@@ -515,6 +665,10 @@ def main():
             run_reference(args, rank, world)
         elif args.workload == "prefill_1p5b_16k":
             run_prefill(args, rank, world)
+        elif args.workload == "ragged_7b_b32":
+            run_ragged(args, rank, world)
+        elif args.workload == "longcot_7b_28l":
+            run_longcot(args, rank, world)
         else:
             run_lisa(args, rank, world)
     finally:
