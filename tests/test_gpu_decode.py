@@ -262,3 +262,32 @@ def test_decode_all_scores_equal(L_ctx, split):
     step.w = np.zeros_like(step.w)
     res = run_decode(cfg, lay, step, np.array([L_ctx - 1]), L_ctx, exact_sets=True, split=split)
     assert res["ndiff"] == 0
+
+
+def test_decode_inputs_and_output_in_pinned_host_memory():
+    """The step's inputs may live in pinned host memory and the output may go
+    there (the kernel reads and writes them across the host link)."""
+    cfg = _replace(get_config("decode_1p5b_16k"), B=2, L=5000)
+    rng = make_rng(23, 0)
+    layer_np = gen_layer(cfg, rng, 4999)
+    step = gen_step(cfg, rng, 1)
+    pos = np.array([4999, 2500])
+    lay = make_layer(L, cfg, 5000, layer_np, n_rows=4999)
+    lay.pos.copy_(torch.from_numpy(pos.astype(np.int32)))
+    x = {k: v.cpu().pin_memory() for k, v in step_tensors(step, cfg, tau=0).items()}
+    out = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=lay.torch_dtype).pin_memory()
+    idx = torch.empty(cfg.B, cfg.Hkv, cfg.M, dtype=torch.int32, device="cuda")
+    L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, out, idx, None)
+    torch.cuda.synchronize()
+    assert int(lay.err_word.item()) == 0
+    kc, vc, kic = (z.astype(np.float64) for z in (layer_np.k_cache, layer_np.v_cache, layer_np.kidx_cache))
+    s0 = lambda a: a[:, 0].astype(np.float64)
+    idx_g = idx.cpu().numpy().astype(np.int64)
+    ref = oracle.decode_step(s0(step.q), s0(step.k), s0(step.v), s0(step.qidx), s0(step.kidx), s0(step.w),
+                             s0(step.lam), kc, vc, kic, layer_np.S0.astype(np.float64), pos, cfg.M,
+                             sel_override=idx_g)
+    for b in range(cfg.B):
+        for g in range(cfg.Hkv):
+            check_set(idx_g[b, g], ref["scores"][b][g], cfg.M, int(pos[b]), where=f"b={b} g={g}")
+    check_out(f64(out), ref["out"], cfg.dtype, where="out")
+    check_state(f64(lay.state), ref["S"], where="state")
