@@ -8,6 +8,7 @@ baseline legs of ``bench.py`` do.  It shares no code with the CUDA path.
 from .lisa_ref import (
     indexer_scores,
     topm_select,
+    window_select,
     topm_threshold,
     borderline_mask,
     sparse_attention,
@@ -21,6 +22,7 @@ from .lisa_ref import (
 __all__ = [
     "indexer_scores",
     "topm_select",
+    "window_select",
     "topm_threshold",
     "borderline_mask",
     "sparse_attention",

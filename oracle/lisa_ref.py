@@ -82,6 +82,22 @@ def topm_select(scores: np.ndarray, M: int) -> np.ndarray:
     return out
 
 
+def window_select(t: int, W: int) -> np.ndarray:
+    """Stage-1 inference variant (arxivdaily.com English abstract: Stage 1
+    pairs the linear attention with a sliding-window attention that the
+    Indexer later replaces; iitog.ru article, key facts): the sparse branch
+    attends to the W most recent positions max(0, t-W+1) .. t, listed in
+    ascending position, padded with -1 up to W entries.
+
+    Parity: pinned against topm_select on scores that increase with the
+    position (the top-W of such scores is the last W positions)."""
+    lo = max(0, t - W + 1)
+    out = np.full(W, -1, dtype=np.int64)
+    keep = np.arange(lo, t + 1, dtype=np.int64)
+    out[: keep.shape[0]] = keep
+    return out
+
+
 def topm_threshold(scores: np.ndarray, M: int) -> float:
     """Score of the M-th entry of the order (the lowest selected score)."""
     n = scores.shape[0]

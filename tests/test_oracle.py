@@ -259,3 +259,31 @@ def test_generators_deterministic():
     np.testing.assert_array_equal(a.q, b.q)
     c = gen_step(cfg, make_rng(cfg.seed, 1))
     assert not np.array_equal(a.q, c.q)
+
+
+@pytest.mark.parametrize("t,W", [(0, 32), (5, 32), (31, 32), (32, 32), (100, 32), (1000, 256)])
+def test_window_is_top_of_position_ordered_scores(t, W):
+    """The sliding window is the top-W of scores that grow with the position,
+    through the full sort of the top-M selection (an independent route)."""
+    scores = np.linspace(0.1, 1.0, t + 1)
+    np.testing.assert_array_equal(oracle.window_select(t, W), oracle.topm_select(scores, W))
+    w = oracle.window_select(t, W)
+    valid = w[w >= 0]
+    assert valid.size == min(W, t + 1) and valid[-1] == t and np.all(np.diff(valid) == 1)
+
+
+def test_window_decode_with_full_window_is_causal_attention():
+    """With W >= t + 1 the window variant attends to the whole prefix: the
+    sparse branch equals full causal softmax attention (separate loop)."""
+    rng = np.random.default_rng(5)
+    t, d = 6, 8
+    K = rng.standard_normal((t + 1, d))
+    V = rng.standard_normal((t + 1, d))
+    q = rng.standard_normal(d)
+    sel = oracle.window_select(t, 32)
+    sel = sel[sel >= 0]
+    o = oracle.sparse_attention(q, K[sel], V[sel])
+    logits = np.array([q @ K[s] for s in range(t + 1)]) / np.sqrt(d)
+    p = np.exp(logits - logits.max())
+    p /= p.sum()
+    np.testing.assert_allclose(o, sum(p[s] * V[s] for s in range(t + 1)), rtol=1e-12, atol=1e-12)
