@@ -550,6 +550,49 @@ def _line(rank, metric, value, unit, args, world, ms_per_step, config, roofline,
     print(json.dumps(line), flush=True)
 
 
+def run_window(args, rank, world):
+    """Stage-1 sliding-window variant at the 1.5B decode shape: the last 256
+    positions instead of the indexer's top-256 (lisa_decode_step_window),
+    16384 cached tokens, 32 concurrent chains over independent instances."""
+    import torch
+    from hybrid_linear_top_b200 import lisa as L
+    cfg = get_config(WORKLOAD)
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    l2 = getattr(torch.cuda.get_device_properties(0), "L2_cache_size", 126 * 2 ** 20)
+    M = min(cfg.M, cfg.L)
+    small = (cfg.Hq * cfg.d * 2 + 4 * cfg.Hkv * cfg.d * 2 + cfg.Hq * 4 + cfg.Hq * cfg.d * 2)
+    step_bytes = cfg.Hkv * M * 2 * cfg.d * 2 + cfg.Hq * cfg.d * cfg.d * 4 * 2 + small
+    S = max(1, args.streams)
+    # instances: enough that the step footprint (window rows, state) exceeds 4x L2
+    R = -(-max(int(np.ceil(4 * l2 / step_bytes)), S) // S) * S
+    inst = [Instance(L, cfg, torch, 2000 * rank + i, None, args.split) for i in range(R)]
+    stream = torch.cuda.Stream()
+    chains = [torch.cuda.Stream() for _ in range(S)]
+    run = lambda x, s_: L.lisa_decode_step_window(x.lay, x.q, x.k, x.v, x.kidx, x.lam, 1, x.out, None, s_)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            run(inst[i % R], stream)
+    per_graph = R * max(1, -(-2048 // R))
+    per_graph = min(per_graph, max(R, args.steps // R * R))
+    n_rot, n_tail = divmod(args.steps, per_graph)
+    rot = _capture(torch, stream, chains, [inst[i % R] for i in range(per_graph)], run)
+    tail = _capture(torch, stream, chains, [inst[i % R] for i in range(n_tail)], run) if n_tail else None
+    rot.replay()
+    ms = max_over_ranks(_timed_replays(torch, stream, [rot] * n_rot + ([tail] if tail else [])), world, "cuda")
+    if any(int(x.lay.err_word.item()) for x in inst):
+        raise RuntimeError("device-side checks flagged the window decode")
+    peak, kind = load_peaks()
+    per = ms / args.steps
+    achieved = step_bytes / (per * 1e-3) / 1e9
+    _line(rank, "LISA Stage-1 window decode tokens/s @16K ctx, W=256", replica_rate(args.steps * cfg.B, ms, world),
+          "tokens/s", args, world, per,
+          {"workload": "window_1p5b_16k", "B": cfg.B, "L": cfg.L, "W": M, "instances": R, "concurrent_chains": S,
+           "decode_split": args.split or "library", "parallelism": f"replicas x{world}"},
+          {"bound": "hbm", "kernel": "decode_cluster_kernel (window mode)", "achieved": achieved, "peak": peak,
+           "unit": "GB/s", "frac": achieved / peak, "peak_kind": kind, "algorithmic_bytes_per_launch": step_bytes,
+           "traffic": None})
+
+
 def run_ragged(args, rank, world):
     """Qwen2.5-7B-shaped batched decode step: B=32 sequences with context
     lengths drawn uniformly in [4096, 16384] (one lisa_decode_step call)."""
@@ -667,7 +710,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l"])
+                    choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l", "window_1p5b_16k"])
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--streams", type=int, default=32)
     ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16])
@@ -677,7 +720,7 @@ def main():
     args.warmup = max(3, args.warmup)
     if args.steps is None:
         args.steps = {WORKLOAD: 200000, "prefill_1p5b_16k": 20, "ragged_7b_b32": 2000,
-                      "longcot_7b_28l": 1024}[args.workload]
+                      "longcot_7b_28l": 1024, "window_1p5b_16k": 200000}[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if world > 1:
@@ -695,6 +738,8 @@ def main():
             run_ragged(args, rank, world)
         elif args.workload == "longcot_7b_28l":
             run_longcot(args, rank, world)
+        elif args.workload == "window_1p5b_16k":
+            run_window(args, rank, world)
         else:
             run_lisa(args, rank, world)
     finally:

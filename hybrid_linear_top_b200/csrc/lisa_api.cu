@@ -82,13 +82,13 @@ struct RowsPlan {
   int row_chunk, L_keys;
   size_t keys, idx, olin, dS, Ptot, total;
 };
-RowsPlan rows_plan(const lisa_layer *L, int T, bool prefill) {
+RowsPlan rows_plan(const lisa_layer *L, int T, bool prefill, bool indexer = true) {
   RowsPlan p;
   const size_t BH = (size_t)L->B * L->Hkv;
   p.row_chunk = T < kRowChunk ? T : kRowChunk;
   p.L_keys = round4(prefill ? T : L->L_max);
   size_t off = 0;
-  p.keys = off; off += round256(BH * p.row_chunk * p.L_keys * 4);
+  p.keys = off; off += indexer ? round256(BH * p.row_chunk * p.L_keys * 4) : 0;
   p.idx = p.olin = p.dS = p.Ptot = 0;
   if (prefill) {
     const size_t nc = (T + lisa::kLinChunk - 1) / lisa::kLinChunk;
@@ -198,6 +198,7 @@ size_t lisa_workspace_bytes(const lisa_layer *layer, int T, int op) {
   if (op == LISA_OP_DECODE) return 0;   // the decode step keeps its intermediates on chip
   if (op == LISA_OP_PREFILL) return T ? rows_plan(layer, T, true).total : 0;
   if (op == LISA_OP_INDEXER_TOPK) return T ? rows_plan(layer, T, false).total : 0;
+  if (op == LISA_OP_PREFILL_WINDOW) return T ? rows_plan(layer, T, true, false).total : 0;
   return 0;
 }
 
@@ -274,6 +275,80 @@ lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, 
   p.out = out; p.idx_out = idx_out;
   cudaError_t e = lisa::launch_decode(p, L->dtype, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode_step");
+  return ok();
+}
+
+lisa_status lisa_decode_step_window(const lisa_layer *L, const void *q, const void *k, const void *v,
+                                    const void *kidx, const float *gate_logit, int fuse_append, void *out,
+                                    int *idx_out, void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (L->B == 0) return ok();
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(L->state, "state"))) return s;
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
+      (s = check_ptr(kidx, "kidx", false)) || (s = check_ptr(gate_logit, "gate_logit")) ||
+      (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)))
+    return s;
+  const int esz = L->dtype == LISA_BF16 ? 2 : 4;
+  if (lisa::decode_smem_bytes(L->L_max, L->M, L->Hq / L->Hkv, L->d, L->dI, esz, 8) > kMaxSmem)
+    return fail(LISA_ERR_UNSUPPORTED, "L_max=%d needs more shared memory per CTA than a B200 SM has", L->L_max);
+  lisa::DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.B = L->B; p.Hq = L->Hq; p.Hkv = L->Hkv; p.G = L->Hq / L->Hkv; p.HI = L->HI; p.R = L->HI / L->Hkv;
+  p.D = L->d; p.DI = L->dI; p.M = L->M; p.L_max = L->L_max; p.fuse_append = fuse_append ? 1 : 0;
+  p.split_req = L->decode_split;
+  p.window = 1;
+  p.scale = (float)(1.0 / sqrt((double)L->d));
+  p.k_cache = L->k_cache; p.v_cache = L->v_cache; p.kidx_cache = L->kidx_cache;
+  p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;
+  p.q = q; p.k = k; p.v = v; p.kidx = kidx; p.qidx = nullptr; p.w = nullptr; p.gate = gate_logit;
+  p.out = out; p.idx_out = idx_out;
+  cudaError_t e = lisa::launch_decode(p, L->dtype, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step_window");
+  return ok();
+}
+
+lisa_status lisa_prefill_window(const lisa_layer *L, int T, const void *q, const void *k, const void *v,
+                                const void *kidx, const float *gate_logit, void *out, int *idx_out, void *workspace,
+                                size_t ws_bytes, void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(L->state, "state"))) return s;
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
+      (s = check_ptr(kidx, "kidx", false)) || (s = check_ptr(gate_logit, "gate_logit")) ||
+      (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)))
+    return s;
+  const RowsPlan plan = rows_plan(L, T, true, false);
+  if (!workspace || ws_bytes < plan.total)
+    return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
+  if ((s = check_ptr(workspace, "workspace"))) return s;
+
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.require_pos0 = 1;
+  r.q = q; r.k = k; r.v = v; r.kidx = kidx; r.qidx = nullptr; r.w = nullptr; r.gate = gate_logit; r.out = out;
+  char *ws = static_cast<char *>(workspace);
+  r.keys = nullptr;
+  r.idx = idx_out ? idx_out : reinterpret_cast<int *>(ws + plan.idx);
+  r.olin = reinterpret_cast<float *>(ws + plan.olin);
+  r.dS = reinterpret_cast<float *>(ws + plan.dS);
+  r.Ptot = reinterpret_cast<float *>(ws + plan.Ptot);
+  r.row_chunk = plan.row_chunk;
+  r.L_keys = plan.L_keys;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = lisa::launch_append(r, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_window append");
+  e = lisa::launch_prefill_linear(r, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_window linear");
+  e = lisa::launch_window_idx(r, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_window index");
+  e = lisa::launch_prefill_attend(r, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_window attend");
   return ok();
 }
 

@@ -223,13 +223,16 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     ks[i] = Dt<T>::to_f(kin[i]);
     vs[i] = Dt<T>::to_f(vin[i]);
   }
-  for (int i = tid; i < R * DI; i += kDecThreads)
-    qis[i] = Dt<T>::to_f(reinterpret_cast<const T *>(p.qidx)[((size_t)b * p.HI + g * R) * DI + i]);
-  if (tid < R) qis[kMaxR * DI + tid] = p.w[(size_t)b * p.HI + g * R + tid];
+  const bool window = p.window != 0;      // sliding-window variant: no indexer, no top-M
+  if (!window) {
+    for (int i = tid; i < R * DI; i += kDecThreads)
+      qis[i] = Dt<T>::to_f(reinterpret_cast<const T *>(p.qidx)[((size_t)b * p.HI + g * R) * DI + i]);
+    if (tid < R) qis[kMaxR * DI + tid] = p.w[(size_t)b * p.HI + g * R + tid];
+  }
   // MMA operand B (indexer queries, heads = columns, padded to 8) and the head weights of this lane
   uint32_t bq[DI / 16][2];
   float wq0 = 0.f, wq1 = 0.f;
-  if constexpr (SG::kMma) {
+  if (SG::kMma && !window) {
     const int nh = lane >> 2, kc = 2 * (lane & 3);
     const uint32_t *qrow = reinterpret_cast<const uint32_t *>(reinterpret_cast<const T *>(p.qidx) +
                                                                ((size_t)b * p.HI + g * R + (nh < R ? nh : 0)) * DI);
@@ -250,7 +253,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   const int k0 = min(n, rank * kpc);
   const int k1 = min(n, k0 + kpc);
   const int cnt = k1 - k0;
-  const int nsub = (cnt + SUB - 1) / SUB;
+  const int nsub = window ? 0 : (cnt + SUB - 1) / SUB;
 
   // ---------------------------------------------------------------- TMA ring
   auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS, and sub-chunk i + NS -> L2
@@ -288,7 +291,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       kc[i] = kin[i];
       vc[i] = vin[i];
     }
-    for (int i = tid; i < DI; i += kDecThreads) kic[i] = kidx_new[i];
+    if (p.kidx)
+      for (int i = tid; i < DI; i += kDecThreads) kic[i] = kidx_new[i];
   }
   __syncthreads();
 
@@ -435,7 +439,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     if (tid == 0 && i + NS < nsub) issue(i + NS);
   }
   // the new token's score, from the argument row (its cache row may be stale)
-  if (t >= k0 && t < k1 && warp == 0) {
+  if (!window && t >= k0 && t < k1 && warp == 0) {
     const float *wsm = qis + kMaxR * DI;
     float score = 0.f;
     for (int r = 0; r < R; ++r) {
@@ -451,7 +455,11 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
 
   // ---------------------------------------------------------------- top-M
   int *sel0 = cluster.map_shared_rank(sel, 0);
-  if (n > M) {
+  if (window) {
+    // the M (= W) most recent positions t-M+1 .. t, or the whole prefix
+    if (rank == 0)
+      for (int j = tid; j < M; j += kDecThreads) sel[j] = n <= M ? (j < n ? j : -1) : t - M + 1 + j;
+  } else if (n > M) {
     constexpr int SEG = kCandCap / NC;                  // candidate slots of each rank in CTA 0
     uint32_t *fh = hist + 1024;                         // CTA 0: 1024-bin histogram of candidate keys
     uint32_t *segp = tot + 64;                          // CTA 0: exclusive prefix of the segment sizes

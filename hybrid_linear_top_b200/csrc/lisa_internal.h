@@ -52,6 +52,7 @@ struct DecodeParams {
   int *idx_out;
   // launch geometry (filled by the launcher)
   int split_req;                        // requested CTAs per (b, g): 0 (library's choice), 4, 8, 16
+  int window;                           // 1: sliding-window variant (M = the window W; no indexer inputs)
   int nc;                               // CTAs per cluster
   int stages;                           // TMA ring stages
   int stage_keys;                       // keys per ring stage
@@ -99,5 +100,7 @@ cudaError_t launch_prefill_linear_tc(const RowsParams &p, cudaStream_t st);
 cudaError_t launch_lin_prefix(const RowsParams &p, cudaStream_t st, int chunk);
 cudaError_t launch_lin_state(const RowsParams &p, cudaStream_t st);
 cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st);
+// Sliding-window variant: idx of every row = its M most recent positions.
+cudaError_t launch_window_idx(const RowsParams &p, cudaStream_t st);
 
 }  // namespace lisa

@@ -40,7 +40,27 @@ __global__ void append_kernel(RowsParams p) {
     kd[i] = ks[i];
     vd[i] = vs[i];
   }
-  for (int i = threadIdx.x; i < ndi; i += blockDim.x) kid[i] = kis[i];
+  if (p.kidx)
+    for (int i = threadIdx.x; i < ndi; i += blockDim.x) kid[i] = kis[i];
+}
+
+// ============================================================ sliding window
+// grid (T, B*Hkv): idx of row tau = the M most recent positions t-M+1 .. t of
+// t = pos[b] + tau (the whole prefix, -1 padded, while t < M).
+__global__ void window_idx_kernel(RowsParams p) {
+  const int tau = blockIdx.x, bg = blockIdx.y;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  if (!rows_pos_ok(p, b)) return;
+  const int t = p.pos[b] + tau, n = t + 1, M = p.M;
+  int *out = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * M;
+  for (int j = threadIdx.x; j < M; j += blockDim.x) out[j] = n <= M ? (j < n ? j : -1) : t - M + 1 + j;
+}
+
+cudaError_t launch_window_idx(const RowsParams &p, cudaStream_t st) {
+  cudaError_t e = prepare_kernel(window_idx_kernel);
+  if (e != cudaSuccess) return e;
+  window_idx_kernel<<<dim3(p.T, p.B * p.Hkv), 128, 0, st>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_append(const RowsParams &p, int dtype, cudaStream_t st) {

@@ -28,6 +28,7 @@ LISA_DEVERR_CHECK = 4
 LISA_OP_DECODE = 0
 LISA_OP_PREFILL = 1
 LISA_OP_INDEXER_TOPK = 2
+LISA_OP_PREFILL_WINDOW = 3
 
 EXPORTED = [
     "lisa_workspace_bytes",
@@ -36,6 +37,8 @@ EXPORTED = [
     "lisa_indexer_topk_noalloc",
     "lisa_decode_step",
     "lisa_prefill",
+    "lisa_decode_step_window",
+    "lisa_prefill_window",
     "lisa_status_str",
     "lisa_last_error_msg",
     "lisa_version",
@@ -77,6 +80,10 @@ def _load():
     lib.lisa_decode_step.restype = ctypes.c_int
     lib.lisa_prefill.argtypes = [L, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.lisa_prefill.restype = ctypes.c_int
+    lib.lisa_decode_step_window.argtypes = [L, P, P, P, P, P, ctypes.c_int, P, P, P]
+    lib.lisa_decode_step_window.restype = ctypes.c_int
+    lib.lisa_prefill_window.argtypes = [L, ctypes.c_int, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.lisa_prefill_window.restype = ctypes.c_int
     lib.lisa_status_str.argtypes = [ctypes.c_int]
     lib.lisa_status_str.restype = ctypes.c_char_p
     lib.lisa_last_error_msg.argtypes = []
@@ -203,6 +210,19 @@ def lisa_decode_step(layer, q, k, v, kidx, qidx, w, gate_logit, fuse_append, out
                                  _ptr(gate_logit), int(bool(fuse_append)), _ptr(out), _ptr(idx_out),
                                  _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                  _stream(stream)))
+
+
+def lisa_decode_step_window(layer, q, k, v, kidx, gate_logit, fuse_append, out, idx_out, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_decode_step_window(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(kidx), _ptr(gate_logit),
+                                        int(bool(fuse_append)), _ptr(out), _ptr(idx_out), _stream(stream)))
+
+
+def lisa_prefill_window(layer, T, q, k, v, kidx, gate_logit, out, idx_out, workspace, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_prefill_window(ctypes.byref(c), int(T), _ptr(q), _ptr(k), _ptr(v), _ptr(kidx),
+                                    _ptr(gate_logit), _ptr(out), _ptr(idx_out), _ptr(workspace),
+                                    workspace.numel() if workspace is not None else 0, _stream(stream)))
 
 
 def lisa_prefill(layer, T, q, k, v, kidx, qidx, w, gate_logit, out, idx_out, workspace, stream=None):

@@ -77,6 +77,7 @@ typedef enum { LISA_BF16 = 0, LISA_FP32 = 1 } lisa_dtype;
 #define LISA_OP_DECODE       0
 #define LISA_OP_PREFILL      1
 #define LISA_OP_INDEXER_TOPK 2
+#define LISA_OP_PREFILL_WINDOW 3
 
 /* One attention layer: geometry plus the caller-owned per-layer buffers. */
 typedef struct {
@@ -172,6 +173,27 @@ LISA_API lisa_status lisa_prefill(const lisa_layer *layer, int T, const void *q,
                          const void *v, const void *kidx, const void *qidx, const float *w,
                          const float *gate_logit, void *out, int *idx_out, void *workspace,
                          size_t ws_bytes, void *stream);
+
+/*
+ * Stage-1 inference variant: sliding window (arXiv 2607.19358, English
+ * abstract on arxivdaily.com: Stage 1 pairs the linear attention with a
+ * sliding-window attention, which Stage 2 replaces by the Lightning Indexer;
+ * iitog.ru article, key facts).  The sparse branch attends to the M most
+ * recent positions max(0, t-M+1) .. t (the layer's M is the window); the
+ * linear branch, the gate and every other definition are those of
+ * lisa_decode_step / lisa_prefill.  No indexer inputs: kidx may be NULL (the
+ * indexer-key cache row is then not written); qidx and w are not taken.
+ * idx_out, when given, receives the window's positions ([B, Hkv, M] for the
+ * step, [B, T, Hkv, M] for the prefill; ascending, -1 padded).  The decode
+ * step needs no workspace; the prefill needs
+ * lisa_workspace_bytes(layer, T, LISA_OP_PREFILL_WINDOW).
+ */
+LISA_API lisa_status lisa_decode_step_window(const lisa_layer *layer, const void *q, const void *k, const void *v,
+                                             const void *kidx, const float *gate_logit, int fuse_append,
+                                             void *out, int *idx_out, void *stream);
+LISA_API lisa_status lisa_prefill_window(const lisa_layer *layer, int T, const void *q, const void *k,
+                                         const void *v, const void *kidx, const float *gate_logit, void *out,
+                                         int *idx_out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * lisa_indexer_topk without a workspace argument, for callers that cannot
