@@ -256,12 +256,12 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   const int nsub = window ? 0 : (cnt + SUB - 1) / SUB;
 
   // ---------------------------------------------------------------- TMA ring
-  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS, and sub-chunk i + NS -> L2
+  auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS; two ring lengths ahead -> L2
     const int s_lo = k0 + i * SUB;
     const int s_hi = min(k1, s_lo + SUB);
     const int ncopy = max(0, min(s_hi, t) - s_lo);   // row t comes from the argument
-    {
-      const int p_lo = s_lo + NS * SUB;
+    for (int ahead = (i < NS ? 1 : 2); ahead <= 2; ++ahead) {   // sub-chunks i + NS and i + 2 NS
+      const int p_lo = s_lo + ahead * NS * SUB;
       const int np = max(0, min(min(k1, p_lo + SUB), t) - p_lo);
       if (np > 0) bulk_prefetch_l2(kidx_cache + (size_t)p_lo * DI, (uint32_t)(np * RB));
     }
