@@ -291,3 +291,14 @@ def test_decode_inputs_and_output_in_pinned_host_memory():
             check_set(idx_g[b, g], ref["scores"][b][g], cfg.M, int(pos[b]), where=f"b={b} g={g}")
     check_out(f64(out), ref["out"], cfg.dtype, where="out")
     check_state(f64(lay.state), ref["S"], where="state")
+
+
+@pytest.mark.parametrize("split", [0, 4])
+def test_decode_long_context_100k(split):
+    """100 000 cached tokens: per-CTA key slices of 6-25K keys, candidate
+    segments and the exact select at a long context."""
+    cfg = _replace(get_config("decode_1p5b_16k"), B=1, L=100000)
+    rng = make_rng(29, 0)
+    lay = gen_layer(cfg, rng, 99999)
+    step = gen_step(cfg, rng, 1)
+    run_decode(cfg, lay, step, np.array([99999]), 100000, split=split)
