@@ -14,7 +14,6 @@ constexpr int kMaxR = 8;        // indexer heads per KV head
 constexpr int kMaxG = 16;       // query heads per KV head
 constexpr int kAttnRows = 32;   // selected rows per attention CTA / tile
 constexpr int kLinChunk = 64;   // chunk length of the chunked linear attention
-constexpr int kRowTile = 64;    // query rows per indexer score tile (row path)
 
 // Raises the dynamic shared-memory limit of kernel `fn` to `dyn_smem` (once per
 // device and size; host-side bookkeeping only).

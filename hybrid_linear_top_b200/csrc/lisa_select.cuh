@@ -4,11 +4,17 @@
 // "top-M"): the first min(M, n) positions in the order (key descending,
 // position ascending), written in ascending position order, padded with -1.
 //
-// Method: MSB-first radix select over the 32-bit key in four 8-bit digits
-// finds the key K* of the M-th entry and how many entries equal to K* are
-// still needed; one ordered ballot/popc pass then emits the positions.  After
-// the first digit only the keys of the threshold bucket are revisited (they are
-// copied to a small shared-memory list when they fit).
+// Two methods:
+//  * block_topm_bounded (long rows): every thread keeps its 4 largest keys;
+//    the bin of the M-th largest of those values gives a bound lb with at
+//    least M keys >= lb; the keys >= lb are compacted in position order; the
+//    exact M-th key K* comes from 1024-bin range histograms (range_kth); an
+//    ordered compaction emits the positions.
+//  * block_topm (short rows, and rows where too many keys pass the bound):
+//    MSB-first radix select over the 32-bit key in four 8-bit digits finds K*
+//    and how many entries equal to K* are still needed; one ordered
+//    ballot/popc pass then emits the positions.  After the first digit only
+//    the keys of the threshold bucket are revisited.
 #pragma once
 
 #include "lisa_common.cuh"
