@@ -17,6 +17,7 @@ from .lisa_ref import (
     gate_fuse,
     decode_step,
     prefill,
+    indexer_kl,
 )
 
 __all__ = [
@@ -31,4 +32,5 @@ __all__ = [
     "gate_fuse",
     "decode_step",
     "prefill",
+    "indexer_kl",
 ]

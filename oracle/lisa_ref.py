@@ -251,3 +251,45 @@ def prefill(q, k, v, qidx, kidx, w, lam, S0, M, rows=None, sel_override=None):
                 o_lin = linear_readout(q[b, t, h], S[b, h])
                 out[b, t, h] = gate_fuse(lam[b, t, h], o_sp, o_lin)
     return dict(out=out, idx=idx, S=S, scores=scores)
+
+
+# --------------------------------------------------------------------------
+# Stage-2 indexer objective (forward): per-head KL      [abs]
+# --------------------------------------------------------------------------
+def indexer_kl(q, k, qidx, kidx, w, rows=None):
+    """Per-head KL divergence between the frozen attention of each query
+    head and the indexer's distribution over the causal prefix (arxivdaily.com
+    English abstract: in Stage 2 the Indexer is trained with a per-head KL
+    divergence that aligns its selection with the teacher's attention
+    pattern).  Reading fixed here: for token t and query head h of KV head
+    g = h // G,
+        p_t,h(s) = softmax_{s <= t}(q[t,h] . k[s,g] / sqrt(d))      (teacher)
+        r_t,g(s) = softmax_{s <= t}(I_g(t, s))                      (indexer)
+        KL[t, h] = sum_s p_t,h(s) * (log p_t,h(s) - log r_t,g(s)).
+    Tokens t = 0..T-1 of a sequence that starts at position 0.
+
+    q [B,T,Hq,d]; k [B,T,Hkv,d]; qidx [B,T,HI,dI]; kidx [B,T,Hkv,dI]; w [B,T,HI].
+    rows: optional token indices to evaluate (default all).
+    Returns kl [B, T, Hq] (rows not requested stay 0).
+
+    Parity: pinned by KL = 0 at t = 0, KL(p || uniform) = log(t+1) - H(p)
+    when w = 0, and scipy's rel_entr on small inputs."""
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    kl = np.zeros((B, T, Hq))
+    rows = range(T) if rows is None else rows
+    for b in range(B):
+        KIb = np.transpose(kidx[b], (1, 0, 2))                  # [Hkv, T, dI]
+        for t in rows:
+            sc = indexer_scores(qidx[b, t], w[b, t], KIb[:, : t + 1, :])   # [Hkv, t+1]
+            for h in range(Hq):
+                g = h // G
+                a = (k[b, : t + 1, g, :] @ q[b, t, h]) / np.sqrt(d)
+                pa = np.exp(a - a.max())
+                pa /= pa.sum()
+                c = sc[g]
+                lr = c - c.max() - np.log(np.exp(c - c.max()).sum())     # log r
+                la = np.log(np.maximum(pa, 1e-300))
+                kl[b, t, h] = float(np.sum(pa * (la - lr)))
+    return kl

@@ -287,3 +287,45 @@ def test_window_decode_with_full_window_is_causal_attention():
     p = np.exp(logits - logits.max())
     p /= p.sum()
     np.testing.assert_allclose(o, sum(p[s] * V[s] for s in range(t + 1)), rtol=1e-12, atol=1e-12)
+
+
+def _kl_inputs(seed, T=12, Hq=4, Hkv=2, d=8, HI=4, dI=4):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((1, T, Hq, d)), rng.standard_normal((1, T, Hkv, d)),
+            rng.standard_normal((1, T, HI, dI)), rng.standard_normal((1, T, Hkv, dI)),
+            rng.random((1, T, HI)))
+
+
+def test_indexer_kl_matches_rel_entr():
+    """Against scipy's elementwise relative entropy on the two distributions
+    built from the definitions (softmax of scaled dot products; softmax of
+    the indexer scores)."""
+    from scipy.special import rel_entr, softmax
+    q, k, qi, ki, w = _kl_inputs(1)
+    kl = oracle.indexer_kl(q, k, qi, ki, w)
+    T, Hq, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    for t in range(T):
+        sc = oracle.indexer_scores(qi[0, t], w[0, t], np.transpose(ki[0, : t + 1], (1, 0, 2)))
+        for h in range(Hq):
+            p = softmax(np.array([q[0, t, h] @ k[0, s, h // G] for s in range(t + 1)]) / math.sqrt(d))
+            r = softmax(sc[h // G])
+            assert kl[0, t, h] == pytest.approx(float(np.sum(rel_entr(p, r))), rel=1e-9, abs=1e-12)
+    assert np.all(kl >= -1e-12)
+
+
+def test_indexer_kl_first_token_is_zero_and_uniform_student():
+    """t = 0: both distributions are the single token, KL = 0.  w = 0: the
+    indexer is uniform over the prefix, KL = log(t+1) - H(teacher)."""
+    q, k, qi, ki, w = _kl_inputs(2)
+    kl = oracle.indexer_kl(q, k, qi, ki, np.zeros_like(w))
+    assert np.allclose(kl[:, 0], 0.0, atol=1e-12)
+    T, Hq, d = q.shape[1], q.shape[2], q.shape[3]
+    G = Hq // k.shape[2]
+    for t in range(1, T):
+        for h in range(Hq):
+            a = np.array([q[0, t, h] @ k[0, s, h // G] for s in range(t + 1)]) / math.sqrt(d)
+            e = np.exp(a - a.max())
+            p = e / e.sum()
+            entropy = -float(np.sum(p * np.log(p)))
+            assert kl[0, t, h] == pytest.approx(math.log(t + 1) - entropy, rel=1e-9, abs=1e-12)
