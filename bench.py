@@ -550,6 +550,47 @@ def _line(rank, metric, value, unit, args, world, ms_per_step, config, roofline,
     print(json.dumps(line), flush=True)
 
 
+def run_kl(args, rank, world):
+    """Stage-2 objective forward (lisa_indexer_kl) over a 16384-token prefix at
+    the 1.5B shape: per-head KL of the teacher's attention against the
+    indexer's distribution for every token and query head."""
+    import torch
+    from hybrid_linear_top_b200 import lisa as L
+    cfg = get_config("prefill_1p5b_16k")
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 * rank + 7)
+    lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.T, L.LISA_BF16)
+    _fill_layer(L, lay, cfg, cfg.T, g, torch)
+    bf = torch.bfloat16
+    q = (torch.randn((cfg.B, cfg.T, cfg.Hq, cfg.d), generator=g, device="cuda") / cfg.d ** 0.5).to(bf)
+    qidx = (torch.randn((cfg.B, cfg.T, cfg.HI, cfg.dI), generator=g, device="cuda") / cfg.dI ** 0.5).to(bf)
+    w = torch.rand((cfg.B, cfg.T, cfg.HI), generator=g, device="cuda")
+    kl = torch.empty(cfg.B, cfg.T, cfg.Hq, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            L.lisa_indexer_kl(lay, cfg.T, q, qidx, w, kl, stream)
+    gr = _capture(torch, stream, [stream], list(range(args.steps)),
+                  lambda i, s_: L.lisa_indexer_kl(lay, cfg.T, q, qidx, w, kl, s_))
+    ms = max_over_ranks(_timed_replays(torch, stream, [gr]), world, "cuda") / args.steps
+    if int(lay.err_word.item()) or not torch.isfinite(kl).all():
+        raise RuntimeError("the KL objective flagged an error")
+    pairs = cfg.T * (cfg.T + 1) // 2
+    flops = cfg.B * (cfg.Hq * pairs * 2 * cfg.d + cfg.HI * pairs * 2 * cfg.dI)
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    _line(rank, "LISA Stage-2 KL objective (forward) tokens/s @16K prefix", replica_rate(cfg.T * cfg.B, ms, world),
+          "tokens/s", args, world, ms,
+          {"workload": "kl_1p5b_16k", "B": cfg.B, "T": cfg.T, "Hq": cfg.Hq, "HI": cfg.HI,
+           "parallelism": f"replicas x{world}"},
+          {"bound": "tensor", "kernel": "indexer_kl_kernel (warp MMAs)", "achieved": tf, "peak": peak,
+           "unit": "TFLOP/s", "frac": tf / peak, "peak_kind": "measured" if peaks else "fallback",
+           "algorithmic_flops_per_call": flops, "traffic": None})
+
+
 def run_window(args, rank, world):
     """Stage-1 sliding-window variant at the 1.5B decode shape: the last 256
     positions instead of the indexer's top-256 (lisa_decode_step_window),
@@ -710,7 +751,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l", "window_1p5b_16k"])
+                    choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l", "window_1p5b_16k", "kl_1p5b_16k"])
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--streams", type=int, default=32)
     ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16])
@@ -720,7 +761,7 @@ def main():
     args.warmup = max(3, args.warmup)
     if args.steps is None:
         args.steps = {WORKLOAD: 200000, "prefill_1p5b_16k": 20, "ragged_7b_b32": 2000,
-                      "longcot_7b_28l": 1024, "window_1p5b_16k": 200000}[args.workload]
+                      "longcot_7b_28l": 1024, "window_1p5b_16k": 200000, "kl_1p5b_16k": 5}[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if world > 1:
@@ -740,6 +781,8 @@ def main():
             run_longcot(args, rank, world)
         elif args.workload == "window_1p5b_16k":
             run_window(args, rank, world)
+        elif args.workload == "kl_1p5b_16k":
+            run_kl(args, rank, world)
         else:
             run_lisa(args, rank, world)
     finally:

@@ -396,6 +396,26 @@ lisa_status lisa_prefill(const lisa_layer *L, int T, const void *q, const void *
   return ok();
 }
 
+lisa_status lisa_indexer_kl(const lisa_layer *L, int T, const void *q, const void *qidx, const float *w, float *kl_out,
+                            void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if (L->dtype != LISA_BF16) return fail(LISA_ERR_UNSUPPORTED, "lisa_indexer_kl supports bf16 storage only");
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) ||
+      (s = check_ptr(kl_out, "kl_out")))
+    return s;
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.q = q; r.qidx = qidx; r.w = w;
+  cudaError_t e = lisa::launch_indexer_kl(r, kl_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer_kl");
+  return ok();
+}
+
 lisa_status lisa_indexer_topk_noalloc(const lisa_layer *L, const void *qidx, const float *w, int T, int *idx_out,
                                       void *stream) {
   lisa_status s;

@@ -99,6 +99,8 @@ cudaError_t launch_prefill_linear_tc(const RowsParams &p, cudaStream_t st);
 cudaError_t launch_lin_prefix(const RowsParams &p, cudaStream_t st, int chunk);
 cudaError_t launch_lin_state(const RowsParams &p, cudaStream_t st);
 cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st);
+// Stage-2 objective (forward): per-head KL of teacher attention vs indexer, kl_out [B, T, Hq].
+cudaError_t launch_indexer_kl(const RowsParams &p, float *kl_out, cudaStream_t st);
 // Sliding-window variant: idx of every row = its M most recent positions.
 cudaError_t launch_window_idx(const RowsParams &p, cudaStream_t st);
 

@@ -39,6 +39,7 @@ EXPORTED = [
     "lisa_prefill",
     "lisa_decode_step_window",
     "lisa_prefill_window",
+    "lisa_indexer_kl",
     "lisa_status_str",
     "lisa_last_error_msg",
     "lisa_version",
@@ -84,6 +85,8 @@ def _load():
     lib.lisa_decode_step_window.restype = ctypes.c_int
     lib.lisa_prefill_window.argtypes = [L, ctypes.c_int, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.lisa_prefill_window.restype = ctypes.c_int
+    lib.lisa_indexer_kl.argtypes = [L, ctypes.c_int, P, P, P, P, P]
+    lib.lisa_indexer_kl.restype = ctypes.c_int
     lib.lisa_status_str.argtypes = [ctypes.c_int]
     lib.lisa_status_str.restype = ctypes.c_char_p
     lib.lisa_last_error_msg.argtypes = []
@@ -223,6 +226,12 @@ def lisa_prefill_window(layer, T, q, k, v, kidx, gate_logit, out, idx_out, works
     _check(_lib.lisa_prefill_window(ctypes.byref(c), int(T), _ptr(q), _ptr(k), _ptr(v), _ptr(kidx),
                                     _ptr(gate_logit), _ptr(out), _ptr(idx_out), _ptr(workspace),
                                     workspace.numel() if workspace is not None else 0, _stream(stream)))
+
+
+def lisa_indexer_kl(layer, T, q, qidx, w, kl_out, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_indexer_kl(ctypes.byref(c), int(T), _ptr(q), _ptr(qidx), _ptr(w), _ptr(kl_out),
+                                _stream(stream)))
 
 
 def lisa_prefill(layer, T, q, k, v, kidx, qidx, w, gate_logit, out, idx_out, workspace, stream=None):

@@ -175,6 +175,23 @@ LISA_API lisa_status lisa_prefill(const lisa_layer *layer, int T, const void *q,
                          size_t ws_bytes, void *stream);
 
 /*
+ * Stage-2 indexer objective, forward (arXiv 2607.19358, English abstract on
+ * arxivdaily.com: the Indexer is trained with a per-head KL divergence that
+ * aligns its selection with the frozen teacher's attention pattern).  For the
+ * T tokens per sequence at positions t = pos[b] + tau and every query head h
+ * (KV head g = h / G):
+ *   p(s) = softmax over s <= t of q[b,tau,h] . k_cache[b,g,s] / sqrt(d)
+ *   r(s) = softmax over s <= t of I_g(t, s)   (the indexer score defined above)
+ *   kl_out[b, tau, h] = sum_s p(s) * (log p(s) - log r(s))      (fp32, >= 0)
+ * The caches must already hold rows 0 .. pos[b]+T-1 (for example after
+ * lisa_prefill or lisa_append_cache).  q [B, T, Hq, d]; qidx [B, T, HI, dI]
+ * (bf16 storage only; LISA_ERR_UNSUPPORTED otherwise); w [B, T, HI] fp32;
+ * kl_out [B, T, Hq] fp32.  No workspace.
+ */
+LISA_API lisa_status lisa_indexer_kl(const lisa_layer *layer, int T, const void *q, const void *qidx,
+                                     const float *w, float *kl_out, void *stream);
+
+/*
  * Stage-1 inference variant: sliding window (arXiv 2607.19358, English
  * abstract on arxivdaily.com: Stage 1 pairs the linear attention with a
  * sliding-window attention, which Stage 2 replaces by the Lightning Indexer;
