@@ -23,6 +23,9 @@ The pages leave these points open; this library fixes them as definitions
     j = g*R + r of w[j] * max(0, qidx[j] . kidx[g, s]); no extra scale;
   * one top-M set per KV head, shared by its G = Hq/Hkv query heads
     (query head h belongs to KV head h // G);
+  * the other readings of the head mapping are variants behind keyword
+    arguments: one indexer key per indexer head, a single top-M set shared by
+    all KV heads, and linear-branch keys / values of their own per query head;
   * order: higher score first, equal scores -> lower position first;
     a prefix with <= M tokens is selected whole; the current token is a
     candidate (causal prefix s <= t);
@@ -42,23 +45,34 @@ import numpy as np
 # --------------------------------------------------------------------------
 # step 1: Lightning Indexer score      [abs], [meth]
 # --------------------------------------------------------------------------
-def indexer_scores(qidx_t: np.ndarray, w_t: np.ndarray, kidx_keys: np.ndarray) -> np.ndarray:
+def indexer_scores(qidx_t: np.ndarray, w_t: np.ndarray, kidx_keys: np.ndarray, groups=None) -> np.ndarray:
     """Scores of every candidate key for one query token.
 
     qidx_t    [HI, dI]      indexer queries of the token
     w_t       [HI]          indexer head weights of the token
-    kidx_keys [Hkv, n, dI]  indexer keys of the candidate positions 0..n-1
-    returns   [Hkv, n]      I_g(s) = sum_r w[gR+r] * max(0, qidx[gR+r] . kidx[g, s])
+    kidx_keys [P, n, dI]    indexer keys of the candidate positions 0..n-1
+    groups    selection groups Gs (default P): the HI heads are split into Gs
+              groups of R = HI / Gs consecutive heads, one score row per group
+    returns   [Gs, n]       I_gs(s) = sum_r w[j] * max(0, qidx[j] . key_j[s]),
+                            j = gs*R + r
+
+    key_j is plane gs when P == Gs (one indexer key per group: per KV head in
+    the default reading, a single key per token for a shared selection) and
+    plane j when P == HI (one indexer key per indexer head, the other reading
+    of the head mapping the pages leave open).
     """
     HI = qidx_t.shape[0]
-    Hkv, n, _ = kidx_keys.shape
-    R = HI // Hkv
-    out = np.zeros((Hkv, n), dtype=np.float64)
-    for g in range(Hkv):
+    P, n, _ = kidx_keys.shape
+    Gs = P if groups is None else int(groups)
+    R = HI // Gs
+    assert Gs * R == HI and P in (Gs, HI), "key planes must be one per group or one per indexer head"
+    out = np.zeros((Gs, n), dtype=np.float64)
+    for gs in range(Gs):
         for r in range(R):
-            j = g * R + r
-            dots = kidx_keys[g] @ qidx_t[j]
-            out[g] += w_t[j] * np.maximum(dots, 0.0)
+            j = gs * R + r
+            plane = gs if P == Gs else j
+            dots = kidx_keys[plane] @ qidx_t[j]
+            out[gs] += w_t[j] * np.maximum(dots, 0.0)
     return out
 
 
@@ -157,25 +171,33 @@ def gate_fuse(lam: float, o_sp: np.ndarray, o_lin: np.ndarray) -> np.ndarray:
 # whole layer: one decode step
 # --------------------------------------------------------------------------
 def decode_step(q, k, v, qidx, kidx, w, lam, k_cache, v_cache, kidx_cache, S, pos, M,
-                sel_override=None):
+                sel_override=None, shared_set=False, k_lin=None, v_lin=None):
     """One decode step for a batch.
 
-    q [B,Hq,d]; k, v [B,Hkv,d]; qidx [B,HI,dI]; kidx [B,Hkv,dI]; w [B,HI];
-    lam [B,Hq]; caches [B,Hkv,>=pos[b],*] hold rows 0..pos[b]-1; S [B,Hq,d,d];
-    pos [B] = position t of the new token.
-    sel_override: optional [B,Hkv,M] index sets to use for the sparse branch
+    q [B,Hq,d]; k, v [B,Hkv,d]; qidx [B,HI,dI]; kidx [B,P,dI]; w [B,HI];
+    lam [B,Hq]; caches [B,Hkv|P,>=pos[b],*] hold rows 0..pos[b]-1; S [B,Hq,d,d];
+    pos [B] = position t of the new token.  P (indexer key planes) is Hkv by
+    default, HI for one indexer key per indexer head, and 1 (or HI) with
+    shared_set.
+    sel_override: optional [B,Gs,M] index sets to use for the sparse branch
     instead of the oracle's own (the "conditional oracle").
+    shared_set: one top-M set for every KV head, scored over all HI indexer
+    heads (Gs = 1 selection group instead of Gs = Hkv).
+    k_lin, v_lin: optional [B,Hq,d] keys / values of the linear branch, one
+    per query head; by default the branch uses the attention's k, v of the
+    head's KV group.
 
-    Returns dict: out [B,Hq,d], idx [B,Hkv,M], S [B,Hq,d,d],
-    scores list (per b) of [Hkv, t+1] arrays, o_sp, o_lin [B,Hq,d].
+    Returns dict: out [B,Hq,d], idx [B,Gs,M], S [B,Hq,d,d],
+    scores list (per b) of [Gs, t+1] arrays, o_sp, o_lin [B,Hq,d].
     """
     B, Hq, d = q.shape
     Hkv = k.shape[1]
     G = Hq // Hkv
+    Gs = 1 if shared_set else Hkv
     out = np.zeros((B, Hq, d))
     o_sp_all = np.zeros((B, Hq, d))
     o_lin_all = np.zeros((B, Hq, d))
-    idx = np.full((B, Hkv, M), -1, dtype=np.int64)
+    idx = np.full((B, Gs, M), -1, dtype=np.int64)
     S_new = np.array(S, dtype=np.float64, copy=True)
     scores_all = []
     for b in range(B):
@@ -183,17 +205,20 @@ def decode_step(q, k, v, qidx, kidx, w, lam, k_cache, v_cache, kidx_cache, S, po
         # candidate keys 0..t: cached rows then the new token
         K = np.concatenate([k_cache[b, :, :t, :], k[b][:, None, :]], axis=1)          # [Hkv, t+1, d]
         V = np.concatenate([v_cache[b, :, :t, :], v[b][:, None, :]], axis=1)
-        KI = np.concatenate([kidx_cache[b, :, :t, :], kidx[b][:, None, :]], axis=1)   # [Hkv, t+1, dI]
-        sc = indexer_scores(qidx[b], w[b], KI)
+        KI = np.concatenate([kidx_cache[b, :, :t, :], kidx[b][:, None, :]], axis=1)   # [P, t+1, dI]
+        sc = indexer_scores(qidx[b], w[b], KI, groups=Gs)
         scores_all.append(sc)
-        for g in range(Hkv):
-            idx[b, g] = topm_select(sc[g], M)
+        for gs in range(Gs):
+            idx[b, gs] = topm_select(sc[gs], M)
         use = idx[b] if sel_override is None else np.asarray(sel_override[b])
         for h in range(Hq):
             g = h // G
-            sel = use[g][use[g] >= 0]
+            gs = 0 if shared_set else g
+            sel = use[gs][use[gs] >= 0]
             o_sp = sparse_attention(q[b, h], K[g, sel], V[g, sel])
-            S_new[b, h] = linear_update(S_new[b, h], k[b, g], v[b, g])
+            kl_h = k[b, g] if k_lin is None else k_lin[b, h]
+            vl_h = v[b, g] if v_lin is None else v_lin[b, h]
+            S_new[b, h] = linear_update(S_new[b, h], kl_h, vl_h)
             o_lin = linear_readout(q[b, h], S_new[b, h])
             o_sp_all[b, h] = o_sp
             o_lin_all[b, h] = o_lin
@@ -204,49 +229,55 @@ def decode_step(q, k, v, qidx, kidx, w, lam, k_cache, v_cache, kidx_cache, S, po
 # --------------------------------------------------------------------------
 # whole layer: causal prefill of T tokens
 # --------------------------------------------------------------------------
-def prefill(q, k, v, qidx, kidx, w, lam, S0, M, rows=None, sel_override=None):
+def prefill(q, k, v, qidx, kidx, w, lam, S0, M, rows=None, sel_override=None, shared_set=False,
+            k_lin=None, v_lin=None):
     """Causal prefill of T tokens starting from an empty cache.
 
-    q [B,T,Hq,d]; k, v [B,T,Hkv,d]; qidx [B,T,HI,dI]; kidx [B,T,Hkv,dI];
-    w [B,T,HI]; lam [B,T,Hq]; S0 [B,Hq,d,d].
+    q [B,T,Hq,d]; k, v [B,T,Hkv,d]; qidx [B,T,HI,dI]; kidx [B,T,P,dI]
+    (P as in decode_step); w [B,T,HI]; lam [B,T,Hq]; S0 [B,Hq,d,d].
     rows: optional iterable of token indices t whose outputs are wanted (the
     state always runs over all T tokens); default all.
-    sel_override: optional callable (b, t) -> [Hkv, M] index sets for the
+    sel_override: optional callable (b, t) -> [Gs, M] index sets for the
     sparse branch (the "conditional oracle"), or None.
+    shared_set, k_lin, v_lin ([B,T,Hq,d]): the variants of decode_step.
 
-    Returns dict: out [B,T,Hq,d] (rows not requested stay 0), idx [B,T,Hkv,M]
+    Returns dict: out [B,T,Hq,d] (rows not requested stay 0), idx [B,T,Gs,M]
     (-1 for rows not requested), S [B,Hq,d,d] = state after token T-1,
-    scores {(b, t): [Hkv, t+1]} for the requested rows.
+    scores {(b, t): [Gs, t+1]} for the requested rows.
     """
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
+    Gs = 1 if shared_set else Hkv
     want = np.zeros(T, dtype=bool)
     if rows is None:
         want[:] = True
     else:
         want[np.asarray(list(rows), dtype=np.int64)] = True
     out = np.zeros((B, T, Hq, d))
-    idx = np.full((B, T, Hkv, M), -1, dtype=np.int64)
+    idx = np.full((B, T, Gs, M), -1, dtype=np.int64)
     S = np.array(S0, dtype=np.float64, copy=True)
     scores = {}
     for b in range(B):
         Kb = np.transpose(k[b], (1, 0, 2))        # [Hkv, T, d]
         Vb = np.transpose(v[b], (1, 0, 2))
-        KIb = np.transpose(kidx[b], (1, 0, 2))    # [Hkv, T, dI]
+        KIb = np.transpose(kidx[b], (1, 0, 2))    # [P, T, dI]
         for t in range(T):
             for h in range(Hq):
-                S[b, h] = linear_update(S[b, h], k[b, t, h // G], v[b, t, h // G])
+                kl_h = k[b, t, h // G] if k_lin is None else k_lin[b, t, h]
+                vl_h = v[b, t, h // G] if v_lin is None else v_lin[b, t, h]
+                S[b, h] = linear_update(S[b, h], kl_h, vl_h)
             if not want[t]:
                 continue
-            sc = indexer_scores(qidx[b, t], w[b, t], KIb[:, : t + 1, :])
+            sc = indexer_scores(qidx[b, t], w[b, t], KIb[:, : t + 1, :], groups=Gs)
             scores[(b, t)] = sc
-            for g in range(Hkv):
-                idx[b, t, g] = topm_select(sc[g], M)
+            for gs in range(Gs):
+                idx[b, t, gs] = topm_select(sc[gs], M)
             use = idx[b, t] if sel_override is None else np.asarray(sel_override(b, t))
             for h in range(Hq):
                 g = h // G
-                sel = use[g][use[g] >= 0]
+                gs = 0 if shared_set else g
+                sel = use[gs][use[gs] >= 0]
                 o_sp = sparse_attention(q[b, t, h], Kb[g, sel], Vb[g, sel])
                 o_lin = linear_readout(q[b, t, h], S[b, h])
                 out[b, t, h] = gate_fuse(lam[b, t, h], o_sp, o_lin)
