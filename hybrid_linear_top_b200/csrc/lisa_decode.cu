@@ -55,7 +55,7 @@ struct ScoreGeom {
 
 struct DecLayout {
   int region0, cand_key, cand_pos, pin;
-  int keys, hist, tot, misc, sel, qs, qi, ks, vs, part, pml, olin, logit, sidx, bars, total;
+  int keys, hist, tot, misc, sel, qs, qi, ks, vs, kis, gl, part, pml, olin, logit, sidx, bars, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
@@ -90,6 +90,8 @@ __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, i
   L.qi = off; off += align16(kMaxR * DI * 4 + kMaxR * 4);
   L.ks = off; off += align16(D * 4);
   L.vs = off; off += align16(D * 4);
+  L.kis = off; off += align16(DI * 4);
+  L.gl = off; off += align16(G * 4);
   L.part = off; off += align16(G * D * 4);
   L.pml = off; off += align16(2 * G * 4);
   L.olin = off; off += align16(G * (D / NC) * 4);
@@ -176,6 +178,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   float *qis = reinterpret_cast<float *>(smem + lay.qi);   // [R][DI] indexer queries, then [R] weights
   float *ks = reinterpret_cast<float *>(smem + lay.ks);
   float *vs = reinterpret_cast<float *>(smem + lay.vs);
+  float *kis = reinterpret_cast<float *>(smem + lay.kis);   // the new token's indexer key
+  float *gls = reinterpret_cast<float *>(smem + lay.gl);    // gate logits of the G heads
   float *part = reinterpret_cast<float *>(smem + lay.part);
   float *pml = reinterpret_cast<float *>(smem + lay.pml);
   float *olin = reinterpret_cast<float *>(smem + lay.olin);
@@ -190,13 +194,45 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   }
   // Everything read below may have been written by the previous kernel.
   grid_dep_wait();
-  grid_dep_launch();
 
   const int t = p.pos[b];                  // in flight while the loads below are issued
   const T *kidx_cache = reinterpret_cast<const T *>(p.kidx_cache) + (size_t)bg * p.L_max * DI;
   const T *kidx_new = reinterpret_cast<const T *>(p.kidx) + (size_t)bg * DI;
 
   // ---------------------------------------------------------------- early loads
+  const T *qin = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + g * G) * D;
+  const T *kin = reinterpret_cast<const T *>(p.k) + (size_t)bg * D;
+  const T *vin = reinterpret_cast<const T *>(p.v) + (size_t)bg * D;
+  const T *qidx_in = reinterpret_cast<const T *>(p.qidx) + ((size_t)b * p.HI + g * R) * DI;
+  const bool window = p.window != 0;      // sliding-window variant: no indexer, no top-M
+  // The step's own rows as 16-byte chunks, [q of the G heads | k | v |
+  // indexer queries of the R heads | new indexer key], loaded into registers
+  // with every load in flight at once (one DRAM round trip, not one per row),
+  // then widened into shared memory below.
+  const int o_k = G * D / VEC, o_v = o_k + D / VEC, o_qi = o_v + D / VEC;
+  const int o_ki = o_qi + (window ? 0 : R * DI / VEC);
+  const int n_in = o_ki + (p.kidx ? DI / VEC : 0);
+  auto chunk_src = [&](int c) -> const uint4 * {
+    if (c < o_k) return reinterpret_cast<const uint4 *>(qin) + c;
+    if (c < o_v) return reinterpret_cast<const uint4 *>(kin) + (c - o_k);
+    if (c < o_qi) return reinterpret_cast<const uint4 *>(vin) + (c - o_v);
+    if (c < o_ki) return reinterpret_cast<const uint4 *>(qidx_in) + (c - o_qi);
+    return reinterpret_cast<const uint4 *>(kidx_new) + (c - o_ki);
+  };
+  auto chunk_dst = [&](int c) -> float * {
+    if (c < o_k) return qs + c * VEC;
+    if (c < o_v) return ks + (c - o_k) * VEC;
+    if (c < o_qi) return vs + (c - o_v) * VEC;
+    if (c < o_ki) return qis + (c - o_qi) * VEC;
+    return kis + (c - o_ki) * VEC;
+  };
+  constexpr int kInRegs = 2;               // chunks per thread held in registers
+  uint4 inr[kInRegs];
+#pragma unroll
+  for (int j = 0; j < kInRegs; ++j)
+    if (tid + j * kDecThreads < n_in) inr[j] = *chunk_src(tid + j * kDecThreads);
+  const float w_in = (!window && tid < R) ? p.w[(size_t)b * p.HI + g * R + tid] : 0.f;
+  const float gl_in = tid < G ? p.gate[(size_t)b * p.Hq + g * G + tid] : 0.f;
   // state slab of the first (up to) HP query heads
   const int c0s = rank * COLS;
   const int cq = tid % QPR;                // same float4 column for every row this thread visits
@@ -215,35 +251,6 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   // heads beyond the first HP: their slab rows requested into L2 now
   for (int i = tid; i < (G - gA) * D; i += kDecThreads)
     prefetch_l2(p.state + ((size_t)b * p.Hq + g * G + gA + i / D) * D * D + (size_t)(i % D) * D + c0s);
-  const T *qin = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + g * G) * D;
-  for (int i = tid; i < G * D; i += kDecThreads) qs[i] = Dt<T>::to_f(qin[i]);
-  const T *kin = reinterpret_cast<const T *>(p.k) + (size_t)bg * D;
-  const T *vin = reinterpret_cast<const T *>(p.v) + (size_t)bg * D;
-  for (int i = tid; i < D; i += kDecThreads) {
-    ks[i] = Dt<T>::to_f(kin[i]);
-    vs[i] = Dt<T>::to_f(vin[i]);
-  }
-  const bool window = p.window != 0;      // sliding-window variant: no indexer, no top-M
-  if (!window) {
-    for (int i = tid; i < R * DI; i += kDecThreads)
-      qis[i] = Dt<T>::to_f(reinterpret_cast<const T *>(p.qidx)[((size_t)b * p.HI + g * R) * DI + i]);
-    if (tid < R) qis[kMaxR * DI + tid] = p.w[(size_t)b * p.HI + g * R + tid];
-  }
-  // MMA operand B (indexer queries, heads = columns, padded to 8) and the head weights of this lane
-  uint32_t bq[DI / 16][2];
-  float wq0 = 0.f, wq1 = 0.f;
-  if (SG::kMma && !window) {
-    const int nh = lane >> 2, kc = 2 * (lane & 3);
-    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(reinterpret_cast<const T *>(p.qidx) +
-                                                               ((size_t)b * p.HI + g * R + (nh < R ? nh : 0)) * DI);
-#pragma unroll
-    for (int s = 0; s < DI / 16; ++s) {
-      bq[s][0] = nh < R ? qrow[(s * 16 + kc) >> 1] : 0u;
-      bq[s][1] = nh < R ? qrow[(s * 16 + kc + 8) >> 1] : 0u;
-    }
-    if (kc < R) wq0 = p.w[(size_t)b * p.HI + g * R + kc];
-    if (kc + 1 < R) wq1 = p.w[(size_t)b * p.HI + g * R + kc + 1];
-  }
   if (t < 0 || t >= p.L_max) {  // same value in every CTA of the cluster: all leave together
     if (rank == 0 && tid == 0) set_err(p.err_word, LISA_DEVERR_POS);
     return;
@@ -281,20 +288,44 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   };
   if (tid == 0)
     for (int i = 0; i < min(NS, nsub); ++i) issue(i);
-  // append the new token (row t) from the CTA whose key slice holds it
-  if (p.fuse_append && t >= k0 && t < k1) {
-    const size_t row = (size_t)bg * p.L_max + t;
-    T *kc = reinterpret_cast<T *>(p.k_cache) + row * D;
-    T *vc = reinterpret_cast<T *>(p.v_cache) + row * D;
-    T *kic = reinterpret_cast<T *>(p.kidx_cache) + row * DI;
-    for (int i = tid; i < D; i += kDecThreads) {
-      kc[i] = kin[i];
-      vc[i] = vin[i];
-    }
-    if (p.kidx)
-      for (int i = tid; i < DI; i += kDecThreads) kic[i] = kidx_new[i];
+  // the step's rows into shared memory; the CTA whose key slice holds row t
+  // also appends the new token's k, v and indexer key to the caches
+  {
+    const bool app = p.fuse_append && t >= k0 && t < k1;
+    const size_t arow = (size_t)bg * p.L_max + t;
+    auto put = [&](int c, const uint4 &u) {
+      Vec16<T>::unpack(u, chunk_dst(c));
+      if (!app) return;
+      if (c >= o_k && c < o_v)
+        reinterpret_cast<uint4 *>(reinterpret_cast<T *>(p.k_cache) + arow * D)[c - o_k] = u;
+      else if (c >= o_v && c < o_qi)
+        reinterpret_cast<uint4 *>(reinterpret_cast<T *>(p.v_cache) + arow * D)[c - o_v] = u;
+      else if (c >= o_ki)
+        reinterpret_cast<uint4 *>(reinterpret_cast<T *>(p.kidx_cache) + arow * DI)[c - o_ki] = u;
+    };
+#pragma unroll
+    for (int j = 0; j < kInRegs; ++j)
+      if (tid + j * kDecThreads < n_in) put(tid + j * kDecThreads, inr[j]);
+    for (int c = tid + kInRegs * kDecThreads; c < n_in; c += kDecThreads) put(c, *chunk_src(c));
+    if (!window && tid < R) qis[kMaxR * DI + tid] = w_in;
+    if (tid < G) gls[tid] = gl_in;
   }
   __syncthreads();
+  // MMA operand B (indexer queries, heads = columns, padded to 8; the floats
+  // hold bf16 values, so re-packing is exact) and the head weights of this lane
+  uint32_t bq[DI / 16][2];
+  float wq0 = 0.f, wq1 = 0.f;
+  if (SG::kMma && !window) {
+    const int nh = lane >> 2, kc = 2 * (lane & 3);
+    const float *qr = qis + (nh < R ? nh : 0) * DI;
+#pragma unroll
+    for (int s = 0; s < DI / 16; ++s) {
+      bq[s][0] = nh < R ? pack_bf16(qr[s * 16 + kc], qr[s * 16 + kc + 1]) : 0u;
+      bq[s][1] = nh < R ? pack_bf16(qr[s * 16 + kc + 8], qr[s * 16 + kc + 9]) : 0u;
+    }
+    if (kc < R) wq0 = qis[kMaxR * DI + kc];
+    if (kc + 1 < R) wq1 = qis[kMaxR * DI + kc + 1];
+  }
 
   // ---------------------------------------------------------------- linear state
   // S_h <- S_h + k^T v on columns [c0s, c0s + COLS); o_lin[h][c] = sum_i q_h[i] S_h[i][c].
@@ -444,7 +475,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     float score = 0.f;
     for (int r = 0; r < R; ++r) {
       float dot = 0.f;
-      for (int c = lane; c < DI; c += 32) dot = fmaf(qis[r * DI + c], Dt<T>::to_f(kidx_new[c]), dot);
+      for (int c = lane; c < DI; c += 32) dot = fmaf(qis[r * DI + c], kis[c], dot);
       dot = warp_sum(dot);
       score = fmaf(wsm[r], fmaxf(dot, 0.f), score);
     }
@@ -841,6 +872,10 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   if (rank == 0 && p.idx_out)
     for (int j = tid; j < M; j += kDecThreads) p.idx_out[(size_t)bg * M + j] = sel[j];
 
+  // The next kernel on the stream may be scheduled from here on: its CTAs
+  // wait in their prologue, so a later trigger keeps them from holding SM
+  // slots through this kernel's key stream and selection.
+  grid_dep_launch();
   // ---------------------------------------------------------------- sparse attention (this CTA's rows)
   unsigned char *kvs = ring;                 // [rpc] K rows then [rpc] V rows, stride RS
   for (int r = tid; r < rpc; r += kDecThreads) {
@@ -1037,7 +1072,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       const int h = g * G + hh;
       const float o_sp = num / den;
       const float o_lin = olin[hh * COLS + c];
-      const float gam = 1.f / (1.f + expf(-p.gate[(size_t)b * p.Hq + h]));
+      const float gam = 1.f / (1.f + expf(-gls[hh]));
       reinterpret_cast<T *>(p.out)[((size_t)b * p.Hq + h) * D + d] = Dt<T>::from_f(gam * o_sp + (1.f - gam) * o_lin);
     }
   }
