@@ -46,7 +46,7 @@ WORKLOAD = "decode_1p5b_16k"
 # DRAM bytes (read + write) of one decode launch from an ncu capture of this
 # kernel on this workload, by CTA split (the ncu summary under profiles/);
 # None where no capture of the current kernel exists.
-DECODE_TRAFFIC = {4: 5378304, 8: None, 16: None, 0: None}
+DECODE_TRAFFIC = {4: None, 8: None, 16: None, 0: None}
 
 
 def algorithmic_bytes(cfg, L, esize=2):

@@ -263,6 +263,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   const int nsub = window ? 0 : (cnt + SUB - 1) / SUB;
 
   // ---------------------------------------------------------------- TMA ring
+  // the indexer keys are read once per step: first out of L2
+  const uint64_t stream_pol = l2_evict_first_policy();
   auto issue = [&](int i) {  // thread 0 only: sub-chunk i -> stage i % NS; two ring lengths ahead -> L2
     const int s_lo = k0 + i * SUB;
     const int s_hi = min(k1, s_lo + SUB);
@@ -270,17 +272,17 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     for (int ahead = (i < NS ? 1 : 2); ahead <= 2; ++ahead) {   // sub-chunks i + NS and i + 2 NS
       const int p_lo = s_lo + ahead * NS * SUB;
       const int np = max(0, min(min(k1, p_lo + SUB), t) - p_lo);
-      if (np > 0) bulk_prefetch_l2(kidx_cache + (size_t)p_lo * DI, (uint32_t)(np * RB));
+      if (np > 0) bulk_prefetch_l2_hint(kidx_cache + (size_t)p_lo * DI, (uint32_t)(np * RB), stream_pol);
     }
     uint64_t *bar = &bars[i % NS];
     unsigned char *dst = ring + (i % NS) * STB;
     if (ncopy > 0) {
       if constexpr (SG::kMma) {
         mbar_arrive_expect_tx(bar, (uint32_t)(SUB * RB));   // the whole box lands, out-of-range rows zero
-        tma_load_2d(dst, &kmap, 0, bg * p.L_max + s_lo, bar);
+        tma_load_2d_hint(dst, &kmap, 0, bg * p.L_max + s_lo, bar, stream_pol);
       } else {
         mbar_arrive_expect_tx(bar, (uint32_t)(ncopy * RB));
-        bulk_g2s(dst, kidx_cache + (size_t)s_lo * DI, (uint32_t)(ncopy * RB), bar);
+        bulk_g2s_hint(dst, kidx_cache + (size_t)s_lo * DI, (uint32_t)(ncopy * RB), bar, stream_pol);
       }
     } else {
       mbar_arrive(bar);
