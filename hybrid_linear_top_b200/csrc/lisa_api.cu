@@ -108,6 +108,92 @@ void fill_rows(lisa::RowsParams &r, const lisa_layer *L, int T) {
   r.scale = (float)(1.0 / sqrt((double)L->d));
   r.k_cache = L->k_cache; r.v_cache = L->v_cache; r.kidx_cache = L->kidx_cache;
   r.state = L->state; r.pos = L->pos; r.err_word = L->err_word;
+  r.sel_heads = L->Hkv;
+}
+
+// ---------------------------------------------------------------- definition variants
+// Geometry of a variant: P indexer-key planes, Gs selection groups.
+struct VariantGeom {
+  bool per_head, shared, lin_kv;
+  int P, Gs;
+  bool row_indexer() const { return per_head || shared; }   // indexer + top-M through the row path
+};
+
+lisa_status check_variant(const lisa_layer *L, int variant, VariantGeom &vg) {
+  if (variant & ~(LISA_VAR_KEY_PER_INDEXER_HEAD | LISA_VAR_SHARED_SET | LISA_VAR_LINEAR_KV_PER_QUERY_HEAD))
+    return fail(LISA_ERR_INVALID_ARG, "unknown variant bits 0x%x", variant);
+  vg.per_head = (variant & LISA_VAR_KEY_PER_INDEXER_HEAD) != 0;
+  vg.shared = (variant & LISA_VAR_SHARED_SET) != 0;
+  vg.lin_kv = (variant & LISA_VAR_LINEAR_KV_PER_QUERY_HEAD) != 0;
+  vg.Gs = vg.shared ? 1 : L->Hkv;
+  vg.P = vg.per_head ? L->HI : vg.Gs;
+  if (!vg.per_head && L->HI / vg.Gs > lisa::kMaxR)
+    return fail(LISA_ERR_UNSUPPORTED, "%d indexer heads per selection group > %d", L->HI / vg.Gs, lisa::kMaxR);
+  return LISA_OK;
+}
+
+struct VarPlan {
+  int row_chunk, L_keys;
+  size_t keys, keys_h, idx, olin, dS, Ptot, total;
+};
+// op: LISA_OP_DECODE (T = 1 row at pos[b]), LISA_OP_INDEXER_TOPK or LISA_OP_PREFILL.
+VarPlan var_plan(const lisa_layer *L, const VariantGeom &vg, int T, int op) {
+  VarPlan p;
+  memset(&p, 0, sizeof(p));
+  const bool prefill = op == LISA_OP_PREFILL;
+  const bool indexer = op == LISA_OP_INDEXER_TOPK || prefill || vg.row_indexer();
+  if (op == LISA_OP_DECODE) T = 1;
+  p.row_chunk = T < kRowChunk ? T : kRowChunk;
+  p.L_keys = round4(prefill ? T : L->L_max);
+  const size_t rk = (size_t)p.row_chunk * p.L_keys * 4;
+  size_t off = 0;
+  if (indexer) {
+    p.keys = off; off += round256((size_t)L->B * vg.Gs * rk);
+    if (vg.P != vg.Gs) { p.keys_h = off; off += round256((size_t)L->B * L->HI * rk); }
+  }
+  if (prefill || (op == LISA_OP_DECODE && vg.row_indexer())) {
+    p.idx = off; off += round256((size_t)L->B * T * vg.Gs * L->M * 4);
+  }
+  if (prefill) {
+    const size_t LH = vg.lin_kv ? L->Hq : L->Hkv;
+    const size_t nc = (T + lisa::kLinChunk - 1) / lisa::kLinChunk;
+    p.olin = off; off += round256((size_t)L->B * T * L->Hq * L->d * 4);
+    p.dS = off; off += round256((size_t)L->B * LH * nc * L->d * L->d * 4);
+    p.Ptot = off; off += round256((size_t)L->B * LH * L->d * L->d * 4);
+  }
+  p.total = off;
+  return p;
+}
+
+void set_select_smem(lisa::RowsParams &r, int n_max);
+
+// Row-path parameters of the variant's indexer: `sel` scores and selects in
+// the Gs selection groups; with one key per indexer head, `ph` first scores
+// every indexer head on its own (the groups' sums are formed afterwards).
+void variant_indexer_params(const lisa_layer *L, const VariantGeom &vg, int T, const VarPlan &plan, char *ws,
+                            const void *qidx, const float *w, int *idx, int n_max, lisa::RowsParams &sel,
+                            lisa::RowsParams &ph) {
+  fill_rows(sel, L, T);
+  sel.Hkv = vg.Gs; sel.R = L->HI / vg.Gs; sel.G = L->Hq / vg.Gs; sel.sel_heads = vg.Gs;
+  sel.qidx = qidx; sel.w = w; sel.idx = idx;
+  sel.keys = reinterpret_cast<uint32_t *>(ws + plan.keys);
+  sel.row_chunk = plan.row_chunk;
+  sel.L_keys = plan.L_keys;
+  set_select_smem(sel, n_max);
+  ph = sel;
+  ph.Hkv = L->HI; ph.R = 1; ph.G = 1; ph.sel_heads = L->HI;
+  ph.keys = vg.P != vg.Gs ? reinterpret_cast<uint32_t *>(ws + plan.keys_h) : nullptr;
+}
+
+// Appends the indexer keys of T tokens ([B, T, P, dI]) at pos[b] + tau.
+cudaError_t append_kidx_planes(const lisa_layer *L, const VariantGeom &vg, int T, const void *kidx, int require_pos0,
+                               cudaStream_t st) {
+  lisa::RowsParams a;
+  fill_rows(a, L, T);
+  a.Hkv = vg.P; a.R = 1; a.G = 1;
+  a.require_pos0 = require_pos0;
+  a.kidx = kidx;
+  return lisa::launch_append(a, L->dtype, st);
 }
 
 void set_select_smem(lisa::RowsParams &r, int n_max) {
@@ -445,6 +531,179 @@ lisa_status lisa_indexer_topk_noalloc(const lisa_layer *L, const void *qidx, con
   set_select_smem(r, L->L_max);
   cudaError_t e = lisa::launch_rows_topk(r, L->dtype, (cudaStream_t)stream, L->L_max);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_noalloc");
+  return ok();
+}
+
+size_t lisa_workspace_bytes_variant(const lisa_layer *layer, int variant, int T, int op) {
+  VariantGeom vg;
+  if (check_layer(layer) != LISA_OK || T < 0 || check_variant(layer, variant, vg) != LISA_OK) return 0;
+  if (op == LISA_OP_DECODE) return vg.row_indexer() ? var_plan(layer, vg, 1, op).total : 0;
+  if (op == LISA_OP_PREFILL || op == LISA_OP_INDEXER_TOPK) return T ? var_plan(layer, vg, T, op).total : 0;
+  return 0;
+}
+
+lisa_status lisa_append_cache_variant(const lisa_layer *L, int variant, const void *k, const void *v,
+                                      const void *kidx, int T, void *stream) {
+  lisa_status s;
+  VariantGeom vg;
+  if ((s = check_layer(L)) || (s = check_variant(L, variant, vg))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) || (s = check_ptr(kidx, "kidx"))) return s;
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.k = k; r.v = v;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = lisa::launch_append(r, L->dtype, st);
+  if (e == cudaSuccess) e = append_kidx_planes(L, vg, T, kidx, 0, st);
+  if (e != cudaSuccess) return cuda_fail(e, "append_cache_variant");
+  return ok();
+}
+
+lisa_status lisa_indexer_topk_variant(const lisa_layer *L, int variant, const void *qidx, const float *w, int T,
+                                      int *idx_out, void *workspace, size_t ws_bytes, void *stream) {
+  lisa_status s;
+  VariantGeom vg;
+  if ((s = check_layer(L)) || (s = check_variant(L, variant, vg))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(idx_out, "idx_out"))) return s;
+  const VarPlan plan = var_plan(L, vg, T, LISA_OP_INDEXER_TOPK);
+  if (!workspace || ws_bytes < plan.total)
+    return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
+  if ((s = check_ptr(workspace, "workspace"))) return s;
+  lisa::RowsParams sel, ph;
+  variant_indexer_params(L, vg, T, plan, static_cast<char *>(workspace), qidx, w, idx_out, L->L_max, sel, ph);
+  cudaError_t e = lisa::launch_rows_topk(sel, L->dtype, (cudaStream_t)stream, L->L_max, ph.keys ? &ph : nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_variant");
+  return ok();
+}
+
+lisa_status lisa_decode_step_variant(const lisa_layer *L, int variant, const void *q, const void *k, const void *v,
+                                     const void *kidx, const void *qidx, const float *w, const float *gate_logit,
+                                     const void *k_lin, const void *v_lin, int fuse_append, void *out, int *idx_out,
+                                     void *workspace, size_t ws_bytes, void *stream) {
+  lisa_status s;
+  VariantGeom vg;
+  if ((s = check_layer(L)) || (s = check_variant(L, variant, vg))) return s;
+  if (L->B == 0) return ok();
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(L->state, "state"))) return s;
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) || (s = check_ptr(kidx, "kidx")) ||
+      (s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(gate_logit, "gate_logit")) ||
+      (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)) ||
+      (s = check_ptr(k_lin, "k_lin", vg.lin_kv)) || (s = check_ptr(v_lin, "v_lin", vg.lin_kv)))
+    return s;
+  const int esz = L->dtype == LISA_BF16 ? 2 : 4;
+  if (lisa::decode_smem_bytes(L->L_max, L->M, L->Hq / L->Hkv, L->d, L->dI, esz, 8, vg.lin_kv) > kMaxSmem)
+    return fail(LISA_ERR_UNSUPPORTED, "L_max=%d needs more shared memory per CTA than a B200 SM has", L->L_max);
+  VarPlan plan;
+  memset(&plan, 0, sizeof(plan));
+  if (vg.row_indexer()) {
+    plan = var_plan(L, vg, 1, LISA_OP_DECODE);
+    if (!workspace || ws_bytes < plan.total)
+      return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
+    if ((s = check_ptr(workspace, "workspace"))) return s;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  lisa::DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.B = L->B; p.Hq = L->Hq; p.Hkv = L->Hkv; p.G = L->Hq / L->Hkv; p.HI = L->HI; p.R = L->HI / L->Hkv;
+  p.D = L->d; p.DI = L->dI; p.M = L->M; p.L_max = L->L_max; p.fuse_append = fuse_append ? 1 : 0;
+  p.split_req = L->decode_split;
+  p.scale = (float)(1.0 / sqrt((double)L->d));
+  p.k_cache = L->k_cache; p.v_cache = L->v_cache; p.kidx_cache = L->kidx_cache;
+  p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;
+  p.q = q; p.k = k; p.v = v; p.kidx = kidx; p.qidx = qidx; p.w = w; p.gate = gate_logit;
+  p.out = out; p.idx_out = idx_out;
+  if (vg.lin_kv) {
+    p.k_lin = k_lin;
+    p.v_lin = v_lin;
+  }
+  cudaError_t e = cudaSuccess;
+  if (vg.row_indexer()) {
+    // the new token's indexer keys go into the cache first: the row path reads rows 0..t there
+    char *ws = static_cast<char *>(workspace);
+    int *idx = idx_out ? idx_out : reinterpret_cast<int *>(ws + plan.idx);
+    if (fuse_append) e = append_kidx_planes(L, vg, 1, kidx, 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode_step_variant append");
+    lisa::RowsParams sel, ph;
+    variant_indexer_params(L, vg, 1, plan, ws, qidx, w, idx, L->L_max, sel, ph);
+    e = lisa::launch_rows_topk(sel, L->dtype, st, L->L_max, ph.keys ? &ph : nullptr);
+    if (e != cudaSuccess) return cuda_fail(e, "decode_step_variant indexer");
+    p.sel_ext = idx;
+    p.sel_groups = vg.Gs;
+    p.kidx = nullptr; p.qidx = nullptr; p.w = nullptr;
+    p.idx_out = nullptr;
+  }
+  e = lisa::launch_decode(p, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step_variant");
+  return ok();
+}
+
+lisa_status lisa_prefill_variant(const lisa_layer *L, int variant, int T, const void *q, const void *k, const void *v,
+                                 const void *kidx, const void *qidx, const float *w, const float *gate_logit,
+                                 const void *k_lin, const void *v_lin, void *out, int *idx_out, void *workspace,
+                                 size_t ws_bytes, void *stream) {
+  lisa_status s;
+  VariantGeom vg;
+  if ((s = check_layer(L)) || (s = check_variant(L, variant, vg))) return s;
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
+  if ((s = check_caches(L))) return s;
+  if ((s = check_ptr(L->state, "state"))) return s;
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) || (s = check_ptr(kidx, "kidx")) ||
+      (s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(gate_logit, "gate_logit")) ||
+      (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)) ||
+      (s = check_ptr(k_lin, "k_lin", vg.lin_kv)) || (s = check_ptr(v_lin, "v_lin", vg.lin_kv)))
+    return s;
+  const VarPlan plan = var_plan(L, vg, T, LISA_OP_PREFILL);
+  if (!workspace || ws_bytes < plan.total)
+    return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, plan.total);
+  if ((s = check_ptr(workspace, "workspace"))) return s;
+  char *ws = static_cast<char *>(workspace);
+  cudaStream_t st = (cudaStream_t)stream;
+  int *idx = idx_out ? idx_out : reinterpret_cast<int *>(ws + plan.idx);
+
+  // k, v and the indexer keys (P planes) into the caches
+  lisa::RowsParams r;
+  fill_rows(r, L, T);
+  r.require_pos0 = 1;
+  r.k = k; r.v = v;
+  cudaError_t e = lisa::launch_append(r, L->dtype, st);
+  if (e == cudaSuccess) e = append_kidx_planes(L, vg, T, kidx, 1, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_variant append");
+  // linear branch: with keys / values per query head it runs as Hq groups of one head
+  r.q = q; r.gate = gate_logit; r.out = out;
+  r.olin = reinterpret_cast<float *>(ws + plan.olin);
+  r.dS = reinterpret_cast<float *>(ws + plan.dS);
+  r.Ptot = reinterpret_cast<float *>(ws + plan.Ptot);
+  {
+    lisa::RowsParams rl = r;
+    if (vg.lin_kv) {
+      rl.Hkv = L->Hq; rl.G = 1;
+      rl.k = k_lin; rl.v = v_lin;
+    }
+    e = lisa::launch_prefill_linear(rl, L->dtype, st);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill_variant linear");
+  }
+  // indexer + top-M in the Gs selection groups
+  lisa::RowsParams sel, ph;
+  variant_indexer_params(L, vg, T, plan, ws, qidx, w, idx, T, sel, ph);
+  sel.require_pos0 = 1;
+  ph.require_pos0 = 1;
+  e = lisa::launch_rows_topk(sel, L->dtype, st, T, ph.keys ? &ph : nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_variant indexer");
+  // sparse attention + gate: every KV head reads its group's list
+  r.idx = idx;
+  r.sel_heads = vg.Gs;
+  e = lisa::launch_prefill_attend(r, L->dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill_variant attend");
   return ok();
 }
 

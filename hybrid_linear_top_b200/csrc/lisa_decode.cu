@@ -55,7 +55,7 @@ struct ScoreGeom {
 
 struct DecLayout {
   int region0, cand_key, cand_pos, pin;
-  int keys, hist, tot, misc, sel, qs, qi, ks, vs, kis, gl, part, pml, olin, logit, sidx, bars, total;
+  int keys, hist, tot, misc, sel, qs, qi, ks, vs, kis, gl, klin, vlin, part, pml, olin, logit, sidx, bars, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
@@ -67,7 +67,8 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // gathered K / V rows (attention) followed by the partials that every rank
 // writes for this CTA's output columns (merge).
 __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, int G, int D, int DI, int esize,
-                                                int NC, int stages = kStages, int stage_bytes = kStageBytes) {
+                                                int NC, int stages = kStages, int stage_bytes = kStageBytes,
+                                                bool lin_kv = false) {
   DecLayout L;
   const int rpc = M / NC;
   const int kv = 2 * rpc * (D * esize + 16);
@@ -92,6 +93,8 @@ __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, i
   L.vs = off; off += align16(D * 4);
   L.kis = off; off += align16(DI * 4);
   L.gl = off; off += align16(G * 4);
+  L.klin = off; off += lin_kv ? align16(G * D * 4) : 0;   // linear-branch k, v per query head (variant)
+  L.vlin = off; off += lin_kv ? align16(G * D * 4) : 0;
   L.part = off; off += align16(G * D * 4);
   L.pml = off; off += align16(2 * G * 4);
   L.olin = off; off += align16(G * (D / NC) * 4);
@@ -167,7 +170,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   const int NS = p.stages;
   const int SUB = p.stage_keys;                  // keys per ring stage
   const int STB = SUB * RB;                      // bytes per ring stage
-  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC, NS, STB);
+  const bool lin_kv = p.k_lin != nullptr;  // variant: linear-branch k, v of its own per query head
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC, NS, STB, lin_kv);
   unsigned char *ring = smem + lay.region0;
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem + lay.keys);
   uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist);
@@ -180,6 +184,8 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   float *vs = reinterpret_cast<float *>(smem + lay.vs);
   float *kis = reinterpret_cast<float *>(smem + lay.kis);   // the new token's indexer key
   float *gls = reinterpret_cast<float *>(smem + lay.gl);    // gate logits of the G heads
+  float *klin = reinterpret_cast<float *>(smem + lay.klin); // [G][D] (variant only)
+  float *vlin = reinterpret_cast<float *>(smem + lay.vlin); // [G][D] (variant only)
   float *part = reinterpret_cast<float *>(smem + lay.part);
   float *pml = reinterpret_cast<float *>(smem + lay.pml);
   float *olin = reinterpret_cast<float *>(smem + lay.olin);
@@ -204,27 +210,36 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   const T *kin = reinterpret_cast<const T *>(p.k) + (size_t)bg * D;
   const T *vin = reinterpret_cast<const T *>(p.v) + (size_t)bg * D;
   const T *qidx_in = reinterpret_cast<const T *>(p.qidx) + ((size_t)b * p.HI + g * R) * DI;
-  const bool window = p.window != 0;      // sliding-window variant: no indexer, no top-M
+  const bool ext = p.sel_ext != nullptr;  // index lists given by the caller
+  const bool window = p.window != 0 || ext;   // no indexer, no top-M: the window's lists or the given ones
   // The step's own rows as 16-byte chunks, [q of the G heads | k | v |
-  // indexer queries of the R heads | new indexer key], loaded into registers
-  // with every load in flight at once (one DRAM round trip, not one per row),
-  // then widened into shared memory below.
+  // indexer queries of the R heads | new indexer key | linear-branch k, v of
+  // the G heads (variant)], loaded into registers with every load in flight
+  // at once (one DRAM round trip, not one per row), then widened into shared
+  // memory below.
   const int o_k = G * D / VEC, o_v = o_k + D / VEC, o_qi = o_v + D / VEC;
   const int o_ki = o_qi + (window ? 0 : R * DI / VEC);
-  const int n_in = o_ki + (p.kidx ? DI / VEC : 0);
+  const int o_kl = o_ki + (p.kidx ? DI / VEC : 0);
+  const int o_vl = o_kl + (lin_kv ? G * D / VEC : 0);
+  const int n_in = o_vl + (lin_kv ? G * D / VEC : 0);
+  const size_t lin_off = ((size_t)b * p.Hq + g * G) * D;
   auto chunk_src = [&](int c) -> const uint4 * {
     if (c < o_k) return reinterpret_cast<const uint4 *>(qin) + c;
     if (c < o_v) return reinterpret_cast<const uint4 *>(kin) + (c - o_k);
     if (c < o_qi) return reinterpret_cast<const uint4 *>(vin) + (c - o_v);
     if (c < o_ki) return reinterpret_cast<const uint4 *>(qidx_in) + (c - o_qi);
-    return reinterpret_cast<const uint4 *>(kidx_new) + (c - o_ki);
+    if (c < o_kl) return reinterpret_cast<const uint4 *>(kidx_new) + (c - o_ki);
+    if (c < o_vl) return reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(p.k_lin) + lin_off) + (c - o_kl);
+    return reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(p.v_lin) + lin_off) + (c - o_vl);
   };
   auto chunk_dst = [&](int c) -> float * {
     if (c < o_k) return qs + c * VEC;
     if (c < o_v) return ks + (c - o_k) * VEC;
     if (c < o_qi) return vs + (c - o_v) * VEC;
     if (c < o_ki) return qis + (c - o_qi) * VEC;
-    return kis + (c - o_ki) * VEC;
+    if (c < o_kl) return kis + (c - o_ki) * VEC;
+    if (c < o_vl) return klin + (c - o_kl) * VEC;
+    return vlin + (c - o_vl) * VEC;
   };
   constexpr int kInRegs = 2;               // chunks per thread held in registers
   uint4 inr[kInRegs];
@@ -302,7 +317,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         reinterpret_cast<uint4 *>(reinterpret_cast<T *>(p.k_cache) + arow * D)[c - o_k] = u;
       else if (c >= o_v && c < o_qi)
         reinterpret_cast<uint4 *>(reinterpret_cast<T *>(p.v_cache) + arow * D)[c - o_v] = u;
-      else if (c >= o_ki)
+      else if (c >= o_ki && c < o_kl)
         reinterpret_cast<uint4 *>(reinterpret_cast<T *>(p.kidx_cache) + arow * DI)[c - o_ki] = u;
     };
 #pragma unroll
@@ -358,18 +373,25 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         if (hh >= hn) continue;
         float *S = p.state + ((size_t)b * p.Hq + g * G + h0 + hh) * D * D;
         const float *qh = qs + (h0 + hh) * D;
+        const float *kh = ks;            // the attention's k, or the head's own (variant)
+        float vh[4] = {vj[0], vj[1], vj[2], vj[3]};
+        if (lin_kv) {
+          kh = klin + (h0 + hh) * D;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) vh[j] = vlin[(h0 + hh) * D + c0s + cq * 4 + j];
+        }
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
         for (int it = 0; it < ITER; ++it) {
           const int idx = tid + it * kDecThreads;
           if (idx < D * QPR) {
             const int i = idx / QPR;
-            const float ki = ks[i], qi = qh[i];
+            const float ki = kh[i], qi = qh[i];
             float4 sn = sv[hh][it];
-            sn.x = fmaf(ki, vj[0], sn.x);
-            sn.y = fmaf(ki, vj[1], sn.y);
-            sn.z = fmaf(ki, vj[2], sn.z);
-            sn.w = fmaf(ki, vj[3], sn.w);
+            sn.x = fmaf(ki, vh[0], sn.x);
+            sn.y = fmaf(ki, vh[1], sn.y);
+            sn.z = fmaf(ki, vh[2], sn.z);
+            sn.w = fmaf(ki, vh[3], sn.w);
             *reinterpret_cast<float4 *>(S + (size_t)i * D + c0s + cq * 4) = sn;
             a0 = fmaf(qi, sn.x, a0);
             a1 = fmaf(qi, sn.y, a1);
@@ -489,9 +511,14 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   // ---------------------------------------------------------------- top-M
   int *sel0 = cluster.map_shared_rank(sel, 0);
   if (window) {
-    // the M (= W) most recent positions t-M+1 .. t, or the whole prefix
-    if (rank == 0)
-      for (int j = tid; j < M; j += kDecThreads) sel[j] = n <= M ? (j < n ? j : -1) : t - M + 1 + j;
+    if (rank == 0) {
+      if (ext) {                         // the caller's list of this (b, group)
+        const int *src = p.sel_ext + ((size_t)b * p.sel_groups + (p.sel_groups == 1 ? 0 : g)) * M;
+        for (int j = tid; j < M; j += kDecThreads) sel[j] = src[j];
+      } else {                           // the M (= W) most recent positions t-M+1 .. t, or the whole prefix
+        for (int j = tid; j < M; j += kDecThreads) sel[j] = n <= M ? (j < n ? j : -1) : t - M + 1 + j;
+      }
+    }
   } else if (n > M) {
     constexpr int SEG = kCandCap / NC;                  // candidate slots of each rank in CTA 0
     uint32_t *fh = hist + 1024;                         // CTA 0: 1024-bin histogram of candidate keys
@@ -1085,7 +1112,7 @@ template <typename T, int D, int DI, int NC>
 static cudaError_t launch_cluster_t(const DecodeParams &p, const CUtensorMap &kmap, cudaStream_t st) {
   auto kern = decode_cluster_kernel<T, D, DI, NC>;
   const DecLayout lay = dec_layout(p.kpc_max, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), NC, p.stages,
-                                   p.stage_keys * ScoreGeom<T, DI>::RB);
+                                   p.stage_keys * ScoreGeom<T, DI>::RB, p.k_lin != nullptr);
   cudaError_t e = prepare_kernel(kern, lay.total);
   if (e != cudaSuccess) return e;
   if (NC > 8) {
@@ -1114,7 +1141,8 @@ template <typename T, int D, int DI>
 static int pick_cluster(const DecodeParams &p) {
   auto kern = decode_cluster_kernel<T, D, DI, 16>;
   const int kpc = (((p.L_max + 15) / 16) + 31) & ~31;
-  const DecLayout lay = dec_layout(kpc, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), 16);
+  const DecLayout lay = dec_layout(kpc, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), 16, kStages, kStageBytes,
+                                   p.k_lin != nullptr);
   if (prepare_kernel(kern, lay.total) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
@@ -1148,7 +1176,7 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
   static int next = 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  const int key = p.L_max * 2 + (p.M << 20) + (p.G << 28);
+  const int key = p.L_max * 2 + (p.k_lin ? 1 : 0) + (p.M << 20) + (p.G << 28);
   int ok16 = -1, sms = 0;
   for (int i = 0; i < 8; ++i)
     if (cache_dev[i] == dev && cache_key[i] == key) {
@@ -1176,7 +1204,8 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
     nc = pairs * 16 <= sms ? 16 : pairs * 8 <= 2 * sms ? 8 : 4;
   }
   if (nc == 16 && !ok16) nc = 8;
-  if (nc == 4 && dec_layout((((p.L_max + 3) / 4) + 31) & ~31, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), 4, 2).total >
+  if (nc == 4 && dec_layout((((p.L_max + 3) / 4) + 31) & ~31, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), 4, 2,
+                            kStageBytes, p.k_lin != nullptr).total >
                      227 * 1024)
     nc = 8;
   p.nc = nc;
@@ -1186,7 +1215,7 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
   p.kpc_max = (((p.L_max + nc - 1) / nc) + 31) & ~31;
   CUtensorMap kmap;
   memset(&kmap, 0, sizeof(kmap));
-  if (ScoreGeom<T, DI>::kMma) {
+  if (ScoreGeom<T, DI>::kMma && !p.sel_ext) {   // given lists: no key stream
     using SG = ScoreGeom<T, DI>;
     if (!make_tmap_2d(&kmap, p.kidx_cache, (int)sizeof(T), (unsigned long long)DI,
                       (unsigned long long)p.B * p.Hkv * p.L_max, (unsigned long long)SG::RB, DI, p.stage_keys, SG::RB))
@@ -1197,9 +1226,9 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
   return launch_cluster_t<T, D, DI, 8>(p, kmap, st);
 }
 
-int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc) {
+int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc, bool lin_kv) {
   const int kpc = (((L_max + nc - 1) / nc) + 31) & ~31;
-  return dec_layout(kpc, L_max, M, G, D, DI, esize, nc).total;
+  return dec_layout(kpc, L_max, M, G, D, DI, esize, nc, kStages, kStageBytes, lin_kv).total;
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t st) {

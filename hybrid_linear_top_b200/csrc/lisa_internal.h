@@ -52,6 +52,9 @@ struct DecodeParams {
   // launch geometry (filled by the launcher)
   int split_req;                        // requested CTAs per (b, g): 0 (library's choice), 4, 8, 16
   int window;                           // 1: sliding-window variant (M = the window W; no indexer inputs)
+  const int *sel_ext;                   // non-NULL: index lists given, [B, sel_groups, M] (no indexer inputs)
+  int sel_groups;                       // selection groups of sel_ext: 1 (one set for every KV head) or Hkv
+  const void *k_lin, *v_lin;            // non-NULL: linear-branch keys / values per query head [B, Hq, d]
   int nc;                               // CTAs per cluster
   int stages;                           // TMA ring stages
   int stage_keys;                       // keys per ring stage
@@ -59,7 +62,7 @@ struct DecodeParams {
 };
 
 // Dynamic shared memory of the decode kernel for a cluster of nc CTAs.
-int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc);
+int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc, bool lin_kv = false);
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t st);
 
 // ------------------------------------------------------------- row path
@@ -75,7 +78,9 @@ struct RowsParams {
   const void *q, *k, *v, *kidx, *qidx;
   const float *w, *gate;
   void *out;
-  int *idx;                             // [B, T, Hkv, M] (caller's idx_out or workspace)
+  int *idx;                             // [B, T, sel_heads, M] (caller's idx_out or workspace)
+  int sel_heads;                        // index lists per token read by the attention: Hkv, or 1 (one set
+                                        // shared by every KV head)
   // workspace
   uint32_t *keys;                       // [B, Hkv, row_chunk, L_keys]
   float *olin;                          // [B, T, Hq, d]
@@ -88,7 +93,11 @@ struct RowsParams {
 };
 
 cudaError_t launch_append(const RowsParams &p, int dtype, cudaStream_t st);
-cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, int key_limit);
+// Indexer scores + row top-M.  With ph != NULL the scores are first computed
+// per indexer head with ph (one head per group, into ph->keys) and then summed
+// over the HI / (p.Hkv) heads of each of p's groups into p.keys.
+cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, int key_limit,
+                             const RowsParams *ph = nullptr);
 // bf16 indexer scores of rows [tau0, tau0 + rows) of the pass on the tensor cores.
 cudaError_t launch_rows_score_tc(const RowsParams &p, cudaStream_t st, int tau0, int rows, int key_hi);
 cudaError_t launch_prefill_linear(const RowsParams &p, int dtype, cudaStream_t st);

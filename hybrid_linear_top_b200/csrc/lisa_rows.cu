@@ -17,7 +17,8 @@ __device__ __forceinline__ bool rows_pos_ok(const RowsParams &p, int b) {
 }
 
 // ============================================================ append
-// grid (T, B*Hkv); copies k, v, kidx row tau of (b, g) to cache row pos[b]+tau.
+// grid (T, B*Hkv); copies k, v, kidx row tau of (b, g) to cache row pos[b]+tau
+// (k and v when p.k is non-NULL, kidx when p.kidx is non-NULL).
 template <typename T>
 __global__ void append_kernel(RowsParams p) {
   const int tau = blockIdx.x;
@@ -36,10 +37,11 @@ __global__ void append_kernel(RowsParams p) {
   uint4 *kd = reinterpret_cast<uint4 *>(p.k_cache) + dst * nd;
   uint4 *vd = reinterpret_cast<uint4 *>(p.v_cache) + dst * nd;
   uint4 *kid = reinterpret_cast<uint4 *>(p.kidx_cache) + dst * ndi;
-  for (int i = threadIdx.x; i < nd; i += blockDim.x) {
-    kd[i] = ks[i];
-    vd[i] = vs[i];
-  }
+  if (p.k)
+    for (int i = threadIdx.x; i < nd; i += blockDim.x) {
+      kd[i] = ks[i];
+      vd[i] = vs[i];
+    }
   if (p.kidx)
     for (int i = threadIdx.x; i < ndi; i += blockDim.x) kid[i] = kis[i];
 }
@@ -207,23 +209,46 @@ __global__ void __launch_bounds__(NT) rows_select_kernel(RowsParams p, int tau0,
     set_err(p.err_word, LISA_DEVERR_CHECK);
 }
 
+// grid (rows of the pass, B*Hkv of p); one indexer key per indexer head: the
+// score of group g is the sum of the per-head scores of its Rc = ph.Hkv / p.Hkv
+// heads (ph scored one head per group), each a weighted ReLU term already.
+__global__ void combine_heads_kernel(RowsParams p, const uint32_t *__restrict__ keys_h, int Rc, int tau0, int rows) {
+  const int rr = blockIdx.x, bg = blockIdx.y;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  if (rr >= rows || !rows_pos_ok(p, b)) return;
+  const int n = p.pos[b] + tau0 + rr + 1;
+  const uint32_t *src = keys_h + (((size_t)b * p.Hkv * Rc + (size_t)g * Rc) * p.row_chunk + rr) * p.L_keys;
+  const size_t plane = (size_t)p.row_chunk * p.L_keys;
+  uint32_t *dst = p.keys + ((size_t)bg * p.row_chunk + rr) * p.L_keys;
+  for (int s = threadIdx.x; s < n; s += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < Rc; ++r) acc += key_score(__ldcg(src + r * plane + s));
+    dst[s] = score_key(acc);
+  }
+}
+
 template <typename T, int DI>
-static cudaError_t rows_topk_t(const RowsParams &p, cudaStream_t st, int key_limit) {
+static cudaError_t rows_topk_t(const RowsParams &p, cudaStream_t st, int key_limit, const RowsParams *ph) {
   constexpr int NT = 256;
   cudaError_t e = prepare_kernel(rows_select_kernel<NT>, (int)p.select_smem);
   if (e != cudaSuccess) return e;
   e = prepare_kernel(rows_score_kernel<T, DI>);
   if (e != cudaSuccess) return e;
+  const RowsParams &ps = ph ? *ph : p;                // the geometry the scores are computed in
   for (int tau0 = 0; tau0 < p.T; tau0 += p.row_chunk) {
     const int rows = min(p.row_chunk, p.T - tau0);
     // prefill (pos 0): keys up to tau0 + rows; general positions: up to key_limit
     const int key_hi = p.require_pos0 ? min(key_limit, tau0 + rows) : key_limit;
     if constexpr (sizeof(T) == 2) {
-      e = launch_rows_score_tc(p, st, tau0, rows, key_hi);      // tensor cores (tcgen05)
+      e = launch_rows_score_tc(ps, st, tau0, rows, key_hi);     // tensor cores (tcgen05)
       if (e != cudaSuccess) return e;
     } else {
-      dim3 g1((key_hi + 63) / 64, (rows + 63) / 64, p.B * p.Hkv);   // fp32: CUDA cores, exact products
-      rows_score_kernel<T, DI><<<g1, 256, 0, st>>>(p, tau0, rows);
+      dim3 g1((key_hi + 63) / 64, (rows + 63) / 64, ps.B * ps.Hkv);   // fp32: CUDA cores, exact products
+      rows_score_kernel<T, DI><<<g1, 256, 0, st>>>(ps, tau0, rows);
+    }
+    if (ph) {
+      dim3 gc(rows, p.B * p.Hkv);
+      combine_heads_kernel<<<gc, 256, 0, st>>>(p, ph->keys, ph->Hkv / p.Hkv, tau0, rows);
     }
     dim3 g2(rows, p.B * p.Hkv);
     rows_select_kernel<NT><<<g2, NT, p.select_smem, st>>>(p, tau0, rows);
@@ -233,13 +258,13 @@ static cudaError_t rows_topk_t(const RowsParams &p, cudaStream_t st, int key_lim
   return cudaSuccess;
 }
 
-cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, int key_limit) {
+cudaError_t launch_rows_topk(const RowsParams &p, int dtype, cudaStream_t st, int key_limit, const RowsParams *ph) {
   if (dtype == LISA_BF16) {
-    if (p.DI == 64) return rows_topk_t<__nv_bfloat16, 64>(p, st, key_limit);
-    if (p.DI == 32) return rows_topk_t<__nv_bfloat16, 32>(p, st, key_limit);
+    if (p.DI == 64) return rows_topk_t<__nv_bfloat16, 64>(p, st, key_limit, ph);
+    if (p.DI == 32) return rows_topk_t<__nv_bfloat16, 32>(p, st, key_limit, ph);
   } else {
-    if (p.DI == 64) return rows_topk_t<float, 64>(p, st, key_limit);
-    if (p.DI == 32) return rows_topk_t<float, 32>(p, st, key_limit);
+    if (p.DI == 64) return rows_topk_t<float, 64>(p, st, key_limit, ph);
+    if (p.DI == 32) return rows_topk_t<float, 32>(p, st, key_limit, ph);
   }
   return cudaErrorInvalidValue;
 }
@@ -273,7 +298,7 @@ __global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
 #pragma unroll
     for (int j = 0; j < kDPL; ++j) acc[s][j] = 0.f;
   }
-  const int *idx = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M;
+  const int *idx = p.idx + (((size_t)b * p.T + tau) * p.sel_heads + (p.sel_heads == 1 ? 0 : g)) * p.M;
   const T *kc = reinterpret_cast<const T *>(p.k_cache) + (size_t)bg * p.L_max * D;
   const T *vc = reinterpret_cast<const T *>(p.v_cache) + (size_t)bg * p.L_max * D;
   constexpr int kSlices = D * (int)sizeof(T) / 16;
@@ -384,7 +409,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
   const int t_abs = p.pos[b] + tau;
   unsigned char *wbuf = s_att + warp * 4 * TILE; // [stage][K | V]
   const uint32_t wbuf_u32 = smem_u32(wbuf);
-  const int *idx = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M + warp * RW;
+  const int *idx = p.idx + (((size_t)b * p.T + tau) * p.sel_heads + (p.sel_heads == 1 ? 0 : g)) * p.M + warp * RW;
   const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(p.k_cache) + (size_t)bg * p.L_max * D;
   const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(p.v_cache) + (size_t)bg * p.L_max * D;
 

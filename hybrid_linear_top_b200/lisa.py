@@ -29,6 +29,9 @@ LISA_OP_DECODE = 0
 LISA_OP_PREFILL = 1
 LISA_OP_INDEXER_TOPK = 2
 LISA_OP_PREFILL_WINDOW = 3
+LISA_VAR_KEY_PER_INDEXER_HEAD = 1
+LISA_VAR_SHARED_SET = 2
+LISA_VAR_LINEAR_KV_PER_QUERY_HEAD = 4
 
 EXPORTED = [
     "lisa_workspace_bytes",
@@ -40,6 +43,11 @@ EXPORTED = [
     "lisa_decode_step_window",
     "lisa_prefill_window",
     "lisa_indexer_kl",
+    "lisa_workspace_bytes_variant",
+    "lisa_append_cache_variant",
+    "lisa_indexer_topk_variant",
+    "lisa_decode_step_variant",
+    "lisa_prefill_variant",
     "lisa_status_str",
     "lisa_last_error_msg",
     "lisa_version",
@@ -87,6 +95,17 @@ def _load():
     lib.lisa_prefill_window.restype = ctypes.c_int
     lib.lisa_indexer_kl.argtypes = [L, ctypes.c_int, P, P, P, P, P]
     lib.lisa_indexer_kl.restype = ctypes.c_int
+    I = ctypes.c_int
+    lib.lisa_workspace_bytes_variant.argtypes = [L, I, I, I]
+    lib.lisa_workspace_bytes_variant.restype = ctypes.c_size_t
+    lib.lisa_append_cache_variant.argtypes = [L, I, P, P, P, I, P]
+    lib.lisa_append_cache_variant.restype = I
+    lib.lisa_indexer_topk_variant.argtypes = [L, I, P, P, I, P, P, ctypes.c_size_t, P]
+    lib.lisa_indexer_topk_variant.restype = I
+    lib.lisa_decode_step_variant.argtypes = [L, I, P, P, P, P, P, P, P, P, P, I, P, P, P, ctypes.c_size_t, P]
+    lib.lisa_decode_step_variant.restype = I
+    lib.lisa_prefill_variant.argtypes = [L, I, I, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.lisa_prefill_variant.restype = I
     lib.lisa_status_str.argtypes = [ctypes.c_int]
     lib.lisa_status_str.restype = ctypes.c_char_p
     lib.lisa_last_error_msg.argtypes = []
@@ -239,3 +258,52 @@ def lisa_prefill(layer, T, q, k, v, kidx, qidx, w, gate_logit, out, idx_out, wor
     _check(_lib.lisa_prefill(ctypes.byref(c), int(T), _ptr(q), _ptr(k), _ptr(v), _ptr(kidx), _ptr(qidx), _ptr(w),
                              _ptr(gate_logit), _ptr(out), _ptr(idx_out), _ptr(workspace),
                              workspace.numel() if workspace is not None else 0, _stream(stream)))
+
+
+# ---------------------------------------------------------------- definition variants
+def variant_planes(layer, variant):
+    """(P, Gs): indexer-key planes and selection groups under `variant`."""
+    Gs = 1 if variant & LISA_VAR_SHARED_SET else layer.Hkv
+    P = layer.HI if variant & LISA_VAR_KEY_PER_INDEXER_HEAD else Gs
+    return P, Gs
+
+
+def lisa_workspace_bytes_variant(layer, variant, T, op):
+    c = layer.c_struct() if isinstance(layer, Layer) else layer
+    return int(_lib.lisa_workspace_bytes_variant(ctypes.byref(c), int(variant), int(T), int(op)))
+
+
+def alloc_workspace_variant(layer, variant, T, op, device="cuda"):
+    n = lisa_workspace_bytes_variant(layer, variant, T, op)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def lisa_append_cache_variant(layer, variant, k, v, kidx, T, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_append_cache_variant(ctypes.byref(c), int(variant), _ptr(k), _ptr(v), _ptr(kidx), int(T),
+                                          _stream(stream)))
+
+
+def lisa_indexer_topk_variant(layer, variant, qidx, w, T, idx_out, workspace, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_indexer_topk_variant(ctypes.byref(c), int(variant), _ptr(qidx), _ptr(w), int(T), _ptr(idx_out),
+                                          _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                          _stream(stream)))
+
+
+def lisa_decode_step_variant(layer, variant, q, k, v, kidx, qidx, w, gate_logit, k_lin, v_lin, fuse_append, out,
+                             idx_out, workspace, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_decode_step_variant(ctypes.byref(c), int(variant), _ptr(q), _ptr(k), _ptr(v), _ptr(kidx),
+                                         _ptr(qidx), _ptr(w), _ptr(gate_logit), _ptr(k_lin), _ptr(v_lin),
+                                         int(bool(fuse_append)), _ptr(out), _ptr(idx_out), _ptr(workspace),
+                                         workspace.numel() if workspace is not None else 0, _stream(stream)))
+
+
+def lisa_prefill_variant(layer, variant, T, q, k, v, kidx, qidx, w, gate_logit, k_lin, v_lin, out, idx_out,
+                         workspace, stream=None):
+    c = layer.c_struct()
+    _check(_lib.lisa_prefill_variant(ctypes.byref(c), int(variant), int(T), _ptr(q), _ptr(k), _ptr(v), _ptr(kidx),
+                                     _ptr(qidx), _ptr(w), _ptr(gate_logit), _ptr(k_lin), _ptr(v_lin), _ptr(out),
+                                     _ptr(idx_out), _ptr(workspace),
+                                     workspace.numel() if workspace is not None else 0, _stream(stream)))

@@ -238,6 +238,71 @@ LISA_API lisa_status lisa_prefill_window(const lisa_layer *layer, int T, const v
 LISA_API lisa_status lisa_indexer_topk_noalloc(const lisa_layer *layer, const void *qidx, const float *w,
                                                int T, int *idx_out, void *stream);
 
+/*
+ * Definition variants of the head mapping.  The pages say only that the
+ * indexer is a ReLU dot product of small query/key projections (gptget.net
+ * digest, method details) and that a linear-attention branch with phi =
+ * identity runs beside the sparse attention (abstract); how indexer heads,
+ * indexer keys and the linear branch's keys and values map onto the attention
+ * heads is left open.  The calls above fix one reading (one indexer key per KV
+ * head, one top-M set per KV head, the attention's own k and v in the linear
+ * branch).  These flags select the other readings:
+ *
+ *   LISA_VAR_KEY_PER_INDEXER_HEAD   every indexer head j has a key of its own:
+ *       I_g(t,s) = sum_{r<R} w[t,j] * max(0, qidx[t,j] . kidx[j, s]), j = g*R + r.
+ *       The indexer-key cache and the new tokens' kidx hold HI planes.
+ *   LISA_VAR_SHARED_SET             one top-M set per token, shared by every
+ *       KV head (Gs = 1 selection group over all HI indexer heads):
+ *       I(t,s) = sum_{j<HI} w[t,j] * max(0, qidx[t,j] . kidx[p(j), s]) with
+ *       p(j) = j under KEY_PER_INDEXER_HEAD and p(j) = 0 (one key per token)
+ *       otherwise.  Index lists have one group instead of Hkv.
+ *   LISA_VAR_LINEAR_KV_PER_QUERY_HEAD  the linear branch takes keys and
+ *       values of its own for every query head: S_h <- S_h + k_lin[h]^T
+ *       v_lin[h] (k_lin, v_lin [B, (T,) Hq, d], storage dtype).
+ *
+ * Shapes under a variant (P = indexer-key planes, Gs = selection groups):
+ *   P  = HI with KEY_PER_INDEXER_HEAD, else 1 with SHARED_SET, else Hkv;
+ *   Gs = 1 with SHARED_SET, else Hkv.
+ * The layer's kidx_cache is then [B, P, L_max, dI] and kidx arguments are
+ * [B, (T,) P, dI]; idx_out is [B, (T,) Gs, M].  Everything else (selection
+ * order, softmax scale, gate, state layout) is as defined at the top.
+ * variant = 0 is the default reading and runs the same kernels as the calls
+ * above.  With KEY_PER_INDEXER_HEAD or SHARED_SET the decode step runs the
+ * indexer and top-M through the row path (scores in the workspace) before the
+ * attention kernel, so it needs
+ * lisa_workspace_bytes_variant(layer, variant, 1, LISA_OP_DECODE) bytes of
+ * workspace; the prefill needs lisa_workspace_bytes_variant(layer, variant, T,
+ * LISA_OP_PREFILL).  Unknown flag bits return LISA_ERR_INVALID_ARG; k_lin and
+ * v_lin are required with LINEAR_KV_PER_QUERY_HEAD and ignored otherwise.
+ */
+#define LISA_VAR_KEY_PER_INDEXER_HEAD     1
+#define LISA_VAR_SHARED_SET               2
+#define LISA_VAR_LINEAR_KV_PER_QUERY_HEAD 4
+
+LISA_API size_t lisa_workspace_bytes_variant(const lisa_layer *layer, int variant, int T, int op);
+/* lisa_append_cache with kidx [B, T, P, dI] (P planes of the variant). */
+LISA_API lisa_status lisa_append_cache_variant(const lisa_layer *layer, int variant, const void *k, const void *v,
+                                               const void *kidx, int T, void *stream);
+/* lisa_indexer_topk under a variant; idx_out [B, T, Gs, M]; workspace
+ * lisa_workspace_bytes_variant(layer, variant, T, LISA_OP_INDEXER_TOPK). */
+LISA_API lisa_status lisa_indexer_topk_variant(const lisa_layer *layer, int variant, const void *qidx,
+                                               const float *w, int T, int *idx_out, void *workspace,
+                                               size_t ws_bytes, void *stream);
+/* lisa_decode_step under a variant: kidx [B, P, dI]; k_lin, v_lin [B, Hq, d];
+ * idx_out NULL or [B, Gs, M]. */
+LISA_API lisa_status lisa_decode_step_variant(const lisa_layer *layer, int variant, const void *q, const void *k,
+                                              const void *v, const void *kidx, const void *qidx, const float *w,
+                                              const float *gate_logit, const void *k_lin, const void *v_lin,
+                                              int fuse_append, void *out, int *idx_out, void *workspace,
+                                              size_t ws_bytes, void *stream);
+/* lisa_prefill under a variant: kidx [B, T, P, dI]; k_lin, v_lin [B, T, Hq, d];
+ * idx_out NULL or [B, T, Gs, M]. */
+LISA_API lisa_status lisa_prefill_variant(const lisa_layer *layer, int variant, int T, const void *q,
+                                          const void *k, const void *v, const void *kidx, const void *qidx,
+                                          const float *w, const float *gate_logit, const void *k_lin,
+                                          const void *v_lin, void *out, int *idx_out, void *workspace,
+                                          size_t ws_bytes, void *stream);
+
 /* Human-readable name of a status. */
 LISA_API const char *lisa_status_str(lisa_status s);
 

@@ -138,3 +138,60 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert "scratch" in L.last_error_msg()
     assert lib.lisa_indexer_topk_noalloc(ctypes.byref(c), FAKE, FAKE, 0, FAKE, None) == L.LISA_OK
     assert lib.lisa_indexer_topk_noalloc(ctypes.byref(_layer()), FAKE, None, 1, FAKE, None) == L.LISA_ERR_INVALID_ARG
+
+
+def _decode_variant(c, variant, ws=FAKE, ws_bytes=1 << 40, **ptrs):
+    args = {n: ptrs.get(n, FAKE) for n in ["q", "k", "v", "kidx", "qidx", "w", "gate", "k_lin", "v_lin", "out"]}
+    return L.lib().lisa_decode_step_variant(ctypes.byref(c), variant, args["q"], args["k"], args["v"], args["kidx"],
+                                            args["qidx"], args["w"], args["gate"], args["k_lin"], args["v_lin"], 1,
+                                            args["out"], None, ws, ws_bytes, None)
+
+
+def test_variant_flags_are_validated():
+    c = _layer()
+    assert _decode_variant(c, 8) == L.LISA_ERR_INVALID_ARG
+    assert "variant" in L.last_error_msg()
+    # the linear branch's own keys / values are required by that variant only
+    assert _decode_variant(c, L.LISA_VAR_LINEAR_KV_PER_QUERY_HEAD, k_lin=None) == L.LISA_ERR_INVALID_ARG
+    assert "k_lin" in L.last_error_msg()
+    assert _decode_variant(_layer(B=0), L.LISA_VAR_LINEAR_KV_PER_QUERY_HEAD, k_lin=None) == L.LISA_OK
+    # a shared set sums all indexer heads in one group: at most 8 without per-head keys
+    big = _layer(Hq=16, Hkv=4, HI=16)
+    assert _decode_variant(big, L.LISA_VAR_SHARED_SET) == L.LISA_ERR_UNSUPPORTED
+    assert L.lisa_workspace_bytes_variant(big, L.LISA_VAR_SHARED_SET, 1, L.LISA_OP_DECODE) == 0
+    assert L.lisa_workspace_bytes_variant(
+        big, L.LISA_VAR_SHARED_SET | L.LISA_VAR_KEY_PER_INDEXER_HEAD, 1, L.LISA_OP_DECODE) > 0
+
+
+def test_variant_workspace_sizes():
+    c = _layer()
+    V1, V2, V3 = L.LISA_VAR_KEY_PER_INDEXER_HEAD, L.LISA_VAR_SHARED_SET, L.LISA_VAR_LINEAR_KV_PER_QUERY_HEAD
+    ws = lambda v, T, op: L.lisa_workspace_bytes_variant(c, v, T, op)
+    # variant 0 needs what the default calls need
+    assert ws(0, 1, L.LISA_OP_DECODE) == 0
+    assert ws(0, 300, L.LISA_OP_PREFILL) == L.lisa_workspace_bytes(c, 300, L.LISA_OP_PREFILL)
+    assert ws(0, 7, L.LISA_OP_INDEXER_TOPK) == L.lisa_workspace_bytes(c, 7, L.LISA_OP_INDEXER_TOPK)
+    # the linear branch's own k / v alone keeps the fused decode kernel
+    assert ws(V3, 1, L.LISA_OP_DECODE) == 0
+    assert ws(V3, 300, L.LISA_OP_PREFILL) > ws(0, 300, L.LISA_OP_PREFILL)   # per-query-head increments
+    # the other two run the indexer through the row path: order keys of every cached position
+    for v in (V1, V2, V1 | V2):
+        assert ws(v, 1, L.LISA_OP_DECODE) >= 16384 * 4
+    # per-head keys: the per-head scores are kept beside the group sums
+    assert ws(V1, 7, L.LISA_OP_INDEXER_TOPK) > ws(0, 7, L.LISA_OP_INDEXER_TOPK)
+    assert ws(V2, 7, L.LISA_OP_INDEXER_TOPK) < ws(0, 7, L.LISA_OP_INDEXER_TOPK)    # one group instead of two
+    assert ws(8, 7, L.LISA_OP_INDEXER_TOPK) == 0
+
+
+def test_variant_calls_validate():
+    lib = L.lib()
+    c = _layer(L_max=100)
+    V1 = L.LISA_VAR_KEY_PER_INDEXER_HEAD
+    assert _decode_variant(c, V1, ws_bytes=16) == L.LISA_ERR_WORKSPACE
+    assert lib.lisa_append_cache_variant(ctypes.byref(c), V1, FAKE, FAKE, None, 5, None) == L.LISA_ERR_INVALID_ARG
+    assert lib.lisa_indexer_topk_variant(ctypes.byref(c), V1, FAKE, FAKE, 5, FAKE, FAKE, 16,
+                                         None) == L.LISA_ERR_WORKSPACE
+    assert lib.lisa_prefill_variant(ctypes.byref(c), V1, 101, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                                    FAKE, None, FAKE, 1 << 40, None) == L.LISA_ERR_INVALID_ARG
+    assert lib.lisa_prefill_variant(ctypes.byref(c), 0, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                                    FAKE, None, FAKE, 0, None) == L.LISA_OK
