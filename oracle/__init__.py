@@ -18,6 +18,10 @@ from .lisa_ref import (
     decode_step,
     prefill,
     indexer_kl,
+    PROJ_FIELDS,
+    proj_widths,
+    project_in,
+    project_out,
 )
 
 __all__ = [
@@ -33,4 +37,8 @@ __all__ = [
     "decode_step",
     "prefill",
     "indexer_kl",
+    "PROJ_FIELDS",
+    "proj_widths",
+    "project_in",
+    "project_out",
 ]

@@ -324,3 +324,54 @@ def indexer_kl(q, k, qidx, kidx, w, rows=None):
                 la = np.log(np.maximum(pa, 1e-300))
                 kl[b, t, h] = float(np.sum(pa * (la - lr)))
     return kl
+
+
+# --------------------------------------------------------------------------
+# projection front-end and output projection      [abs], [meth]
+# --------------------------------------------------------------------------
+# The abstract and the method details name the inputs of the layer -- the
+# attention's q, k, v, the indexer's small query / key projections, the
+# indexer head weights and the gate -- as projections of the hidden state,
+# and the layer's output goes back to the hidden size.  The pages give no
+# weights and no fused form; this library reads the front-end as ONE linear
+# map of the hidden state whose output columns are, in this order,
+#   q [Hq*d] | k [Hkv*d] | v [Hkv*d] | qidx [HI*dI] | kidx [P*dI] | w [HI] | lam [Hq]
+# (P = Hkv indexer-key planes by default), and the output projection as the
+# linear map o [Hq*d] -> y [Hm].  Weights are stored out-features x
+# in-features (row n of W holds the weights of output column n).
+PROJ_FIELDS = ("q", "k", "v", "qidx", "kidx", "w", "lam")
+
+
+def proj_widths(Hq, Hkv, d, HI, dI, P=None):
+    """Column count of every front-end field, in PROJ_FIELDS order."""
+    P = Hkv if P is None else P
+    return (Hq * d, Hkv * d, Hkv * d, HI * dI, P * dI, HI, Hq)
+
+
+def project_in(x, W_in, Hq, Hkv, d, HI, dI, P=None):
+    """Front-end: z = x W_in^T, split into the fields of the layer.
+
+    x [..., Hm]; W_in [N_in, Hm] with N_in = sum(proj_widths(...)).
+    Returns dict q [..., Hq, d], k, v [..., Hkv, d], qidx [..., HI, dI],
+    kidx [..., P, dI], w [..., HI], lam [..., Hq].
+
+    Parity: pinned by a brute-force triple loop on tiny inputs and by one-hot
+    weight rows that route a chosen hidden coordinate into every field."""
+    widths = proj_widths(Hq, Hkv, d, HI, dI, P)
+    assert W_in.shape[0] == sum(widths), "W_in rows must equal the total field width"
+    z = x @ W_in.T
+    out, c = {}, 0
+    shapes = {"q": (Hq, d), "k": (Hkv, d), "v": (Hkv, d), "qidx": (HI, dI),
+              "kidx": (Hkv if P is None else P, dI), "w": (HI,), "lam": (Hq,)}
+    for name, wd in zip(PROJ_FIELDS, widths):
+        out[name] = z[..., c:c + wd].reshape(z.shape[:-1] + shapes[name])
+        c += wd
+    return out
+
+
+def project_out(o, W_o):
+    """Output projection y = o W_o^T.  o [..., Hq, d]; W_o [Hm, Hq*d].
+
+    Parity: pinned by the brute-force loop and by W_o = identity (Hm = Hq*d)."""
+    flat = o.reshape(o.shape[:-2] + (o.shape[-2] * o.shape[-1],))
+    return flat @ W_o.T
