@@ -707,4 +707,65 @@ lisa_status lisa_prefill_variant(const lisa_layer *L, int variant, int T, const 
   return ok();
 }
 
+lisa_status lisa_project_in(const lisa_layer *L, int variant, const lisa_proj *proj, int T, const void *x, void *q,
+                            void *k, void *v, void *qidx, void *kidx, float *w, float *gate_logit, void *stream) {
+  lisa_status s;
+  VariantGeom vg;
+  if ((s = check_layer(L)) || (s = check_variant(L, variant, vg))) return s;
+  if (!proj) return fail(LISA_ERR_INVALID_ARG, "proj is NULL");
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (L->dtype != LISA_BF16) return fail(LISA_ERR_UNSUPPORTED, "projections support bf16 storage only");
+  if (proj->Hm < 8 || proj->Hm % 8) return fail(LISA_ERR_UNSUPPORTED, "Hm=%d is not a positive multiple of 8", proj->Hm);
+  if ((s = check_ptr(proj->W_in, "W_in")) || (s = check_ptr(x, "x")) || (s = check_ptr(q, "q")) ||
+      (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) || (s = check_ptr(qidx, "qidx")) ||
+      (s = check_ptr(kidx, "kidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(gate_logit, "gate_logit")))
+    return s;
+  lisa::ProjParams p;
+  memset(&p, 0, sizeof(p));
+  p.rows = L->B * T;
+  p.K = proj->Hm;
+  p.err_word = L->err_word;
+  const int widths[7] = {L->Hq * L->d, L->Hkv * L->d, L->Hkv * L->d, L->HI * L->dI, vg.P * L->dI, L->HI, L->Hq};
+  void *ptrs[7] = {q, k, v, qidx, kidx, w, gate_logit};
+  int c = 0;
+  for (int i = 0; i < 7; ++i) {
+    p.seg[i].c0 = c;
+    p.seg[i].width = widths[i];
+    p.seg[i].ptr = ptrs[i];
+    p.seg[i].f32 = i >= 5;
+    c += widths[i];
+  }
+  p.nseg = 7;
+  p.N = c;
+  cudaError_t e = lisa::launch_proj(p, x, proj->W_in, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "project_in");
+  return ok();
+}
+
+lisa_status lisa_project_out(const lisa_layer *L, const lisa_proj *proj, int T, const void *o, void *y, void *stream) {
+  lisa_status s;
+  if ((s = check_layer(L))) return s;
+  if (!proj) return fail(LISA_ERR_INVALID_ARG, "proj is NULL");
+  if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
+  if (T == 0 || L->B == 0) return ok();
+  if (L->dtype != LISA_BF16) return fail(LISA_ERR_UNSUPPORTED, "projections support bf16 storage only");
+  if (proj->Hm < 8 || proj->Hm % 8) return fail(LISA_ERR_UNSUPPORTED, "Hm=%d is not a positive multiple of 8", proj->Hm);
+  if ((s = check_ptr(proj->W_o, "W_o")) || (s = check_ptr(o, "o")) || (s = check_ptr(y, "y"))) return s;
+  lisa::ProjParams p;
+  memset(&p, 0, sizeof(p));
+  p.rows = L->B * T;
+  p.K = L->Hq * L->d;
+  p.N = proj->Hm;
+  p.err_word = L->err_word;
+  p.nseg = 1;
+  p.seg[0].c0 = 0;
+  p.seg[0].width = proj->Hm;
+  p.seg[0].ptr = y;
+  p.seg[0].f32 = 0;
+  cudaError_t e = lisa::launch_proj(p, o, proj->W_o, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "project_out");
+  return ok();
+}
+
 }  // extern "C"

@@ -113,4 +113,20 @@ cudaError_t launch_indexer_kl(const RowsParams &p, float *kl_out, cudaStream_t s
 // Sliding-window variant: idx of every row = its M most recent positions.
 cudaError_t launch_window_idx(const RowsParams &p, cudaStream_t st);
 
+// ------------------------------------------------------------- projections
+// Z[rows x N] = X[rows x K] W^T (bf16, W [N x K]); output column c belongs to
+// the segment with c0 <= c < c0 + width and goes to ptr[row * width + c - c0].
+struct ProjSeg {
+  int c0, width;
+  void *ptr;
+  int f32;                              // 1: fp32 output, 0: bf16
+};
+struct ProjParams {
+  int rows, N, K;
+  int nseg;
+  ProjSeg seg[8];
+  int *err_word;
+};
+cudaError_t launch_proj(const ProjParams &p, const void *x, const void *W, cudaStream_t st);
+
 }  // namespace lisa

@@ -48,6 +48,8 @@ EXPORTED = [
     "lisa_indexer_topk_variant",
     "lisa_decode_step_variant",
     "lisa_prefill_variant",
+    "lisa_project_in",
+    "lisa_project_out",
     "lisa_status_str",
     "lisa_last_error_msg",
     "lisa_version",
@@ -63,6 +65,10 @@ class LisaLayerC(ctypes.Structure):
         ("state", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("err_word", ctypes.c_void_p),
         ("decode_split", ctypes.c_int),
     ]
+
+
+class LisaProjC(ctypes.Structure):
+    _fields_ = [("Hm", ctypes.c_int), ("W_in", ctypes.c_void_p), ("W_o", ctypes.c_void_p)]
 
 
 class LisaError(RuntimeError):
@@ -106,6 +112,11 @@ def _load():
     lib.lisa_decode_step_variant.restype = I
     lib.lisa_prefill_variant.argtypes = [L, I, I, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.lisa_prefill_variant.restype = I
+    PJ = ctypes.POINTER(LisaProjC)
+    lib.lisa_project_in.argtypes = [L, I, PJ, I, P, P, P, P, P, P, P, P, P]
+    lib.lisa_project_in.restype = I
+    lib.lisa_project_out.argtypes = [L, PJ, I, P, P, P]
+    lib.lisa_project_out.restype = I
     lib.lisa_status_str.argtypes = [ctypes.c_int]
     lib.lisa_status_str.restype = ctypes.c_char_p
     lib.lisa_last_error_msg.argtypes = []
@@ -307,3 +318,33 @@ def lisa_prefill_variant(layer, variant, T, q, k, v, kidx, qidx, w, gate_logit, 
                                      _ptr(qidx), _ptr(w), _ptr(gate_logit), _ptr(k_lin), _ptr(v_lin), _ptr(out),
                                      _ptr(idx_out), _ptr(workspace),
                                      workspace.numel() if workspace is not None else 0, _stream(stream)))
+
+
+# ---------------------------------------------------------------- projections
+class Proj:
+    """Projection weights of one layer (a lisa_proj): W_in [N_in, Hm] and
+    W_o [Hm, Hq*d], bf16 CUDA tensors (out-features x in-features)."""
+
+    def __init__(self, Hm, W_in, W_o):
+        self.Hm, self.W_in, self.W_o = Hm, W_in, W_o
+
+    def c_struct(self):
+        return LisaProjC(int(self.Hm), _ptr(self.W_in), _ptr(self.W_o))
+
+
+def proj_widths(layer, variant=0):
+    """Column widths of the front-end fields q, k, v, qidx, kidx, w, gate_logit."""
+    P, _ = variant_planes(layer, variant)
+    return (layer.Hq * layer.d, layer.Hkv * layer.d, layer.Hkv * layer.d, layer.HI * layer.dI, P * layer.dI,
+            layer.HI, layer.Hq)
+
+
+def lisa_project_in(layer, variant, proj, T, x, q, k, v, qidx, kidx, w, gate_logit, stream=None):
+    c, pj = layer.c_struct(), proj.c_struct()
+    _check(_lib.lisa_project_in(ctypes.byref(c), int(variant), ctypes.byref(pj), int(T), _ptr(x), _ptr(q), _ptr(k),
+                                _ptr(v), _ptr(qidx), _ptr(kidx), _ptr(w), _ptr(gate_logit), _stream(stream)))
+
+
+def lisa_project_out(layer, proj, T, o, y, stream=None):
+    c, pj = layer.c_struct(), proj.c_struct()
+    _check(_lib.lisa_project_out(ctypes.byref(c), ctypes.byref(pj), int(T), _ptr(o), _ptr(y), _stream(stream)))

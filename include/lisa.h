@@ -303,6 +303,38 @@ LISA_API lisa_status lisa_prefill_variant(const lisa_layer *layer, int variant, 
                                           const void *v_lin, void *out, int *idx_out, void *workspace,
                                           size_t ws_bytes, void *stream);
 
+/*
+ * Projections on either side of the layer (abstract and gptget.net digest,
+ * method details: the attention's q, k, v, the indexer's query / key
+ * projections, its head weights and the gate are projections of the hidden
+ * state; the layer's output returns to the hidden size).  The pages give no
+ * fused form; this library reads the front-end as ONE linear map of the
+ * hidden state x [Hm] whose output columns are, in this order,
+ *   q [Hq*d] | k [Hkv*d] | v [Hkv*d] | qidx [HI*dI] | kidx [P*dI] | w [HI] | gate_logit [Hq]
+ * (P indexer-key planes as for the variants above; Hkv by default), and the
+ * output projection as y = o W_o^T.  Weights are stored out-features x
+ * in-features, bf16: W_in [N_in, Hm] with N_in the sum of the widths above,
+ * W_o [Hm, Hq*d].  Accumulation is fp32 on the tensor cores; w and gate_logit
+ * are written in fp32, everything else in bf16.  bf16 storage only
+ * (LISA_ERR_UNSUPPORTED otherwise); Hm a multiple of 8.
+ */
+typedef struct {
+  int Hm;              /* hidden size */
+  const void *W_in;    /* [N_in, Hm] bf16 */
+  const void *W_o;     /* [Hm, Hq * d] bf16 */
+} lisa_proj;
+
+/* Front-end for T tokens per sequence: x [B, T, Hm] -> q [B, T, Hq, d],
+ * k, v [B, T, Hkv, d], qidx [B, T, HI, dI], kidx [B, T, P, dI] (bf16),
+ * w [B, T, HI], gate_logit [B, T, Hq] (fp32): the inputs of lisa_prefill /
+ * lisa_decode_step (T = 1) and their _variant forms.  variant only sets P. */
+LISA_API lisa_status lisa_project_in(const lisa_layer *layer, int variant, const lisa_proj *proj, int T,
+                                     const void *x, void *q, void *k, void *v, void *qidx, void *kidx, float *w,
+                                     float *gate_logit, void *stream);
+/* Output projection for T tokens per sequence: o [B, T, Hq, d] -> y [B, T, Hm] (bf16). */
+LISA_API lisa_status lisa_project_out(const lisa_layer *layer, const lisa_proj *proj, int T, const void *o,
+                                      void *y, void *stream);
+
 /* Human-readable name of a status. */
 LISA_API const char *lisa_status_str(lisa_status s);
 

@@ -195,3 +195,21 @@ def test_variant_calls_validate():
                                     FAKE, None, FAKE, 1 << 40, None) == L.LISA_ERR_INVALID_ARG
     assert lib.lisa_prefill_variant(ctypes.byref(c), 0, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
                                     FAKE, None, FAKE, 0, None) == L.LISA_OK
+
+
+def test_projection_calls_validate():
+    lib = L.lib()
+    c = _layer()
+    pj = L.LisaProjC(1536, 0x30000, 0x30000)
+    args = [FAKE] * 8
+    assert lib.lisa_project_in(ctypes.byref(c), 0, None, 4, FAKE, *args[:7], None) == L.LISA_ERR_INVALID_ARG
+    assert lib.lisa_project_in(ctypes.byref(c), 0, ctypes.byref(pj), 4, FAKE, *args[:6], None,
+                               None) == L.LISA_ERR_INVALID_ARG
+    bad = L.LisaProjC(1537, 0x30000, 0x30000)
+    assert lib.lisa_project_in(ctypes.byref(c), 0, ctypes.byref(bad), 4, FAKE, *args[:7],
+                               None) == L.LISA_ERR_UNSUPPORTED
+    assert lib.lisa_project_out(ctypes.byref(_layer(dtype=L.LISA_FP32)), ctypes.byref(pj), 4, FAKE, FAKE,
+                                None) == L.LISA_ERR_UNSUPPORTED
+    assert lib.lisa_project_out(ctypes.byref(c), ctypes.byref(pj), 0, FAKE, FAKE, None) == L.LISA_OK
+    assert lib.lisa_project_in(ctypes.byref(c), 16, ctypes.byref(pj), 4, FAKE, *args[:7],
+                               None) == L.LISA_ERR_INVALID_ARG

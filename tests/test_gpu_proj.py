@@ -1,0 +1,106 @@
+"""GPU parity of the projection front-end and the output projection
+(tcgen05 GEMMs) against the fp64 oracle, through the C ABI.
+
+Tolerance, from the arithmetic: products of bf16 values are exact in fp32 and
+the tensor cores accumulate K of them in fp32, so the accumulation error is at
+most about K * 2^-24 * A with A = sum_k |x_k W_nk| (<= 1e-4 * A for the sizes
+here); bf16 outputs are then rounded once (<= 2^-9 relative).  The test allows
+|y - y*| <= 2^-8 |y*| + 1e-4 A for bf16 fields and 1e-4 A for the fp32 fields
+(w, gate_logit)."""
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lisa_inputs import get_config, make_rng
+from lisa_inputs.gen import round_to_dtype
+from harness import dev, f64
+
+pytestmark = pytest.mark.gpu
+
+L = pytest.importorskip("hybrid_linear_top_b200.lisa")
+
+HIDDEN = {"decode_1p5b_16k": 1536, "ragged_7b_b32": 3584}
+
+
+def _bf16(rng, shape, scale=1.0):
+    return round_to_dtype(rng.standard_normal(size=shape, dtype=np.float32) * np.float32(scale), "bf16")
+
+
+def _check(got, x, W, f32, where):
+    ref = x @ W.T
+    A = np.abs(x) @ np.abs(W).T
+    bound = 1e-4 * A + (0.0 if f32 else 2.0 ** -8 * np.abs(ref))
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), f"{where}: non-finite"
+    bad = err > bound
+    assert not bad.any(), f"{where}: {int(bad.sum())} elements out of bound, worst {float((err - bound).max()):.3g}"
+
+
+@pytest.mark.parametrize("cfg_name,B,T,variant", [
+    ("decode_1p5b_16k", 1, 1, 0),       # a decode step: narrow column tiles
+    ("decode_1p5b_16k", 1, 300, 0),     # several row tiles with a ragged tail
+    ("decode_1p5b_16k", 3, 50, 1),      # one indexer key per indexer head (4 planes)
+    ("decode_1p5b_16k", 16, 1, 1),      # 16 decode tokens: the weight-streaming path at its row limit
+    ("decode_1p5b_16k", 17, 1, 0),      # 17 rows: the tensor-core path
+    ("decode_1p5b_16k", 5, 1, 2),       # 5 rows: weights as the M operand, one shared key plane
+    ("decode_1p5b_16k", 2, 1, 0),       # 2 rows: the weight-streaming CUDA-core path
+    ("ragged_7b_b32", 12, 1, 0),        # 7B shape, 12 rows: K split over a cluster of 3
+    ("ragged_7b_b32", 8, 1, 0),         # 7B shape, batch of 8 decode tokens
+    ("ragged_7b_b32", 1, 260, 2),       # 7B shape, one shared key plane
+])
+def test_project_in(cfg_name, B, T, variant):
+    cfg = dataclasses.replace(get_config(cfg_name), B=B)
+    Hm = HIDDEN[cfg_name]
+    lay = L.Layer.allocate(B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, 16)
+    widths = L.proj_widths(lay, variant)
+    P = widths[4] // cfg.dI
+    rng = make_rng(400 + T, 0)
+    x = _bf16(rng, (B, T, Hm))
+    W = _bf16(rng, (sum(widths), Hm), 1.0 / np.sqrt(Hm))
+    proj = L.Proj(Hm, dev(W, "bf16"), None)
+    bf = torch.bfloat16
+    outs = dict(q=torch.empty(B, T, cfg.Hq, cfg.d, dtype=bf, device="cuda"),
+                k=torch.empty(B, T, cfg.Hkv, cfg.d, dtype=bf, device="cuda"),
+                v=torch.empty(B, T, cfg.Hkv, cfg.d, dtype=bf, device="cuda"),
+                qidx=torch.empty(B, T, cfg.HI, cfg.dI, dtype=bf, device="cuda"),
+                kidx=torch.empty(B, T, P, cfg.dI, dtype=bf, device="cuda"),
+                w=torch.empty(B, T, cfg.HI, dtype=torch.float32, device="cuda"),
+                lam=torch.empty(B, T, cfg.Hq, dtype=torch.float32, device="cuda"))
+    for t in outs.values():
+        t.fill_(float("nan"))
+    L.lisa_project_in(lay, variant, proj, T, dev(x, "bf16"), outs["q"], outs["k"], outs["v"], outs["qidx"],
+                      outs["kidx"], outs["w"], outs["lam"])
+    torch.cuda.synchronize()
+    assert int(lay.err_word.item()) == 0
+    a = lambda z: z.astype(np.float64)
+    ref = oracle.project_in(a(x), a(W), cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, P)
+    c = 0
+    xf = a(x).reshape(B * T, Hm)
+    for name, wd in zip(oracle.PROJ_FIELDS, widths):
+        got = f64(outs[name]).reshape(B * T, wd)
+        assert ref[name].reshape(B * T, wd).shape == got.shape
+        _check(got, xf, a(W)[c:c + wd], name in ("w", "lam"), name)
+        c += wd
+
+
+@pytest.mark.parametrize("cfg_name,B,T", [("decode_1p5b_16k", 1, 1), ("decode_1p5b_16k", 2, 300),
+                                          ("ragged_7b_b32", 32, 1)])
+def test_project_out(cfg_name, B, T):
+    cfg = dataclasses.replace(get_config(cfg_name), B=B)
+    Hm = HIDDEN[cfg_name]
+    lay = L.Layer.allocate(B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, 16)
+    rng = make_rng(500 + T, 0)
+    o = _bf16(rng, (B, T, cfg.Hq, cfg.d), 1.0 / np.sqrt(cfg.d))
+    Wo = _bf16(rng, (Hm, cfg.Hq * cfg.d), 1.0 / np.sqrt(cfg.Hq * cfg.d))
+    proj = L.Proj(Hm, None, dev(Wo, "bf16"))
+    y = torch.full((B, T, Hm), float("nan"), dtype=torch.bfloat16, device="cuda")
+    L.lisa_project_out(lay, proj, T, dev(o, "bf16"), y)
+    torch.cuda.synchronize()
+    a = lambda z: z.astype(np.float64)
+    ref = oracle.project_out(a(o), a(Wo))
+    assert ref.shape == (B, T, Hm)
+    _check(f64(y).reshape(B * T, Hm), a(o).reshape(B * T, -1), a(Wo), False, "y")
