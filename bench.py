@@ -46,7 +46,7 @@ WORKLOAD = "decode_1p5b_16k"
 # DRAM bytes (read + write) of one decode launch from an ncu capture of this
 # kernel on this workload, by CTA split (the ncu summary under profiles/);
 # None where no capture of the current kernel exists.
-DECODE_TRAFFIC = {4: None, 8: None, 16: None, 0: None}
+DECODE_TRAFFIC = {4: 5391872, 8: None, 16: None, 0: None}
 
 
 def algorithmic_bytes(cfg, L, esize=2):
@@ -591,6 +591,79 @@ def run_kl(args, rank, world):
            "algorithmic_flops_per_call": flops, "traffic": None})
 
 
+def run_proj(args, rank, world):
+    """Projections on either side of the layer at the 1.5B shape (hidden size
+    1536): the front-end x -> q, k, v, qidx, kidx, w, gate logits and the
+    output projection o -> y, for a 16384-token prefill (tcgen05 GEMMs; the
+    headline) and for one decode token (weight streams, reported beside it,
+    rotating over weight copies larger than L2)."""
+    import torch
+    from hybrid_linear_top_b200 import lisa as L
+    cfg = get_config("prefill_1p5b_16k")
+    Hm = 1536
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 * rank + 11)
+    bf = torch.bfloat16
+
+    def setup(B, T, copies):
+        lay = L.Layer.allocate(B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, 16, L.LISA_BF16)
+        N = sum(L.proj_widths(lay))
+        projs = [L.Proj(Hm, (torch.randn((N, Hm), generator=g, device="cuda") / Hm ** 0.5).to(bf),
+                        (torch.randn((Hm, cfg.Hq * cfg.d), generator=g, device="cuda") / (cfg.Hq * cfg.d) ** 0.5).to(bf))
+                 for _ in range(copies)]
+        x = torch.randn((B, T, Hm), generator=g, device="cuda").to(bf)
+        o = {"q": torch.empty(B, T, cfg.Hq, cfg.d, dtype=bf, device="cuda"),
+             "k": torch.empty(B, T, cfg.Hkv, cfg.d, dtype=bf, device="cuda"),
+             "v": torch.empty(B, T, cfg.Hkv, cfg.d, dtype=bf, device="cuda"),
+             "qidx": torch.empty(B, T, cfg.HI, cfg.dI, dtype=bf, device="cuda"),
+             "kidx": torch.empty(B, T, cfg.Hkv, cfg.dI, dtype=bf, device="cuda"),
+             "w": torch.empty(B, T, cfg.HI, device="cuda"), "lam": torch.empty(B, T, cfg.Hq, device="cuda"),
+             "y": torch.empty(B, T, Hm, dtype=bf, device="cuda")}
+
+        def step(i, s_):
+            pj = projs[i % copies]
+            L.lisa_project_in(lay, 0, pj, T, x, o["q"], o["k"], o["v"], o["qidx"], o["kidx"], o["w"], o["lam"], s_)
+            L.lisa_project_out(lay, pj, T, o["q"], o["y"], s_)
+        return lay, N, step
+
+    stream = torch.cuda.Stream()
+    # prefill-size: T = 16384 rows (inputs and outputs far larger than L2)
+    T = cfg.T
+    lay, N, step = setup(1, T, 1)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, stream)
+    gr = _capture(torch, stream, [stream], list(range(args.steps)), step)
+    ms = max_over_ranks(_timed_replays(torch, stream, [gr]), world, "cuda") / args.steps
+    flops = 2 * T * Hm * N + 2 * T * cfg.Hq * cfg.d * Hm
+    tf = flops / (ms * 1e-3) / 1e12
+    # decode-size: one token, rotating over weight copies that exceed 4x L2
+    wbytes = 2 * (N * Hm + Hm * cfg.Hq * cfg.d)
+    copies = int(4 * 126 * 2 ** 20 // wbytes) + 1
+    lay1, _, step1 = setup(1, 1, copies)
+    n1 = 20 * copies
+    g1 = _capture(torch, stream, [stream], list(range(n1)), step1)
+    g1.replay()
+    ms1 = max_over_ranks(_timed_replays(torch, stream, [g1]), world, "cuda") / n1
+    if int(lay.err_word.item()) or int(lay1.err_word.item()):
+        raise RuntimeError("a projection flagged an error")
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    hbm, hbm_kind = load_peaks()
+    dec_gbs = (wbytes + 2 * (Hm + N + cfg.Hq * cfg.d + Hm)) / (ms1 * 1e-3) / 1e9
+    _line(rank, "LISA projection front-end + output projection tokens/s @16K-token prefill",
+          replica_rate(T, ms, world), "tokens/s", args, world, ms,
+          {"workload": "proj_1p5b_16k", "T": T, "Hm": Hm, "N_in": N, "parallelism": f"replicas x{world}"},
+          {"bound": "tensor", "kernel": "proj_tc_kernel<256> (tcgen05), front-end + output projection",
+           "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+           "peak_kind": "measured" if peaks else "fallback", "algorithmic_flops_per_step": flops, "traffic": None},
+          {"decode_token": {"us_per_token": ms1 * 1e3, "achieved_gbs": dec_gbs, "peak_gbs": hbm,
+                            "frac": dec_gbs / hbm, "peak_kind": hbm_kind, "weight_copies": copies,
+                            "kernels": "proj_gemv_kernel (TMA weight stream), both projections"}})
+
+
 def run_window(args, rank, world):
     """Stage-1 sliding-window variant at the 1.5B decode shape: the last 256
     positions instead of the indexer's top-256 (lisa_decode_step_window),
@@ -751,7 +824,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l", "window_1p5b_16k", "kl_1p5b_16k"])
+                    choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l", "window_1p5b_16k", "kl_1p5b_16k",
+                             "proj_1p5b_16k"])
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--streams", type=int, default=32)
     ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16])
@@ -761,7 +835,8 @@ def main():
     args.warmup = max(3, args.warmup)
     if args.steps is None:
         args.steps = {WORKLOAD: 200000, "prefill_1p5b_16k": 20, "ragged_7b_b32": 2000,
-                      "longcot_7b_28l": 1024, "window_1p5b_16k": 200000, "kl_1p5b_16k": 5}[args.workload]
+                      "longcot_7b_28l": 1024, "window_1p5b_16k": 200000, "kl_1p5b_16k": 5,
+                      "proj_1p5b_16k": 50}[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if world > 1:
@@ -783,6 +858,8 @@ def main():
             run_window(args, rank, world)
         elif args.workload == "kl_1p5b_16k":
             run_kl(args, rank, world)
+        elif args.workload == "proj_1p5b_16k":
+            run_proj(args, rank, world)
         else:
             run_lisa(args, rank, world)
     finally:
