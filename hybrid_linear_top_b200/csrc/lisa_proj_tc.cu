@@ -9,12 +9,14 @@
 // output columns are [q | k | v | qidx | kidx | w | lambda] (lisa.h).
 //
 // Z[rows x N] = X[rows x K] W^T with X and W (N x K, out-features x
-// in-features) bf16 and K-major, fp32 accumulation in tensor memory.  A CTA
-// owns 128 rows x BN columns: warp 0 lane 0 loads 64-wide K blocks of X and W
-// through a TMA ring (128-byte swizzle), warp 1 lane 0 issues the MMAs
-// (M = 128, N = BN, K = 16 per instruction) and owns the TMEM columns, and
-// warps 4-7 (one TMEM lane quadrant each, one row per thread) write the
-// accumulator to the column segments' own dense arrays (bf16 or fp32).
+// in-features) bf16 and K-major, fp32 accumulation in tensor memory.  Tiles
+// of 128 rows x BN columns; one persistent CTA per SM walks its share of
+// them: warp 0 lane 0 loads 64-wide K blocks of X and W through a TMA ring
+// (128-byte swizzle), warp 1 lane 0 issues the MMAs (M = 128, N = BN, K = 16
+// per instruction) into one of two TMEM accumulator buffers and owns the TMEM
+// columns, and warps 4-7 (one TMEM lane quadrant each, one row per thread)
+// write a finished tile to the column segments' own dense arrays (bf16 or
+// fp32) while the MMAs of the next tile fill the other buffer.
 // BN = 256 for many rows (the contraction is tensor-bound); BN = 32 for up to
 // 128 rows (narrow column tiles put more SMs on the weight stream).  Up to 16
 // rows (a decode step) go to a CUDA-core weight-streaming kernel instead: that
@@ -64,22 +66,27 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * PG::kStageBytes);
-  uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 1);
+  uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S, *acc_empty = bars + 2 * S + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int col0 = blockIdx.x * BN, row0 = blockIdx.y * kProjRows;
+  const int ntn = (p.N + BN - 1) / BN;
+  const int ntiles = ntn * ((p.rows + kProjRows - 1) / kProjRows);
   const int nk = (p.K + kProjKB - 1) / kProjKB;
+  constexpr uint32_t kCols = 2 * BN;               // two accumulator buffers
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4 * 32);            // every epilogue thread has read the buffer
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
-    tc_alloc(tmem_slot, BN);
+    tc_alloc(tmem_slot, kCols);
     tc_relinquish();
   }
   tc_fence_before();
@@ -87,79 +94,99 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Persistent: CTA c takes tiles c, c + gridDim.x, ...; tile = (row block, column block).
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % S;
-        if (kb >= S && !mbar_wait_bounded(&empty[st], (uint32_t)(((kb / S) - 1) & 1)))
-          set_err(p.err_word, LISA_DEVERR_TIMEOUT);
-        unsigned char *a = smem + st * PG::kStageBytes;
-        mbar_arrive_expect_tx(&full[st], (uint32_t)PG::kStageBytes);   // whole boxes land, out of range zero
-        tma_load_2d(a, &xmap, kb * kProjKB, row0, &full[st]);
-        tma_load_2d(a + PG::kABytes, &wmap, kb * kProjKB, col0, &full[st]);
+      int it = 0;                                   // K blocks issued so far (ring position)
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int row0 = (tile / ntn) * kProjRows, col0 = (tile % ntn) * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int st = it % S;
+          if (it >= S && !mbar_wait_bounded(&empty[st], (uint32_t)(((it / S) - 1) & 1)))
+            set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+          unsigned char *a = smem + st * PG::kStageBytes;
+          mbar_arrive_expect_tx(&full[st], (uint32_t)PG::kStageBytes);   // whole boxes land, out of range zero
+          tma_load_2d(a, &xmap, kb * kProjKB, row0, &full[st]);
+          tma_load_2d(a + PG::kABytes, &wmap, kb * kProjKB, col0, &full[st]);
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = tc_idesc_bf16(kProjRows, BN);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int st = kb % S;
-        if (!mbar_wait_bounded(&full[st], (uint32_t)((kb / S) & 1))) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+      int it = 0, lt = 0;                           // K blocks consumed, tiles done by this CTA
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        if (lt >= 2 && !mbar_wait_bounded(&acc_empty[buf], (uint32_t)(((lt >> 1) - 1) & 1)))
+          set_err(p.err_word, LISA_DEVERR_TIMEOUT);
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + st * PG::kStageBytes);
-        const uint64_t adesc = tc_sdesc_kmajor(a, 128), bdesc = tc_sdesc_kmajor(a + PG::kABytes, 128);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int st = it % S;
+          if (!mbar_wait_bounded(&full[st], (uint32_t)((it / S) & 1))) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + st * PG::kStageBytes);
+          const uint64_t adesc = tc_sdesc_kmajor(a, 128), bdesc = tc_sdesc_kmajor(a + PG::kABytes, 128);
 #pragma unroll
-        for (int ks = 0; ks < kProjKB / 16; ++ks)   // +32 bytes along K inside the swizzle atom
-          tc_mma_bf16(tmem, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kb | ks) != 0);
-        tc_commit(&empty[st]);                      // the stage may be refilled once these MMAs are done
+          for (int ks = 0; ks < kProjKB / 16; ++ks)   // +32 bytes along K inside the swizzle atom
+            tc_mma_bf16(tmem + (uint32_t)(buf * BN), adesc + 2 * ks, bdesc + 2 * ks, idesc, (kb | ks) != 0);
+          tc_commit(&empty[st]);                    // the stage may be refilled once these MMAs are done
+        }
+        tc_commit(&acc_full[buf]);                  // this tile's accumulator is complete
       }
-      tc_commit(acc_full);                          // the accumulator is complete
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue: thread = row
+    // overlaps the MMAs of the next tile, which go to the other buffer
     const int quad = warp - 4;
-    const int row = row0 + quad * 32 + lane;
-    if (!mbar_wait_bounded(acc_full, 0) && lane == 0) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
-    __syncwarp();
-    tc_fence_after();
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      const int row = (tile / ntn) * kProjRows + quad * 32 + lane, col0 = (tile % ntn) * BN;
+      if (!mbar_wait_bounded(&acc_full[buf], (uint32_t)((lt >> 1) & 1)) && lane == 0)
+        set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+      __syncwarp();
+      tc_fence_after();
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      uint32_t v[16];
-      tc_ld16(tmem + lane_base + (uint32_t)c, v);
-      tc_wait_ld();
-      const int gc = col0 + c;
-      if (row >= p.rows || gc >= p.N) continue;
-      // the 16 columns inside one bf16 segment, 16-column aligned in it: two 16-byte stores
-      int s = 0;
-      while (s < p.nseg && !(gc >= p.seg[s].c0 && gc < p.seg[s].c0 + p.seg[s].width)) ++s;
-      const bool vec = s < p.nseg && !p.seg[s].f32 && gc + 16 <= p.seg[s].c0 + p.seg[s].width &&
-                       ((gc - p.seg[s].c0) & 15) == 0 && (p.seg[s].width & 7) == 0;
-      if (vec) {
-        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.seg[s].ptr) +
-                                               (size_t)row * p.seg[s].width + (gc - p.seg[s].c0));
-        dst[0] = make_uint4(pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
-                            pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
-                            pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
-                            pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
-        dst[1] = make_uint4(pack_bf16(__uint_as_float(v[8]), __uint_as_float(v[9])),
-                            pack_bf16(__uint_as_float(v[10]), __uint_as_float(v[11])),
-                            pack_bf16(__uint_as_float(v[12]), __uint_as_float(v[13])),
-                            pack_bf16(__uint_as_float(v[14]), __uint_as_float(v[15])));
-      } else {
+      for (int c = 0; c < BN; c += 16) {
+        uint32_t v[16];
+        tc_ld16(tmem + lane_base + (uint32_t)(buf * BN + c), v);
+        tc_wait_ld();
+        const int gc = col0 + c;
+        if (row >= p.rows || gc >= p.N) continue;
+        // the 16 columns inside one bf16 segment, 16-column aligned in it: two 16-byte stores
+        int s = 0;
+        while (s < p.nseg && !(gc >= p.seg[s].c0 && gc < p.seg[s].c0 + p.seg[s].width)) ++s;
+        const bool vec = s < p.nseg && !p.seg[s].f32 && gc + 16 <= p.seg[s].c0 + p.seg[s].width &&
+                         ((gc - p.seg[s].c0) & 15) == 0 && (p.seg[s].width & 7) == 0;
+        if (vec) {
+          uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.seg[s].ptr) +
+                                                 (size_t)row * p.seg[s].width + (gc - p.seg[s].c0));
+          dst[0] = make_uint4(pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                              pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                              pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                              pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+          dst[1] = make_uint4(pack_bf16(__uint_as_float(v[8]), __uint_as_float(v[9])),
+                              pack_bf16(__uint_as_float(v[10]), __uint_as_float(v[11])),
+                              pack_bf16(__uint_as_float(v[12]), __uint_as_float(v[13])),
+                              pack_bf16(__uint_as_float(v[14]), __uint_as_float(v[15])));
+        } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (gc + j < p.N) proj_store(p, row, gc + j, __uint_as_float(v[j]));
+          for (int j = 0; j < 16; ++j)
+            if (gc + j < p.N) proj_store(p, row, gc + j, __uint_as_float(v[j]));
+        }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);                 // the MMAs of tile lt + 2 may overwrite the buffer
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tc_dealloc(tmem, BN);
+    tc_dealloc(tmem, kCols);
   }
 }
 
@@ -174,8 +201,14 @@ static cudaError_t proj_t(const ProjParams &p, const void *x, const void *W, cud
       !make_tmap_2d(&wmap, W, 2, (unsigned long long)p.K, (unsigned long long)p.N, (unsigned long long)p.K * 2,
                     kProjKB, BN, 128))
     return cudaErrorInvalidValue;
-  dim3 grid((p.N + BN - 1) / BN, (p.rows + kProjRows - 1) / kProjRows);
-  proj_tc_kernel<BN><<<grid, kProjThreads, PG::kSmem, st>>>(p, xmap, wmap);
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  const int ntiles = ((p.N + BN - 1) / BN) * ((p.rows + kProjRows - 1) / kProjRows);
+  proj_tc_kernel<BN><<<std::min(ntiles, sms), kProjThreads, PG::kSmem, st>>>(p, xmap, wmap);   // persistent
   return cudaGetLastError();
 }
 
@@ -308,36 +341,36 @@ static cudaError_t proj_gemv_t(const ProjParams &p, const void *x, const void *W
 }
 
 // ============================================================ few rows on the tensor cores
-// Up to 16 rows with a wide K: the weights are the M = 128 operand and the
-// rows of X the N = 16 operand (Z^T = W X^T), so every byte a stage brings in
-// is a weight byte the step needs.  A cluster of CS CTAs owns 128 output
+// Up to 32 rows with a wide K: the weights are the M = 128 operand and the
+// rows of X the N = 16 or 32 operand (Z^T = W X^T), so nearly every byte a
+// stage brings in is a weight byte the step needs.  A cluster of CS CTAs owns 128 output
 // columns; CTA r streams the weight rows' K range r through a deep TMA ring.
 // CS (up to 4) is chosen so that the clusters fill the SMs in one wave.  TMEM lane = output column, TMEM
 // column = row of X.  Ranks 1.. store their partial sums into rank 0's shared
 // memory (distributed shared memory); after one cluster barrier rank 0 adds
 // them and writes each column for every row (32 lanes = 32 consecutive
 // columns: coalesced per row).
-constexpr int kSwapRows = 16;      // MMA N: rows of X per CTA (padded)
+constexpr int kSwapRowsMax = 32;   // rows handled by this path at most
 constexpr int kSwapStages = 8;
 constexpr int kSwapABytes = kProjRows * kProjKB * 2;      // 128 weight rows x 64 K
-constexpr int kSwapBBytes = kSwapRows * kProjKB * 2;      // 16 rows of X x 64 K
-constexpr int kSwapStageBytes = kSwapABytes + kSwapBBytes;
-// shared memory: ring, barriers, and the partials of ranks 1..CS-1 ([CS-1][128][16] fp32)
-__host__ __device__ constexpr int swap_smem(int CS) {
-  return 1024 + kSwapStages * kSwapStageBytes + 256 + (CS - 1) * kProjRows * kSwapRows * 4;
+// per stage: the weight tile and SR rows of X (SR = MMA N: 16 or 32, rows padded)
+__host__ __device__ constexpr int swap_stage_bytes(int SR) { return kSwapABytes + SR * kProjKB * 2; }
+// shared memory: ring, barriers, and the partials of ranks 1..CS-1 ([CS-1][128][SR] fp32)
+__host__ __device__ constexpr int swap_smem(int CS, int SR) {
+  return 1024 + kSwapStages * swap_stage_bytes(SR) + 256 + (CS - 1) * kProjRows * SR * 4;
 }
 
-template <int CS>
+template <int CS, int SR>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_swap_tc_kernel(const __grid_constant__ ProjParams p, const __grid_constant__ CUtensorMap wmap,
                         const __grid_constant__ CUtensorMap xmap) {
   constexpr int S = kSwapStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * kSwapStageBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * swap_stage_bytes(SR));
   uint64_t *full = bars, *empty = bars + S, *acc_full = bars + 2 * S;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 1);
-  float *red = reinterpret_cast<float *>(smem + S * kSwapStageBytes + 256);   // [CS-1][128][16]
+  float *red = reinterpret_cast<float *>(smem + S * swap_stage_bytes(SR) + 256);   // [CS-1][128][SR]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
@@ -355,7 +388,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tc_alloc(tmem_slot, 32);
+    tc_alloc(tmem_slot, SR < 32 ? 32 : SR);   // at least 32 columns
     tc_relinquish();
   }
   tc_fence_before();
@@ -369,20 +402,20 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const int st = kb % S;
         if (kb >= S && !mbar_wait_bounded(&empty[st], (uint32_t)(((kb / S) - 1) & 1)))
           set_err(p.err_word, LISA_DEVERR_TIMEOUT);
-        unsigned char *a = smem + st * kSwapStageBytes;
-        mbar_arrive_expect_tx(&full[st], (uint32_t)kSwapStageBytes);   // whole boxes, out of range zero
+        unsigned char *a = smem + st * swap_stage_bytes(SR);
+        mbar_arrive_expect_tx(&full[st], (uint32_t)swap_stage_bytes(SR));   // whole boxes, out of range zero
         tma_load_2d(a, &wmap, (kb0 + kb) * kProjKB, col0, &full[st]);
         tma_load_2d(a + kSwapABytes, &xmap, (kb0 + kb) * kProjKB, 0, &full[st]);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = tc_idesc_bf16(kProjRows, kSwapRows);
+      const uint32_t idesc = tc_idesc_bf16(kProjRows, SR);
       for (int kb = 0; kb < nk; ++kb) {
         const int st = kb % S;
         if (!mbar_wait_bounded(&full[st], (uint32_t)((kb / S) & 1))) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + st * kSwapStageBytes);
+        const uint32_t a = smem_u32(smem + st * swap_stage_bytes(SR));
         const uint64_t adesc = tc_sdesc_kmajor(a, 128), bdesc = tc_sdesc_kmajor(a + kSwapABytes, 128);
 #pragma unroll
         for (int ks = 0; ks < kProjKB / 16; ++ks)
@@ -393,26 +426,29 @@ __global__ void __launch_bounds__(kProjThreads, 1)
       else mbar_arrive(acc_full);                   // no K range for this rank: nothing was issued
     }
   }
-  float part[kSwapRows];
+  float part[SR];
 #pragma unroll
-  for (int r = 0; r < kSwapRows; ++r) part[r] = 0.f;
+  for (int r = 0; r < SR; ++r) part[r] = 0.f;
   const int quad = warp - 4, cl = quad * 32 + lane;   // epilogue: local output column of this thread
   if (warp >= 4) {
     if (!mbar_wait_bounded(acc_full, 0) && lane == 0) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
     __syncwarp();
     tc_fence_after();
     if (nk > 0) {
-      uint32_t v[16];
-      tc_ld16(tmem + ((uint32_t)(quad * 32) << 16), v);
-      tc_wait_ld();
 #pragma unroll
-      for (int r = 0; r < kSwapRows; ++r) part[r] = __uint_as_float(v[r]);
+      for (int c = 0; c < SR; c += 16) {
+        uint32_t v[16];
+        tc_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c, v);
+        tc_wait_ld();
+#pragma unroll
+        for (int r = 0; r < 16; ++r) part[c + r] = __uint_as_float(v[r]);
+      }
     }
     if (rank > 0) {                                 // partial sums into rank 0
       float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(red, 0) +
-                                               ((size_t)(rank - 1) * kProjRows + cl) * kSwapRows);
+                                               ((size_t)(rank - 1) * kProjRows + cl) * SR);
 #pragma unroll
-      for (int q4 = 0; q4 < kSwapRows / 4; ++q4)
+      for (int q4 = 0; q4 < SR / 4; ++q4)
         dst[q4] = make_float4(part[4 * q4], part[4 * q4 + 1], part[4 * q4 + 2], part[4 * q4 + 3]);
     }
   }
@@ -420,9 +456,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   if (warp >= 4 && rank == 0) {
     const int n = col0 + cl;
     for (int j = 1; j < CS; ++j) {
-      const float4 *src = reinterpret_cast<const float4 *>(red + ((size_t)(j - 1) * kProjRows + cl) * kSwapRows);
+      const float4 *src = reinterpret_cast<const float4 *>(red + ((size_t)(j - 1) * kProjRows + cl) * SR);
 #pragma unroll
-      for (int q4 = 0; q4 < kSwapRows / 4; ++q4) {
+      for (int q4 = 0; q4 < SR / 4; ++q4) {
         const float4 a = src[q4];
         part[4 * q4] += a.x;
         part[4 * q4 + 1] += a.y;
@@ -432,26 +468,26 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
     if (n < p.N)
 #pragma unroll
-      for (int r = 0; r < kSwapRows; ++r)
+      for (int r = 0; r < SR; ++r)
         if (r < p.rows) proj_store(p, r, n, part[r]);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tc_dealloc(tmem, 32);
+    tc_dealloc(tmem, SR < 32 ? 32 : SR);
   }
 }
 
-template <int CS>
+template <int CS, int SR>
 static cudaError_t proj_swap_t(const ProjParams &p, const void *x, const void *W, cudaStream_t st) {
-  cudaError_t e = prepare_kernel(proj_swap_tc_kernel<CS>, swap_smem(CS));
+  cudaError_t e = prepare_kernel(proj_swap_tc_kernel<CS, SR>, swap_smem(CS, SR));
   if (e != cudaSuccess) return e;
   CUtensorMap wmap, xmap;
   if (!make_tmap_2d(&wmap, W, 2, (unsigned long long)p.K, (unsigned long long)p.N, (unsigned long long)p.K * 2,
                     kProjKB, kProjRows, 128) ||
       !make_tmap_2d(&xmap, x, 2, (unsigned long long)p.K, (unsigned long long)p.rows, (unsigned long long)p.K * 2,
-                    kProjKB, kSwapRows, 128))
+                    kProjKB, SR, 128))
     return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -461,16 +497,16 @@ static cudaError_t proj_swap_t(const ProjParams &p, const void *x, const void *W
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(((p.N + kProjRows - 1) / kProjRows) * CS);
   cfg.blockDim = dim3(kProjThreads);
-  cfg.dynamicSmemBytes = swap_smem(CS);
+  cfg.dynamicSmemBytes = swap_smem(CS, SR);
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, proj_swap_tc_kernel<CS>, p, wmap, xmap);
+  return cudaLaunchKernelEx(&cfg, proj_swap_tc_kernel<CS, SR>, p, wmap, xmap);
 }
 
 cudaError_t launch_proj(const ProjParams &p, const void *x, const void *W, cudaStream_t st) {
   if (p.rows <= 0 || p.N <= 0) return cudaSuccess;
-  if (p.rows > 2 && p.rows <= kSwapRows) {
+  if (p.rows > 2 && p.rows <= kSwapRowsMax) {
     // K split over a cluster of CS CTAs: as many as still fit the SMs in one wave
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
@@ -481,11 +517,19 @@ cudaError_t launch_proj(const ProjParams &p, const void *x, const void *W, cudaS
     const int tiles = (p.N + kProjRows - 1) / kProjRows;
     // (larger clusters measured slower: they fit the GPCs less evenly)
     const int cs = std::max(1, std::min(4, sms / tiles));
+    if (p.rows <= 16) {
+      switch (cs) {
+        case 1: return proj_swap_t<1, 16>(p, x, W, st);
+        case 2: return proj_swap_t<2, 16>(p, x, W, st);
+        case 3: return proj_swap_t<3, 16>(p, x, W, st);
+        default: return proj_swap_t<4, 16>(p, x, W, st);
+      }
+    }
     switch (cs) {
-      case 1: return proj_swap_t<1>(p, x, W, st);
-      case 2: return proj_swap_t<2>(p, x, W, st);
-      case 3: return proj_swap_t<3>(p, x, W, st);
-      default: return proj_swap_t<4>(p, x, W, st);
+      case 1: return proj_swap_t<1, 32>(p, x, W, st);
+      case 2: return proj_swap_t<2, 32>(p, x, W, st);
+      case 3: return proj_swap_t<3, 32>(p, x, W, st);
+      default: return proj_swap_t<4, 32>(p, x, W, st);
     }
   }
   if (p.rows <= kGemvRowsMax && gemv_smem_bytes<32>(p.rows, p.K) <= 227 * 1024) {

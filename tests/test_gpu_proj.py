@@ -49,6 +49,7 @@ def _check(got, x, W, f32, where):
     ("decode_1p5b_16k", 5, 1, 2),       # 5 rows: weights as the M operand, one shared key plane
     ("decode_1p5b_16k", 2, 1, 0),       # 2 rows: the weight-streaming CUDA-core path
     ("ragged_7b_b32", 12, 1, 0),        # 7B shape, 12 rows: K split over a cluster of 3
+    ("ragged_7b_b32", 32, 1, 1),        # 7B shape, 32 rows: weights as the M operand with N = 32
     ("ragged_7b_b32", 8, 1, 0),         # 7B shape, batch of 8 decode tokens
     ("ragged_7b_b32", 1, 260, 2),       # 7B shape, one shared key plane
 ])
