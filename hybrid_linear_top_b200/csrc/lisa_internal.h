@@ -110,6 +110,9 @@ cudaError_t launch_lin_state(const RowsParams &p, cudaStream_t st);
 cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t st);
 // Stage-2 objective (forward): per-head KL of teacher attention vs indexer, kl_out [B, T, Hq].
 cudaError_t launch_indexer_kl(const RowsParams &p, float *kl_out, cudaStream_t st);
+// Its tensor-core (tcgen05) form, for d = 128 and at most 4 indexer heads per KV head.
+bool indexer_kl_tc_supported(const RowsParams &p);
+cudaError_t launch_indexer_kl_tc(const RowsParams &p, float *kl_out, cudaStream_t st);
 // Sliding-window variant: idx of every row = its M most recent positions.
 cudaError_t launch_window_idx(const RowsParams &p, cudaStream_t st);
 

@@ -275,6 +275,7 @@ static cudaError_t kl_t(const RowsParams &p, float *kl_out, cudaStream_t st) {
 }
 
 cudaError_t launch_indexer_kl(const RowsParams &p, float *kl_out, cudaStream_t st) {
+  if (indexer_kl_tc_supported(p)) return launch_indexer_kl_tc(p, kl_out, st);   // tcgen05 (lisa_kl_tc.cu)
   if (p.D == 128 && p.DI == 64) return kl_t<128, 64>(p, kl_out, st);
   if (p.D == 128 && p.DI == 32) return kl_t<128, 32>(p, kl_out, st);
   if (p.D == 64 && p.DI == 64) return kl_t<64, 64>(p, kl_out, st);

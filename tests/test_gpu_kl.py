@@ -47,10 +47,17 @@ def test_kl_1p5b_shape(T):
     run_kl(cfg, T, seed=T)
 
 
-@pytest.mark.parametrize("d,dI,HI,Hq", [(64, 32, 2, 8), (128, 32, 16, 32)])
+@pytest.mark.parametrize("d,dI,HI,Hq", [(64, 32, 2, 8), (128, 32, 16, 32), (128, 32, 8, 14), (128, 64, 2, 14)])
 def test_kl_other_shapes(d, dI, HI, Hq):
     cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=200, B=1, d=d, dI=dI, HI=HI, Hq=Hq, Hkv=2)
     run_kl(cfg, 200, seed=d + HI)
+
+
+def test_kl_two_sequences_ragged_block():
+    """Two sequences of 300 tokens: the last 128-token block of sequence 0
+    runs into sequence 1's rows (their results must not leak)."""
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=300, B=2)
+    run_kl(cfg, 300, seed=5)
 
 
 def test_kl_2k_sampled_rows():
