@@ -38,6 +38,8 @@ constexpr int kKlStages = 4;
 constexpr int kKlThreads = 384;    // warps 0-3: TMA, MMA, two idle; warps 4-11: epilogue
 constexpr int kKlEpiThreads = 256;
 constexpr int kKlBufCols = 256;    // per buffer: heads at j * 32, indexer heads at 96 + r * 32
+constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
+constexpr float kLn2 = 0.6931471805599453f;     // ln(2)
 
 template <int DI>
 struct KlTcGeom {
@@ -53,6 +55,14 @@ struct KlTcGeom {
   static __host__ __device__ int bar_off(int R) { return ring_off(R) + kKlStages * kStage; }
   static __host__ __device__ int smem(int R) { return 1024 + bar_off(R) + 256; }
 };
+
+// 2^x (PTX ex2.approx: one special-function instruction; the epilogue keeps
+// its logits in log2 units so that no multiply precedes it)
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ float tree_max16(const float *x) {
   float s8[8], s4[4];
@@ -180,7 +190,10 @@ __global__ void __launch_bounds__(kKlThreads, 1)
     float wr[kKlMaxR];
 #pragma unroll
     for (int r = 0; r < kKlMaxR; ++r)
-      wr[r] = (ok && r < R) ? p.w[((size_t)b * p.T + tau0 + row) * p.HI + g * R + r] : 0.f;
+      wr[r] = (ok && r < R) ? p.w[((size_t)b * p.T + tau0 + row) * p.HI + g * R + r] * kLog2e : 0.f;
+    // Logits in log2 units: c2 = c log2(e) (folded into the weights), a2 =
+    // a log2(e) (folded into the scale); every exponential is then 2^(x - m).
+    const float scale2 = p.scale * kLog2e;
     float ma[kKlHeads], za[kKlHeads], ua[kKlHeads];
 #pragma unroll
     for (int j = 0; j < kKlHeads; ++j) {
@@ -232,8 +245,8 @@ __global__ void __launch_bounds__(kKlThreads, 1)
         if (nmc != -INFINITY) {                       // some key of the prefix seen (per lane: no sync inside)
           float z4[4] = {0.f, 0.f, 0.f, 0.f};         // four partial sums: short chains
 #pragma unroll
-          for (int k = 0; k < HK; ++k) z4[k & 3] += __expf(c[k] - nmc);   // 0 for masked keys
-          zc = (mc == -INFINITY ? 0.f : zc * __expf(mc - nmc)) + ((z4[0] + z4[1]) + (z4[2] + z4[3]));
+          for (int k = 0; k < HK; ++k) z4[k & 3] += exp2_approx(c[k] - nmc);   // 0 for masked keys
+          zc = (mc == -INFINITY ? 0.f : zc * exp2_approx(mc - nmc)) + ((z4[0] + z4[1]) + (z4[2] + z4[3]));
           mc = nmc;
         }
         tc_wait_ld();                                 // the query heads' logits
@@ -246,14 +259,14 @@ __global__ void __launch_bounds__(kKlThreads, 1)
           float a[HK];
 #pragma unroll
           for (int k = 0; k < HK; ++k)
-            a[k] = (FULL || k < nvalid) ? __uint_as_float(va[j][k]) * p.scale : -INFINITY;
+            a[k] = (FULL || k < nvalid) ? __uint_as_float(va[j][k]) * scale2 : -INFINITY;
           const float nm = fmaxf(ma[j], tree_max16(a));
           if (nm == -INFINITY) continue;              // no key of the prefix yet (this lane)
-          const float f = ma[j] == -INFINITY ? 0.f : __expf(ma[j] - nm);
+          const float f = ma[j] == -INFINITY ? 0.f : exp2_approx(ma[j] - nm);
           float z4[4] = {0.f, 0.f, 0.f, 0.f}, u4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int k = 0; k < HK; ++k) {
-            const float ek = __expf(a[k] - nm);        // 0 for masked keys
+            const float ek = exp2_approx(a[k] - nm);   // 0 for masked keys
             z4[k & 3] += ek;
             u4[k & 3] = fmaf(ek, (FULL || k < nvalid) ? a[k] - c[k] : 0.f, u4[k & 3]);
           }
@@ -286,20 +299,20 @@ __global__ void __launch_bounds__(kKlThreads, 1)
     if (half == 0 && ok) {
       auto merge = [](float &m, float &z, float &u, float m2, float z2, float u2) {
         const float nm = fmaxf(m, m2);
-        const float f1 = m == -INFINITY ? 0.f : __expf(m - nm), f2 = m2 == -INFINITY ? 0.f : __expf(m2 - nm);
+        const float f1 = m == -INFINITY ? 0.f : exp2_approx(m - nm), f2 = m2 == -INFINITY ? 0.f : exp2_approx(m2 - nm);
         z = z * f1 + z2 * f2;
         u = u * f1 + u2 * f2;
         m = nm;
       };
       float du = 0.f;
       merge(mc, zc, du, mrg[row * MS + 0], mrg[row * MS + 1], 0.f);
-      const float lse_c = mc + logf(zc);
+      const float lse_c = mc + log2f(zc);           // log2 units; KL = ln 2 x (...) below
 #pragma unroll
       for (int j = 0; j < kKlHeads; ++j)
         if (j < hc) {
           merge(ma[j], za[j], ua[j], mrg[row * MS + 2 + 3 * j], mrg[row * MS + 3 + 3 * j], mrg[row * MS + 4 + 3 * j]);
           kl_out[((size_t)b * p.T + tau0 + row) * p.Hq + g * G + h0 + j] =
-              ua[j] / za[j] - (ma[j] + logf(za[j])) + lse_c;
+              kLn2 * (ua[j] / za[j] - (ma[j] + log2f(za[j])) + lse_c);
         }
     }
   }
