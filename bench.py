@@ -817,6 +817,82 @@ def run_longcot(args, rank, world):
           {"note": "steps = sequential decode steps of every layer; value = B x steps / time of the whole stack"})
 
 
+def run_stack(args, rank, world):
+    """The long-CoT shape as a stack of whole layers: 28 layers of the 7B
+    shape (hidden size 3584), B=8, 16384 prefilled rows, sequential decode
+    steps, every launch in one stream in layer order.  Per step and layer:
+    the projection front-end of a hidden state, the decode step (appending
+    its token) and the output projection.  The hidden inputs are drawn
+    afresh per layer: a chain of random-init layers without the norm and
+    residual the pages do not describe grows without bound (the linear
+    branch's state amplifies), so the layers are not chained numerically."""
+    import torch
+    from hybrid_linear_top_b200 import lisa as L
+    cfg = get_config("longcot_7b_28l")
+    Hm = 3584
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    n_steps = args.steps
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 * rank + 12)
+    bf = torch.bfloat16
+    lays, projs = [], []
+    for _ in range(cfg.layers):
+        lay = L.Layer.allocate(cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, cfg.L + n_steps + 1,
+                               L.LISA_BF16, decode_split=0)      # one stream: the library's (latency) choice
+        _fill_layer(L, lay, cfg, cfg.L, g, torch)
+        lays.append(lay)
+        N = sum(L.proj_widths(lay))
+        projs.append(L.Proj(Hm, (torch.randn((N, Hm), generator=g, device="cuda") / Hm ** 0.5).to(bf),
+                            (torch.randn((Hm, cfg.Hq * cfg.d), generator=g, device="cuda") /
+                             (cfg.Hq * cfg.d) ** 0.5).to(bf)))
+    x0 = [torch.randn((cfg.B, Hm), generator=g, device="cuda").to(bf) for _ in range(4)]
+    hid = torch.empty(cfg.B, Hm, dtype=bf, device="cuda")           # a layer's output projection
+    B_, Hq, Hkv, d, HI, dI = cfg.B, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI
+    t_in = {"q": torch.empty(B_, Hq, d, dtype=bf, device="cuda"), "k": torch.empty(B_, Hkv, d, dtype=bf, device="cuda"),
+            "v": torch.empty(B_, Hkv, d, dtype=bf, device="cuda"),
+            "qidx": torch.empty(B_, HI, dI, dtype=bf, device="cuda"),
+            "kidx": torch.empty(B_, Hkv, dI, dtype=bf, device="cuda"),
+            "w": torch.empty(B_, HI, device="cuda"), "lam": torch.empty(B_, Hq, device="cuda")}
+    out = torch.empty(B_, Hq, d, dtype=bf, device="cuda")
+    pos_all = (torch.arange(n_steps, device="cuda", dtype=torch.int32)[:, None] + cfg.L).repeat(1, cfg.B).contiguous()
+    stream = torch.cuda.Stream()
+
+    def one(n, s_):
+        for l in range(cfg.layers):
+            lay, pj = lays[l], projs[l]
+            lay.pos = pos_all[n]
+            src = x0[(n + l) % 4]
+            L.lisa_project_in(lay, 0, pj, 1, src, t_in["q"], t_in["k"], t_in["v"], t_in["qidx"], t_in["kidx"],
+                              t_in["w"], t_in["lam"], s_)
+            L.lisa_decode_step(lay, t_in["q"], t_in["k"], t_in["v"], t_in["kidx"], t_in["qidx"], t_in["w"],
+                               t_in["lam"], 1, out, None, None, s_)
+            L.lisa_project_out(lay, pj, 1, out, hid, s_)
+
+    block = 16
+    graphs = [_capture(torch, stream, [stream], list(range(n0, min(n_steps, n0 + block))), one)
+              for n0 in range(0, n_steps, block)]
+    graphs[0].replay()                     # warm-up (rewrites the rows the timed pass writes)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(_timed_replays(torch, stream, graphs), world, "cuda")
+    if any(int(l.err_word.item()) for l in lays) or not torch.isfinite(hid.float()).all():
+        raise RuntimeError("the chained stack flagged an error")
+    wbytes = cfg.layers * sum(2 * p_.W_in.numel() + 2 * p_.W_o.numel() for p_ in projs[:1])
+    lisa_bytes = cfg.layers * sum(_decode_bytes(cfg, cfg.L + n + 1) for n in range(n_steps))
+    total_bytes = lisa_bytes + n_steps * wbytes
+    peak, kind = load_peaks()
+    achieved = total_bytes / (ms * 1e-3) / 1e9
+    _line(rank, "LISA 28-layer stack decode tokens/s with projections, 7B shape, B=8, 16K context, M=256",
+          replica_rate(cfg.B * n_steps, ms, world), "tokens/s", args, world, ms / n_steps,
+          {"workload": "stack_7b_28l", "B": cfg.B, "layers": cfg.layers, "steps": n_steps, "L0": cfg.L, "Hm": Hm,
+           "decode_split": "library", "parallelism": f"replicas x{world}"},
+          {"bound": "hbm", "kernel": "whole stack: projections + decode_cluster_kernel per layer", "achieved": achieved,
+           "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": kind,
+           "algorithmic_bytes_total": total_bytes, "traffic": None},
+          {"note": "per layer: front-end, decode step, output projection; one stream in layer order; "
+                   "value = B x steps / time of the stack",
+           "us_per_layer": ms * 1e3 / (n_steps * cfg.layers)})
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -825,7 +901,7 @@ def main():
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=[WORKLOAD, "prefill_1p5b_16k", "ragged_7b_b32", "longcot_7b_28l", "window_1p5b_16k", "kl_1p5b_16k",
-                             "proj_1p5b_16k"])
+                             "proj_1p5b_16k", "stack_7b_28l"])
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--streams", type=int, default=32)
     ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16])
@@ -836,7 +912,7 @@ def main():
     if args.steps is None:
         args.steps = {WORKLOAD: 200000, "prefill_1p5b_16k": 20, "ragged_7b_b32": 2000,
                       "longcot_7b_28l": 1024, "window_1p5b_16k": 200000, "kl_1p5b_16k": 5,
-                      "proj_1p5b_16k": 50}[args.workload]
+                      "proj_1p5b_16k": 50, "stack_7b_28l": 256}[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if world > 1:
@@ -860,6 +936,8 @@ def main():
             run_kl(args, rank, world)
         elif args.workload == "proj_1p5b_16k":
             run_proj(args, rank, world)
+        elif args.workload == "stack_7b_28l":
+            run_stack(args, rank, world)
         else:
             run_lisa(args, rank, world)
     finally:
