@@ -17,10 +17,11 @@
 // columns, and warps 4-7 (one TMEM lane quadrant each, one row per thread)
 // write a finished tile to the column segments' own dense arrays (bf16 or
 // fp32) while the MMAs of the next tile fill the other buffer.
-// BN = 256 for many rows (the contraction is tensor-bound); BN = 32 for up to
-// 128 rows (narrow column tiles put more SMs on the weight stream).  Up to 16
-// rows (a decode step) go to a CUDA-core weight-streaming kernel instead: that
-// case is bound by HBM, not by the tensor cores.
+// BN = 256 for many rows (the contraction is tensor-bound), BN = 32 up to 128.
+// A decode step projects a few rows, which is bound by HBM (every weight read
+// once), not by the tensor cores: 3 to 32 rows take the weights as the M
+// operand with K split over a cluster (proj_swap_tc_kernel), 1 or 2 rows a
+// CUDA-core weight stream (proj_gemv_kernel).
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -223,7 +224,7 @@ static cudaError_t proj_t(const ProjParams &p, const void *x, const void *W, cud
 // lane.
 // A warp reduction per (row, column) gives the result.
 constexpr int kGemvWarps = 8;      // consumer warps; one more warp produces
-constexpr int kGemvRowsMax = 16;   // rows handled by this path at most
+constexpr int kGemvRowsMax = 2;    // rows handled by this path at most
 constexpr int kGemvKB = 256;       // K elements per stage tile (512 bytes per weight row)
 
 template <int CPC>
@@ -506,7 +507,13 @@ static cudaError_t proj_swap_t(const ProjParams &p, const void *x, const void *W
 
 cudaError_t launch_proj(const ProjParams &p, const void *x, const void *W, cudaStream_t st) {
   if (p.rows <= 0 || p.N <= 0) return cudaSuccess;
-  if (p.rows > 2 && p.rows <= kSwapRowsMax) {
+  if (p.rows <= kGemvRowsMax && gemv_smem_bytes<32>(p.rows, p.K) <= 227 * 1024) {
+    // enough CTAs to put every SM on the weight stream: 16 columns per CTA
+    // while that gives at most ~2 waves, else 32 (X is re-read by fewer warps)
+    if ((p.N + 15) / 16 <= 2 * 148) return proj_gemv_t<16>(p, x, W, st);
+    return proj_gemv_t<32>(p, x, W, st);
+  }
+  if (p.rows <= kSwapRowsMax) {
     // K split over a cluster of CS CTAs: as many as still fit the SMs in one wave
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
@@ -531,12 +538,6 @@ cudaError_t launch_proj(const ProjParams &p, const void *x, const void *W, cudaS
       case 3: return proj_swap_t<3, 32>(p, x, W, st);
       default: return proj_swap_t<4, 32>(p, x, W, st);
     }
-  }
-  if (p.rows <= kGemvRowsMax && gemv_smem_bytes<32>(p.rows, p.K) <= 227 * 1024) {
-    // enough CTAs to put every SM on the weight stream: 16 columns per CTA
-    // while that gives at most ~2 waves, else 32 (X is re-read by fewer warps)
-    if ((p.N + 15) / 16 <= 2 * 148) return proj_gemv_t<16>(p, x, W, st);
-    return proj_gemv_t<32>(p, x, W, st);
   }
   // more rows: tensor cores; narrow column tiles while the rows fit one tile
   return p.rows <= kProjRows ? proj_t<32>(p, x, W, st) : proj_t<256>(p, x, W, st);
