@@ -105,3 +105,41 @@ def test_project_out(cfg_name, B, T):
     ref = oracle.project_out(a(o), a(Wo))
     assert ref.shape == (B, T, Hm)
     _check(f64(y).reshape(B * T, Hm), a(o).reshape(B * T, -1), a(Wo), False, "y")
+
+
+@pytest.mark.parametrize("which", ["in", "out"])
+def test_projections_full_prefill_sampled_rows(which):
+    """16384 tokens of the 1.5B shape, as the bench runs them: 1280 tiles over
+    one persistent CTA per SM, so every CTA walks several tiles and reuses
+    both TMEM buffers.  Sampled rows (every tile row block, the ragged edges)
+    are checked in full against the oracle."""
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), B=1)
+    Hm, T = HIDDEN["decode_1p5b_16k"], 16384
+    lay = L.Layer.allocate(1, cfg.Hq, cfg.Hkv, cfg.d, cfg.HI, cfg.dI, cfg.M, 16)
+    rng = make_rng(700, 0)
+    rows = np.unique(np.concatenate([np.arange(0, T, 127), [1, 127, 128, 129, T - 129, T - 128, T - 1]]))
+    a = lambda z: z.astype(np.float64)
+    bf = torch.bfloat16
+    if which == "in":
+        widths = L.proj_widths(lay)
+        x = _bf16(rng, (1, T, Hm))
+        W = _bf16(rng, (sum(widths), Hm), 1.0 / np.sqrt(Hm))
+        proj = L.Proj(Hm, dev(W, "bf16"), None)
+        outs = [torch.full((1, T, wd), float("nan"), dtype=torch.float32 if i >= 5 else bf, device="cuda")
+                for i, wd in enumerate(widths)]
+        L.lisa_project_in(lay, 0, proj, T, dev(x, "bf16"), *outs)
+        torch.cuda.synchronize()
+        xs = a(x[0, rows])
+        c = 0
+        for i, wd in enumerate(widths):
+            _check(f64(outs[i][0, rows]), xs, a(W)[c:c + wd], i >= 5, f"field {i}")
+            c += wd
+    else:
+        o = _bf16(rng, (1, T, cfg.Hq, cfg.d), 1.0 / np.sqrt(cfg.d))
+        Wo = _bf16(rng, (Hm, cfg.Hq * cfg.d), 1.0 / np.sqrt(cfg.Hq * cfg.d))
+        proj = L.Proj(Hm, None, dev(Wo, "bf16"))
+        y = torch.full((1, T, Hm), float("nan"), dtype=bf, device="cuda")
+        L.lisa_project_out(lay, proj, T, dev(o, "bf16"), y)
+        torch.cuda.synchronize()
+        _check(f64(y[0, rows]), a(o[0, rows]).reshape(len(rows), -1), a(Wo), False, "y")
+    assert int(lay.err_word.item()) == 0
