@@ -329,3 +329,52 @@ def test_indexer_kl_first_token_is_zero_and_uniform_student():
             p = e / e.sum()
             entropy = -float(np.sum(p * np.log(p)))
             assert kl[0, t, h] == pytest.approx(math.log(t + 1) - entropy, rel=1e-9, abs=1e-12)
+
+
+# ---------------------------------------------------------------- KV groups
+def _group_problem(seed, B=2, Hq=6, Hkv=2, d=8, HI=4, dI=4, t=30):
+    rng = np.random.default_rng(seed)
+    f = lambda *s: rng.standard_normal(s)
+    return dict(q=f(B, Hq, d), k=f(B, Hkv, d), v=f(B, Hkv, d), qidx=f(B, HI, dI), kidx=f(B, Hkv, dI),
+                w=rng.random((B, HI)), lam=f(B, Hq), k_cache=f(B, Hkv, t, d), v_cache=f(B, Hkv, t, d),
+                kidx_cache=f(B, Hkv, t, dI), S=f(B, Hq, d, d), pos=np.array([t, t - 11][:B]))
+
+
+def test_decode_kv_groups_are_independent_problems():
+    """KV head g's query heads get what a layer with g's KV head alone gives
+    them (its K/V, its R indexer heads and key plane, its query heads): with
+    M below the prefix length the groups select different sets, so a wrong
+    group index anywhere (selection, cache, heads) changes the result."""
+    pr = _group_problem(21)
+    M = 7
+    run = lambda x: oracle.decode_step(x["q"], x["k"], x["v"], x["qidx"], x["kidx"], x["w"], x["lam"],
+                                       x["k_cache"], x["v_cache"], x["kidx_cache"], x["S"], x["pos"], M)
+    full = run(pr)
+    G, R = 3, 2
+    assert not np.array_equal(full["idx"][:, 0], full["idx"][:, 1])     # the sets differ
+    for g in range(2):
+        hs, rs, gs = slice(g * G, (g + 1) * G), slice(g * R, (g + 1) * R), slice(g, g + 1)
+        sub = run(dict(q=pr["q"][:, hs], k=pr["k"][:, gs], v=pr["v"][:, gs], qidx=pr["qidx"][:, rs],
+                       kidx=pr["kidx"][:, gs], w=pr["w"][:, rs], lam=pr["lam"][:, hs], k_cache=pr["k_cache"][:, gs],
+                       v_cache=pr["v_cache"][:, gs], kidx_cache=pr["kidx_cache"][:, gs], S=pr["S"][:, hs],
+                       pos=pr["pos"]))
+        np.testing.assert_array_equal(full["idx"][:, g], sub["idx"][:, 0])
+        np.testing.assert_allclose(full["out"][:, hs], sub["out"], rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(full["S"][:, hs], sub["S"], rtol=1e-13, atol=1e-13)
+
+
+def test_prefill_kv_groups_are_independent_problems():
+    rng = np.random.default_rng(22)
+    B, T, Hq, Hkv, d, HI, dI, M = 1, 25, 4, 2, 8, 4, 4, 5
+    f = lambda *s: rng.standard_normal(s)
+    q, k, v, qi, ki = f(B, T, Hq, d), f(B, T, Hkv, d), f(B, T, Hkv, d), f(B, T, HI, dI), f(B, T, Hkv, dI)
+    w, lam, S0 = rng.random((B, T, HI)), f(B, T, Hq), f(B, Hq, d, d)
+    full = oracle.prefill(q, k, v, qi, ki, w, lam, S0, M)
+    G, R = 2, 2
+    for g in range(Hkv):
+        hs, rs, gs = slice(g * G, (g + 1) * G), slice(g * R, (g + 1) * R), slice(g, g + 1)
+        sub = oracle.prefill(q[:, :, hs], k[:, :, gs], v[:, :, gs], qi[:, :, rs], ki[:, :, gs], w[:, :, rs],
+                             lam[:, :, hs], S0[:, hs], M)
+        np.testing.assert_array_equal(full["idx"][:, :, g], sub["idx"][:, :, 0])
+        np.testing.assert_allclose(full["out"][:, :, hs], sub["out"], rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(full["S"][:, hs], sub["S"], rtol=1e-13, atol=1e-13)

@@ -38,12 +38,19 @@ def test_project_in_equals_brute_force(P):
     assert got["w"].shape == (T, HI) and got["lam"].shape == (T, Hq)
 
 
+# the column order the library states for the front-end (lisa.h, lisa_project_in)
+DOCUMENTED_ORDER = [("q", lambda Hq, Hkv, d, HI, dI: Hq * d), ("k", lambda Hq, Hkv, d, HI, dI: Hkv * d),
+                    ("v", lambda Hq, Hkv, d, HI, dI: Hkv * d), ("qidx", lambda Hq, Hkv, d, HI, dI: HI * dI),
+                    ("kidx", lambda Hq, Hkv, d, HI, dI: Hkv * dI), ("w", lambda Hq, Hkv, d, HI, dI: HI),
+                    ("lam", lambda Hq, Hkv, d, HI, dI: Hq)]
+
+
 def test_project_in_field_order():
-    """Row n of W_in copies hidden coordinate f(n) = index of its field:
-    every entry of field i must equal x[i] (a boundary shifted by one column
-    or two fields swapped changes some entry)."""
+    """Rows of W_in copy hidden coordinate i into the i-th field of the
+    documented order: every entry of that field must equal x[i] (a boundary
+    shifted by one column or two fields swapped changes some entry)."""
     Hq, Hkv, d, HI, dI = 2, 1, 4, 2, 3
-    widths = oracle.proj_widths(Hq, Hkv, d, HI, dI)
+    widths = [fn(Hq, Hkv, d, HI, dI) for _, fn in DOCUMENTED_ORDER]
     Hm = len(widths)
     W = np.zeros((sum(widths), Hm))
     c = 0
@@ -52,8 +59,8 @@ def test_project_in_field_order():
         c += wd
     x = np.arange(1.0, Hm + 1.0)[None, :] * 10.0
     got = oracle.project_in(x, W, Hq, Hkv, d, HI, dI)
-    for i, f in enumerate(oracle.PROJ_FIELDS):
-        assert np.all(got[f] == x[0, i]), f
+    for i, (name, _) in enumerate(DOCUMENTED_ORDER):
+        assert np.all(got[name] == x[0, i]), name
 
 
 def test_project_out_identity_and_brute_force():
