@@ -213,3 +213,27 @@ def test_projection_calls_validate():
     assert lib.lisa_project_out(ctypes.byref(c), ctypes.byref(pj), 0, FAKE, FAKE, None) == L.LISA_OK
     assert lib.lisa_project_in(ctypes.byref(c), 16, ctypes.byref(pj), 4, FAKE, *args[:7],
                                None) == L.LISA_ERR_INVALID_ARG
+
+
+def test_variant_workspace_formula():
+    """Variant workspace = the documented pieces, each rounded to 256 bytes:
+    order keys per selection group (and per indexer head with one key per
+    head), the index lists, and for the prefill o_lin and the chunk
+    increments of the linear branch (per query head with its own k, v)."""
+    r256 = lambda x: (x + 255) // 256 * 256
+    c = _layer(L_max=1000)
+    B, Hq, Hkv, d, HI, M, T = 1, 12, 2, 128, 4, 256, 300
+    V1, V2, V3 = L.LISA_VAR_KEY_PER_INDEXER_HEAD, L.LISA_VAR_SHARED_SET, L.LISA_VAR_LINEAR_KV_PER_QUERY_HEAD
+    # decode (one row, every cached position): keys [Gs][L_keys] (+ [HI][L_keys]) + idx [Gs][M]
+    Lk = 1000
+    assert L.lisa_workspace_bytes_variant(c, V2, 1, L.LISA_OP_DECODE) == r256(Lk * 4) + r256(M * 4)
+    assert L.lisa_workspace_bytes_variant(c, V1, 1, L.LISA_OP_DECODE) == (
+        r256(Hkv * Lk * 4) + r256(HI * Lk * 4) + r256(Hkv * M * 4))
+    # prefill: keys [Gs][T][T] + idx [T][Gs][M] + o_lin [T][Hq][d] + dS [LH][chunks][d][d] + total [LH][d][d]
+    nc = (T + 63) // 64
+    for v, Gs, LH, per_head in [(0, Hkv, Hkv, False), (V2, 1, Hkv, False), (V3, Hkv, Hq, False),
+                                (V1 | V2, 1, Hkv, True)]:
+        want = (r256(Gs * T * T * 4) + (r256(HI * T * T * 4) if per_head else 0) + r256(T * Gs * M * 4) +
+                r256(T * Hq * d * 4) + r256(LH * nc * d * d * 4) + r256(LH * d * d * 4))
+        assert L.lisa_workspace_bytes_variant(c, v, T, L.LISA_OP_PREFILL) == want, v
+    assert B == 1
