@@ -3,14 +3,18 @@ allocate device memory (its scratch is a fixed array inside the library).
 
 Checked through the C ABI against lisa_indexer_topk (which takes a caller
 workspace) on two calls in a row: index sets are integer results, so they must
-be identical.  This file is collected last on purpose."""
+be identical.  Sampled rows (the first and the last of every pass over the
+fixed scratch) are also checked against the fp64 oracle's scores and top-M,
+under the same set rule as every other parity test, so a fault shared by both
+calls cannot pass.  This file is collected last on purpose."""
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from lisa_inputs import get_config, make_rng, gen_layer, gen_step
-from harness import make_layer, step_tensors
+from harness import check_set, make_layer, step_tensors
 
 pytestmark = pytest.mark.gpu
 
@@ -20,6 +24,21 @@ L = pytest.importorskip("hybrid_linear_top_b200.lisa")
 def _replace(cfg, **kw):
     import dataclasses
     return dataclasses.replace(cfg, **kw)
+
+
+def _check_rows_vs_oracle(got, lay_np, step, pos, rows, M):
+    """got [B, T, Hkv, M] from the GPU; rows: (b, tau) pairs to check against
+    the oracle's indexer scores over the causal prefix of token pos[b] + tau
+    (cached rows below pos[b] from the generated caches, then the appended
+    tokens 0..tau)."""
+    a = lambda z: np.asarray(z, dtype=np.float64)
+    for b, tau in rows:
+        t = int(pos[b]) + tau
+        keys = np.concatenate([a(lay_np.kidx_cache[b][:, :pos[b]]),
+                               a(step.kidx[b, :tau + 1]).transpose(1, 0, 2)], axis=1)
+        sc = oracle.indexer_scores(a(step.qidx[b, tau]), a(step.w[b, tau]), keys)
+        for g in range(sc.shape[0]):
+            check_set(got[b, tau, g], sc[g], M, t, where=f"b={b} tau={tau} g={g}")
 
 
 def test_noalloc_indexer_matches_workspace_call_twice():
@@ -43,6 +62,8 @@ def test_noalloc_indexer_matches_workspace_call_twice():
         L.lisa_indexer_topk_noalloc(lay, x["qidx"], x["w"], T, got)
         torch.cuda.synchronize()
         assert torch.equal(got, ref), f"call {call}: index sets differ"
+        _check_rows_vs_oracle(got.cpu().numpy(), lay_np, step, pos, [(0, 0), (0, T - 1), (1, 0), (1, T - 1)],
+                              cfg.M)
     assert int(lay.err_word.item()) == 0
     # sanity: the sets are real selections (M entries per row, ascending, inside the prefix)
     r = ref.cpu().numpy()
@@ -65,7 +86,12 @@ def test_noalloc_indexer_many_passes():
     x = step_tensors(step, cfg)
     L.lisa_append_cache(lay, x["k"], x["v"], x["kidx"], T)
     per_row = cfg.B * cfg.Hkv * 16384 * 4
-    assert L.NOALLOC_SCRATCH_BYTES // per_row < T      # more than one pass
+    rows_per_pass = L.NOALLOC_SCRATCH_BYTES // per_row
+    assert rows_per_pass < T      # more than one pass
+    # the first and last row of every pass (the last pass is partial), over the batch
+    taus = sorted({tau for p0 in range(0, T, rows_per_pass) for tau in (p0, min(T, p0 + rows_per_pass) - 1)})
+    sample = [(i % cfg.B, tau) for i, tau in enumerate(taus)]
+    pos = np.full(cfg.B, 16384 - T)
     ws = L.alloc_workspace(lay, T, L.LISA_OP_INDEXER_TOPK)
     ref = torch.empty((cfg.B, T, cfg.Hkv, cfg.M), dtype=torch.int32, device="cuda")
     L.lisa_indexer_topk(lay, x["qidx"], x["w"], T, ref, ws)
@@ -74,4 +100,5 @@ def test_noalloc_indexer_many_passes():
         L.lisa_indexer_topk_noalloc(lay, x["qidx"], x["w"], T, got)
         torch.cuda.synchronize()
         assert torch.equal(got, ref), f"call {call}"
+        _check_rows_vs_oracle(got.cpu().numpy(), lay_np, step, pos, sample, cfg.M)
     assert int(lay.err_word.item()) == 0
