@@ -354,6 +354,8 @@ lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, 
   p.B = L->B; p.Hq = L->Hq; p.Hkv = L->Hkv; p.G = L->Hq / L->Hkv; p.HI = L->HI; p.R = L->HI / L->Hkv;
   p.D = L->d; p.DI = L->dI; p.M = L->M; p.L_max = L->L_max; p.fuse_append = fuse_append ? 1 : 0;
   p.split_req = L->decode_split;
+  p.independent = L->independent ? 1 : 0;
+  p.debug_flags = L->debug_flags;
   p.scale = (float)(1.0 / sqrt((double)L->d));
   p.k_cache = L->k_cache; p.v_cache = L->v_cache; p.kidx_cache = L->kidx_cache;
   p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;
@@ -384,6 +386,8 @@ lisa_status lisa_decode_step_window(const lisa_layer *L, const void *q, const vo
   p.B = L->B; p.Hq = L->Hq; p.Hkv = L->Hkv; p.G = L->Hq / L->Hkv; p.HI = L->HI; p.R = L->HI / L->Hkv;
   p.D = L->d; p.DI = L->dI; p.M = L->M; p.L_max = L->L_max; p.fuse_append = fuse_append ? 1 : 0;
   p.split_req = L->decode_split;
+  p.independent = L->independent ? 1 : 0;
+  p.debug_flags = L->debug_flags;
   p.window = 1;
   p.scale = (float)(1.0 / sqrt((double)L->d));
   p.k_cache = L->k_cache; p.v_cache = L->v_cache; p.kidx_cache = L->kidx_cache;
@@ -615,6 +619,8 @@ lisa_status lisa_decode_step_variant(const lisa_layer *L, int variant, const voi
   p.B = L->B; p.Hq = L->Hq; p.Hkv = L->Hkv; p.G = L->Hq / L->Hkv; p.HI = L->HI; p.R = L->HI / L->Hkv;
   p.D = L->d; p.DI = L->dI; p.M = L->M; p.L_max = L->L_max; p.fuse_append = fuse_append ? 1 : 0;
   p.split_req = L->decode_split;
+  p.independent = L->independent ? 1 : 0;
+  p.debug_flags = L->debug_flags;
   p.scale = (float)(1.0 / sqrt((double)L->d));
   p.k_cache = L->k_cache; p.v_cache = L->v_cache; p.kidx_cache = L->kidx_cache;
   p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;
@@ -624,6 +630,9 @@ lisa_status lisa_decode_step_variant(const lisa_layer *L, int variant, const voi
     p.k_lin = k_lin;
     p.v_lin = v_lin;
   }
+  // with the row-path indexer the attention kernel reads the lists that the
+  // launch before it writes: it always waits for that launch
+  if (vg.row_indexer()) p.independent = 0;
   cudaError_t e = cudaSuccess;
   if (vg.row_indexer()) {
     // the new token's indexer keys go into the cache first: the row path reads rows 0..t there

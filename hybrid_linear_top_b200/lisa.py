@@ -25,6 +25,7 @@ LISA_FP32 = 1
 LISA_DEVERR_POS = 1
 LISA_DEVERR_TIMEOUT = 2
 LISA_DEVERR_CHECK = 4
+LISA_DEBUG_FORCE_TIMEOUT = 1
 LISA_OP_DECODE = 0
 LISA_OP_PREFILL = 1
 LISA_OP_INDEXER_TOPK = 2
@@ -63,7 +64,7 @@ class LisaLayerC(ctypes.Structure):
         ("dtype", ctypes.c_int),
         ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("kidx_cache", ctypes.c_void_p),
         ("state", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("err_word", ctypes.c_void_p),
-        ("decode_split", ctypes.c_int),
+        ("decode_split", ctypes.c_int), ("independent", ctypes.c_int), ("debug_flags", ctypes.c_int),
     ]
 
 
@@ -173,15 +174,19 @@ class Layer:
     k_cache, v_cache [B, Hkv, L_max, d]; kidx_cache [B, Hkv, L_max, dI] in the
     storage dtype; state [B, Hq, d, d] fp32; pos [B] int32; err_word [1] int32
     (all on one CUDA device).  decode_split: CTAs per (sequence, KV head) of
-    the decode step (0 = the library's choice, or 4, 8, 16)."""
+    the decode step (0 = the library's choice, or 4, 8, 16).  independent: 1
+    declares the layer's decode steps independent of the launch before them on
+    the stream (no wait for it).  debug_flags: LISA_DEBUG_* bits."""
 
     def __init__(self, B, Hq, Hkv, d, HI, dI, M, L_max, dtype, k_cache, v_cache, kidx_cache, state, pos,
-                 err_word=None, decode_split=0):
+                 err_word=None, decode_split=0, independent=0, debug_flags=0):
         self.B, self.Hq, self.Hkv, self.d, self.HI, self.dI, self.M, self.L_max = B, Hq, Hkv, d, HI, dI, M, L_max
         self.dtype = dtype
         self.k_cache, self.v_cache, self.kidx_cache = k_cache, v_cache, kidx_cache
         self.state, self.pos, self.err_word = state, pos, err_word
         self.decode_split = decode_split
+        self.independent = independent
+        self.debug_flags = debug_flags
 
     @classmethod
     def allocate(cls, B, Hq, Hkv, d, HI, dI, M, L_max, dtype=LISA_BF16, device="cuda", decode_split=0):
@@ -198,7 +203,7 @@ class Layer:
         return LisaLayerC(
             self.B, self.Hq, self.Hkv, self.d, self.HI, self.dI, self.M, self.L_max, self.dtype,
             _ptr(self.k_cache), _ptr(self.v_cache), _ptr(self.kidx_cache), _ptr(self.state), _ptr(self.pos),
-            _ptr(self.err_word), int(self.decode_split),
+            _ptr(self.err_word), int(self.decode_split), int(self.independent), int(self.debug_flags),
         )
 
     @property

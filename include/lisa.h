@@ -25,7 +25,14 @@
  *
  * Conventions for every entry point
  *   - All tensor arguments are DEVICE pointers to dense row-major arrays owned
- *     by the caller.  The library never allocates, frees or synchronises.
+ *     by the caller, with one exception: the per-step inputs and outputs of
+ *     lisa_decode_step (q, k, v, kidx, qidx, w, gate_logit, out, idx_out) may
+ *     also be page-locked host memory mapped into the device's address space
+ *     (cudaHostAlloc / cudaHostRegister with unified addressing, as torch's
+ *     pin_memory() gives); the kernel then reads and writes them across the
+ *     host link.  The layer's caches, state, pos and err_word, and every
+ *     workspace, must be device memory.  The library never allocates, frees
+ *     or synchronises.
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL =
  *     legacy default stream) and returns immediately.
  *   - Arguments are validated on the host before anything is launched; on
@@ -34,7 +41,16 @@
  *   - Launch failures reported by the CUDA runtime map to LISA_ERR_CUDA.
  *   - Checks that need device data (pos[b] out of range) are made on the
  *     device: the kernels skip the affected sequence and OR a bit into
- *     *err_word (when err_word is non-NULL); they never trap.
+ *     *err_word (when err_word is non-NULL); they never trap.  A call is
+ *     asynchronous, so a status returned by the call can only describe what
+ *     the host saw; everything found on the device (a bad position, a bounded
+ *     wait that ran out, a failed self-check) is reported through these bits,
+ *     which the caller reads after synchronising.
+ *   - Every wait inside a kernel on an asynchronous copy or on another warp's
+ *     progress is bounded in time (LISA_WAIT_LIMIT_NS per wait, measured with
+ *     the GPU's global nanosecond timer); a wait that runs out sets
+ *     LISA_DEVERR_TIMEOUT and the kernel carries on to its end without
+ *     waiting again for that stage.
  *   - Storage dtype (q, k, v, caches, out): bf16 or fp32, per lisa_layer.dtype.
  *     w, gate logits and the state are always fp32; indices are int32.
  *   - Supported shapes: d in {64, 128}; dI in {32, 64}; M a multiple of 32 in
@@ -73,6 +89,16 @@ typedef enum { LISA_BF16 = 0, LISA_FP32 = 1 } lisa_dtype;
 #define LISA_DEVERR_CHECK    4   /* an internal consistency check failed (a selected index out of
                                     range, or no threshold bucket); the access was skipped */
 
+/* Time limit of one bounded wait inside a kernel, in nanoseconds. */
+#define LISA_WAIT_LIMIT_NS   100000000ull
+
+/* Bits of lisa_layer.debug_flags (testing the failure path; 0 in normal use). */
+#define LISA_DEBUG_FORCE_TIMEOUT 1   /* lisa_decode_step: every CTA makes its first bounded wait on a
+                                        barrier that no copy will complete, with a limit of 20
+                                        microseconds, BEFORE issuing any copy; the wait runs out,
+                                        LISA_DEVERR_TIMEOUT is ORed into err_word, and every CTA
+                                        returns with nothing in flight.  Nothing else is written. */
+
 /* Operation codes for lisa_workspace_bytes(). */
 #define LISA_OP_DECODE       0
 #define LISA_OP_PREFILL      1
@@ -106,6 +132,17 @@ typedef struct {
                         shortest single step; 4 the least SM time per step when
                         many steps run concurrently.  Results do not depend on it
                         beyond float summation order.  Other calls ignore it. */
+  int independent;   /* lisa_decode_step only.  0 (default): the step waits until the
+                        launch before it on the stream has finished before it touches
+                        memory (it is launched with programmatic dependent launch, so
+                        only its start-up overlaps that launch).  1: the caller
+                        declares that this call reads nothing the previous launch on
+                        the stream writes, and writes nothing that launch reads or
+                        writes (for example steps of independent layers or sequences
+                        interleaved on one stream); the step then does not wait for
+                        it and consecutive steps run concurrently on the device.
+                        A wrong declaration gives wrong results, not an error. */
+  int debug_flags;   /* LISA_DEBUG_* bits; 0 in normal use */
 } lisa_layer;
 
 /*

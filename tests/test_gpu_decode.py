@@ -302,3 +302,42 @@ def test_decode_long_context_100k(split):
     lay = gen_layer(cfg, rng, 99999)
     step = gen_step(cfg, rng, 1)
     run_decode(cfg, lay, step, np.array([99999]), 100000, split=split)
+
+
+def test_decode_bench_launch_configuration():
+    """The headline workload in the launch configuration the bench times:
+    full-size instances (16384 cached tokens, 1.5B shape), one stream, every
+    step declared independent of the launch before it, captured in a CUDA
+    graph and replayed, the bench's CTA split.  Every instance's set, output,
+    state and appended row are checked against the oracle on the instance's
+    own data (read back from the device)."""
+    import bench
+    cfg = get_config("decode_1p5b_16k")
+    rng = make_rng(cfg.seed, 0)
+    exact = (gen_layer(cfg, rng, cfg.L - 1), gen_step(cfg, rng, 1))
+    R = 6
+    inst = [bench.Instance(L, cfg, torch, 77 + i, exact if i == 0 else None, 4) for i in range(R)]
+    for x in inst:
+        x.lay.independent = 1
+    n = cfg.L - 1
+    a = lambda t: t.detach().float().cpu().numpy().astype(np.float64)
+    before = [dict(kc=a(x.lay.k_cache[:, :, :n]), vc=a(x.lay.v_cache[:, :, :n]), kic=a(x.lay.kidx_cache[:, :, :n]),
+                   S=a(x.lay.state)) for x in inst]
+    stream = torch.cuda.Stream()
+    per, n_full, tail = bench.plan_graphs(R, R)
+    g = bench._capture(torch, stream, [stream], [inst[i % R] for i in range(per)], lambda x, s_: x.step(L, None, s_))
+    g.replay()
+    torch.cuda.synchronize()
+    for i, x in enumerate(inst):
+        assert int(x.lay.err_word.item()) == 0, f"instance {i}"
+        st = {k: a(getattr(x, k)) for k in ("q", "k", "v", "kidx", "qidx", "w", "lam")}
+        idx_g = x.idx.cpu().numpy().astype(np.int64)
+        bf = before[i]
+        ref = oracle.decode_step(st["q"], st["k"], st["v"], st["qidx"], st["kidx"], st["w"], st["lam"],
+                                 bf["kc"], bf["vc"], bf["kic"], bf["S"], np.array([n]), cfg.M, sel_override=idx_g)
+        for gg in range(cfg.Hkv):
+            check_set(idx_g[0, gg], ref["scores"][0][gg], cfg.M, n, where=f"instance {i} g={gg}")
+        check_out(f64(x.out), ref["out"], "bf16", where=f"instance {i} out")
+        check_state(f64(x.lay.state), ref["S"], where=f"instance {i} state")
+        np.testing.assert_array_equal(a(x.lay.k_cache[:, :, n]), st["k"])
+        np.testing.assert_array_equal(a(x.lay.kidx_cache[:, :, n]), st["kidx"])
