@@ -141,7 +141,7 @@ __device__ __forceinline__ void dec_find_bucket(const uint32_t *tot, uint32_t *m
   }
 }
 
-template <typename T, int D, int DI, int NC>
+template <typename T, int D, int DI, int NC, bool WIDE = false>
 __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 : 1)
     decode_cluster_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -159,7 +159,14 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
-  const int bg = blockIdx.x / NC;
+  // Cluster form: the NC CTAs of one cluster serve (b, g); CTA `rank` scores
+  // key slice `rank` and owns state columns slab `rank`.  Wide form: NSL CTAs
+  // (NSL / NC clusters) serve (b, g); CTA `slice` scores key slice `slice`
+  // and updates state rows slab `slice`, and the last cluster to finish
+  // selects and attends.
+  const int NSL = WIDE ? p.nw : NC;
+  const int bg = blockIdx.x / NSL;
+  const int slice = WIDE ? (int)(blockIdx.x % NSL) : rank;
   const int g = bg % p.Hkv, b = bg / p.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G, M = p.M, R = p.R;
@@ -198,8 +205,23 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
-  // Everything read below may have been written by the previous kernel.
-  grid_dep_wait();
+  if (p.independent) {
+    // The caller declared this step independent of the launch before it on the
+    // stream: no wait, and the launch after it may start at once.
+    grid_dep_launch();
+  } else {
+    // Everything read below may have been written by the previous kernel.
+    grid_dep_wait();
+  }
+  if (p.debug_flags & LISA_DEBUG_FORCE_TIMEOUT) {
+    // Failure-path test: no copy has been issued, so the first ring stage
+    // never completes and the bounded wait runs out.  Every CTA of the
+    // cluster returns here, before any cluster barrier or copy.
+    __syncthreads();                     // the barriers are initialised
+    const bool done = mbar_wait_bounded(&bars[0], 0u, 20000ull);
+    if (!done && tid == 0) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+    return;
+  }
 
   const int t = p.pos[b];                  // in flight while the loads below are issued
   const T *kidx_cache = reinterpret_cast<const T *>(p.kidx_cache) + (size_t)bg * p.L_max * DI;
@@ -271,10 +293,11 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     return;
   }
   const int n = t + 1;
-  const int kpc = (((n + NC - 1) / NC) + 31) & ~31;
-  const int k0 = min(n, rank * kpc);
-  const int k1 = min(n, k0 + kpc);
-  const int cnt = k1 - k0;
+  const int kpc = (((n + NSL - 1) / NSL) + 31) & ~31;
+  // this CTA's key slice (the wide form's last cluster later takes wider ranges)
+  int k0 = min(n, slice * kpc);
+  int k1 = min(n, k0 + kpc);
+  int cnt = k1 - k0;
   const int nsub = window ? 0 : (cnt + SUB - 1) / SUB;
 
   // ---------------------------------------------------------------- TMA ring
@@ -528,9 +551,9 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     //     of the 1024-bin range-histogram bin that holds the kl-th largest of
     //     those values has at least kl of this CTA's keys at or above it.
     //     Also the largest key, for the range of the exact select.
-    const int kl = (M + NC - 1) / NC;
+    const int kl = (M + NSL - 1) / NSL;
     int covered = 0;
-    for (int r = 0; r < NC; ++r) {
+    for (int r = 0; r < NSL; ++r) {
       const int cr = min(n, (r + 1) * kpc) - min(n, r * kpc);
       if (cr >= kl) covered += kl;
     }
@@ -903,8 +926,9 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
 
   // The next kernel on the stream may be scheduled from here on: its CTAs
   // wait in their prologue, so a later trigger keeps them from holding SM
-  // slots through this kernel's key stream and selection.
-  grid_dep_launch();
+  // slots through this kernel's key stream and selection.  (An independent
+  // step has let it start already.)
+  if (!p.independent) grid_dep_launch();
   // ---------------------------------------------------------------- sparse attention (this CTA's rows)
   unsigned char *kvs = ring;                 // [rpc] K rows then [rpc] V rows, stride RS
   for (int r = tid; r < rpc; r += kDecThreads) {

@@ -59,7 +59,21 @@ struct DecodeParams {
   int stages;                           // TMA ring stages
   int stage_keys;                       // keys per ring stage
   int kpc_max;                          // order keys per CTA, upper bound
+  int independent;                      // 1: no wait on the previous launch of the stream (lisa_layer.independent)
+  int debug_flags;                      // LISA_DEBUG_* bits
+  // wide form (nw > 0): nw CTAs per (b, g) stream the keys and the state; the
+  // last of their clusters to finish selects and attends.  Workspace per (b, g):
+  int nw;                               // CTAs per (b, g), a multiple of 8, >= G; 0: the cluster form
+  uint32_t *wkeys;                      // [B*Hkv][wkeys_stride] order keys of positions 0..t
+  uint32_t *wtheta;                     // [B*Hkv][nw][2] per-CTA bound and largest key
+  float *wpart;                         // [B*Hkv][nw][2][d] per-CTA partial o_lin of (up to) two heads
+  unsigned *wcount;                     // [B*Hkv] arrival counters (zero between calls)
+  int wkeys_stride;
 };
+// Workspace of the wide decode form (0 when it does not apply).
+size_t decode_wide_workspace_bytes(int B, int Hkv, int G, int D, int L_max, int nw);
+// CTAs per (b, g) the wide form would use for this layer (0: the cluster form).
+int decode_wide_nw(int B, int Hkv, int G, int D, int DI, int dtype, int sms);
 
 // Dynamic shared memory of the decode kernel for a cluster of nc CTAs.
 int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc, bool lin_kv = false);
