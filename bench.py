@@ -48,7 +48,7 @@ WORKLOAD = "decode_1p5b_16k"
 # DRAM bytes (read + write) of one decode launch from an ncu capture of this
 # kernel on this workload, by CTA split (the ncu summary under profiles/);
 # None where no capture of the current kernel exists.
-DECODE_TRAFFIC = {4: None, 8: None, 16: None, 0: None}
+DECODE_TRAFFIC = {4: 5395456, 8: None, 16: None, 0: None, 32: None, 64: None}
 # nominal HBM3e bandwidth of a B200 (about 8 TB/s), for the second fraction
 NOMINAL_HBM_GBS = 8000.0
 
@@ -265,6 +265,8 @@ class Instance:
         self.lay.pos.fill_(n)
         self.out = torch.empty(cfg.B, cfg.Hq, cfg.d, dtype=bf, device=dev)
         self.idx = torch.empty(cfg.B, cfg.Hkv, cfg.M, dtype=torch.int32, device=dev)
+        # a workspace of its own (steps of different instances may run concurrently)
+        self.ws = L.alloc_workspace(self.lay, 1, L.LISA_OP_DECODE)
         self.host_in = None
 
     def step(self, L, ws, stream=None):
@@ -421,12 +423,11 @@ def run_lisa(args, rank, world):
     rng = make_rng(cfg.seed, 0)
     exact = (gen_layer(cfg, rng, cfg.L - 1), gen_step(cfg, rng, 1))
     inst = [Instance(L, cfg, torch, 1000 * rank + i, exact if i == 0 else None, args.split) for i in range(R)]
-    ws = L.alloc_workspace(inst[0].lay, 1, L.LISA_OP_DECODE)
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
     chains = [torch.cuda.Stream() for _ in range(S)]
-    run = lambda x, s_: x.step(L, ws, s_)
+    run = lambda x, s_: x.step(L, x.ws, s_)
 
     def set_mode(independent, split):
         for x in inst:
@@ -445,7 +446,7 @@ def run_lisa(args, rank, world):
     set_mode(True, args.split)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            inst[i % R].step(L, ws, stream)
+            inst[i % R].step(L, inst[i % R].ws, stream)
     stream.synchronize()
 
     # ---- headline: exactly K steps in ONE stream rotating over the R
@@ -485,7 +486,7 @@ def run_lisa(args, rank, world):
             flush_l2(torch, 4 * l2)
             torch.cuda._sleep(400000)
             e0.record(stream)
-            inst[i].step(L, ws, stream)
+            inst[i].step(L, inst[i].ws, stream)
             e1.record(stream)
         torch.cuda.synchronize()
         lat.append(e0.elapsed_time(e1) * 1e3)
@@ -517,8 +518,8 @@ def run_lisa(args, rank, world):
     h2d = inst[0].in_bytes
     d2h = inst[0].out.numel() * inst[0].out.element_size()
     e2e = {}
-    for mode, fn in (("zero_copy", lambda x, s_: x.step_e2e(L, ws, s_)),
-                     ("copy_engine", lambda x, s_: x.step_e2e_dma(L, ws, s_))):
+    for mode, fn in (("zero_copy", lambda x, s_: x.step_e2e(L, x.ws, s_)),
+                     ("copy_engine", lambda x, s_: x.step_e2e_dma(L, x.ws, s_))):
         e_ms = max_over_ranks(_timed_steps(torch, stream, one_stream(K, fn), l2, barrier), world, "cuda")
         e2e[mode] = replica_rate(K * cfg.B, e_ms, world)
     if any(int(x.lay.err_word.item()) for x in inst):
@@ -1005,7 +1006,7 @@ def main():
                              "proj_1p5b_16k", "stack_7b_28l"])
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--streams", type=int, default=32)
-    ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16])
+    ap.add_argument("--split", type=int, default=4, choices=[0, 4, 8, 16, 32, 64])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

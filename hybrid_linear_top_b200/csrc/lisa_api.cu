@@ -56,8 +56,9 @@ lisa_status check_layer(const lisa_layer *L) {
   if (L->dI != 32 && L->dI != 64) return fail(LISA_ERR_UNSUPPORTED, "dI=%d not in {32,64}", L->dI);
   if (L->M % 32 || L->M < 32 || L->M > 1024) return fail(LISA_ERR_UNSUPPORTED, "M=%d not a multiple of 32 in [32,1024]", L->M);
   if ((long long)L->B * L->Hkv > 65535) return fail(LISA_ERR_UNSUPPORTED, "B*Hkv=%lld > 65535", (long long)L->B * L->Hkv);
-  if (L->decode_split != 0 && L->decode_split != 4 && L->decode_split != 8 && L->decode_split != 16)
-    return fail(LISA_ERR_INVALID_ARG, "decode_split=%d not in {0, 4, 8, 16}", L->decode_split);
+  if (L->decode_split != 0 && L->decode_split != 4 && L->decode_split != 8 && L->decode_split != 16 &&
+      L->decode_split != 32 && L->decode_split != 64)
+    return fail(LISA_ERR_INVALID_ARG, "decode_split=%d not in {0, 4, 8, 16, 32, 64}", L->decode_split);
   return LISA_OK;
 }
 
@@ -166,6 +167,72 @@ VarPlan var_plan(const lisa_layer *L, const VariantGeom &vg, int T, int op) {
 }
 
 void set_select_smem(lisa::RowsParams &r, int n_max);
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Workspace of lisa_decode_step: that of the wide form (bf16), sized for 64
+// CTAs per (sequence, KV head); 0 for fp32 storage.
+size_t decode_workspace_bytes(const lisa_layer *L) {
+  if (L->dtype != LISA_BF16) return 0;
+  return lisa::decode_wide_workspace_bytes(L->B, L->Hkv, L->Hq / L->Hkv, L->d, L->L_max, 64);
+}
+
+// Picks the decode form.  The wide form (decode_split 32 or 64, or the
+// library's choice when the workspace is given and few (sequence, KV head)
+// pairs leave SMs idle) needs bf16 storage and the decode workspace; its
+// pieces are carved out of the workspace here.
+lisa_status plan_decode_form(const lisa_layer *L, void *workspace, size_t ws_bytes, lisa::DecodeParams &p) {
+  const int G = L->Hq / L->Hkv;
+  const size_t need = decode_workspace_bytes(L);
+  const bool explicit_wide = L->decode_split == 32 || L->decode_split == 64;
+  int nw = 0;
+  if (explicit_wide) {
+    if (L->dtype != LISA_BF16)
+      return fail(LISA_ERR_UNSUPPORTED, "decode_split=%d (the wide form) needs bf16 storage", L->decode_split);
+    if (L->decode_split < G)
+      return fail(LISA_ERR_UNSUPPORTED, "decode_split=%d is smaller than Hq/Hkv=%d", L->decode_split, G);
+    if (!workspace || ws_bytes < need)
+      return fail(LISA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace ? ws_bytes : 0, need);
+    nw = L->decode_split;
+  } else if (L->decode_split == 0 && need && workspace && ws_bytes >= need) {
+    nw = lisa::decode_wide_nw(L->B, L->Hkv, G, L->d, L->dI, L->dtype, sm_count());
+  }
+  if (nw && lisa::decode_wide_smem_bytes(L->L_max, L->M, G, L->d, L->dI, nw) > kMaxSmem) {
+    if (explicit_wide)
+      return fail(LISA_ERR_UNSUPPORTED, "L_max=%d needs more shared memory per CTA than a B200 SM has", L->L_max);
+    nw = 0;
+  }
+  if (!nw) return LISA_OK;
+  lisa_status s;
+  if ((s = check_ptr(workspace, "workspace"))) return s;
+  const size_t pairs = (size_t)L->B * L->Hkv;
+  char *ws = static_cast<char *>(workspace);
+  size_t off = 0;
+  p.wcount = reinterpret_cast<unsigned *>(ws + off); off += round256(pairs * 4);
+  p.wtheta = reinterpret_cast<uint32_t *>(ws + off); off += round256(pairs * 64 * 2 * 4);
+  p.wpart = reinterpret_cast<float *>(ws + off); off += round256(pairs * 64 * 2 * L->d * 4);
+  p.wkeys = reinterpret_cast<uint32_t *>(ws + off);
+  p.wkeys_stride = round4(L->L_max);
+  p.nw = nw;
+  return LISA_OK;
+}
 
 // Row-path parameters of the variant's indexer: `sel` scores and selects in
 // the Gs selection groups; with one key per indexer head, `ph` first scores
@@ -281,7 +348,7 @@ const char *lisa_status_str(lisa_status s) {
 
 size_t lisa_workspace_bytes(const lisa_layer *layer, int T, int op) {
   if (check_layer(layer) != LISA_OK || T < 0) return 0;
-  if (op == LISA_OP_DECODE) return 0;   // the decode step keeps its intermediates on chip
+  if (op == LISA_OP_DECODE) return decode_workspace_bytes(layer);
   if (op == LISA_OP_PREFILL) return T ? rows_plan(layer, T, true).total : 0;
   if (op == LISA_OP_INDEXER_TOPK) return T ? rows_plan(layer, T, false).total : 0;
   if (op == LISA_OP_PREFILL_WINDOW) return T ? rows_plan(layer, T, true, false).total : 0;
@@ -343,8 +410,6 @@ lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, 
       (s = check_ptr(qidx, "qidx")) || (s = check_ptr(w, "w")) || (s = check_ptr(gate_logit, "gate_logit")) ||
       (s = check_ptr(out, "out")) || (s = check_ptr(idx_out, "idx_out", false)))
     return s;
-  (void)workspace;
-  (void)ws_bytes;
   const int esz = L->dtype == LISA_BF16 ? 2 : 4;
   if (lisa::decode_smem_bytes(L->L_max, L->M, L->Hq / L->Hkv, L->d, L->dI, esz, 8) > kMaxSmem)
     return fail(LISA_ERR_UNSUPPORTED, "L_max=%d needs more shared memory per CTA than a B200 SM has", L->L_max);
@@ -361,6 +426,7 @@ lisa_status lisa_decode_step(const lisa_layer *L, const void *q, const void *k, 
   p.state = L->state; p.pos = L->pos; p.err_word = L->err_word;
   p.q = q; p.k = k; p.v = v; p.kidx = kidx; p.qidx = qidx; p.w = w; p.gate = gate_logit;
   p.out = out; p.idx_out = idx_out;
+  if ((s = plan_decode_form(L, workspace, ws_bytes, p))) return s;
   cudaError_t e = lisa::launch_decode(p, L->dtype, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode_step");
   return ok();
@@ -466,11 +532,11 @@ lisa_status lisa_prefill(const lisa_layer *L, int T, const void *q, const void *
   r.require_pos0 = 1;
   r.q = q; r.k = k; r.v = v; r.kidx = kidx; r.qidx = qidx; r.w = w; r.gate = gate_logit; r.out = out;
   char *ws = static_cast<char *>(workspace);
-  r.keys = reinterpret_cast<uint32_t *>(ws + plan.keys);
   r.idx = idx_out ? idx_out : reinterpret_cast<int *>(ws + plan.idx);
   r.olin = reinterpret_cast<float *>(ws + plan.olin);
   r.dS = reinterpret_cast<float *>(ws + plan.dS);
   r.Ptot = reinterpret_cast<float *>(ws + plan.Ptot);
+  r.keys = reinterpret_cast<uint32_t *>(ws + plan.keys);
   r.row_chunk = plan.row_chunk;
   r.L_keys = plan.L_keys;
   set_select_smem(r, T);
@@ -541,7 +607,10 @@ lisa_status lisa_indexer_topk_noalloc(const lisa_layer *L, const void *qidx, con
 size_t lisa_workspace_bytes_variant(const lisa_layer *layer, int variant, int T, int op) {
   VariantGeom vg;
   if (check_layer(layer) != LISA_OK || T < 0 || check_variant(layer, variant, vg) != LISA_OK) return 0;
-  if (op == LISA_OP_DECODE) return vg.row_indexer() ? var_plan(layer, vg, 1, op).total : 0;
+  if (op == LISA_OP_DECODE)
+    return vg.row_indexer() ? var_plan(layer, vg, 1, op).total : vg.lin_kv ? 0 : decode_workspace_bytes(layer);
+  if (variant == 0 && (op == LISA_OP_PREFILL || op == LISA_OP_INDEXER_TOPK))
+    return lisa_workspace_bytes(layer, T, op);            // the default calls (variant 0 runs them)
   if (op == LISA_OP_PREFILL || op == LISA_OP_INDEXER_TOPK) return T ? var_plan(layer, vg, T, op).total : 0;
   return 0;
 }
@@ -571,6 +640,7 @@ lisa_status lisa_indexer_topk_variant(const lisa_layer *L, int variant, const vo
   lisa_status s;
   VariantGeom vg;
   if ((s = check_layer(L)) || (s = check_variant(L, variant, vg))) return s;
+  if (variant == 0) return lisa_indexer_topk(L, qidx, w, T, idx_out, workspace, ws_bytes, stream);
   if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
   if (T == 0 || L->B == 0) return ok();
   if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);
@@ -648,6 +718,10 @@ lisa_status lisa_decode_step_variant(const lisa_layer *L, int variant, const voi
     p.sel_groups = vg.Gs;
     p.kidx = nullptr; p.qidx = nullptr; p.w = nullptr;
     p.idx_out = nullptr;
+  } else if (!vg.lin_kv) {
+    // the default reading: the same forms as lisa_decode_step
+    lisa_status s2;
+    if ((s2 = plan_decode_form(L, workspace, ws_bytes, p))) return s2;
   }
   e = lisa::launch_decode(p, L->dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode_step_variant");
@@ -661,6 +735,8 @@ lisa_status lisa_prefill_variant(const lisa_layer *L, int variant, int T, const 
   lisa_status s;
   VariantGeom vg;
   if ((s = check_layer(L)) || (s = check_variant(L, variant, vg))) return s;
+  if (variant == 0)
+    return lisa_prefill(L, T, q, k, v, kidx, qidx, w, gate_logit, out, idx_out, workspace, ws_bytes, stream);
   if (T < 0) return fail(LISA_ERR_INVALID_ARG, "T=%d < 0", T);
   if (T == 0 || L->B == 0) return ok();
   if (T > L->L_max) return fail(LISA_ERR_INVALID_ARG, "T=%d > L_max=%d", T, L->L_max);

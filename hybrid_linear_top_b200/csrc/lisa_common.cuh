@@ -87,6 +87,18 @@ __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" :::);
 }
 
+// ---------------------------------------------------------------- cluster barrier, split
+// barrier.cluster in two halves: every thread of every CTA of the cluster
+// arrives (its earlier shared-memory accesses released), and a later wait
+// returns once all have arrived (acquire).  Work placed between the two
+// overlaps the barrier's latency.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier + bulk copy
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -55,7 +55,7 @@ struct ScoreGeom {
 
 struct DecLayout {
   int region0, cand_key, cand_pos, pin;
-  int keys, hist, tot, misc, sel, qs, qi, ks, vs, kis, gl, klin, vlin, part, pml, olin, logit, sidx, bars, total;
+  int keys, hist, tot, misc, sel, qs, qi, ks, vs, kis, gl, klin, vlin, part, pml, olin, logit, sidx, wred, bars, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
@@ -68,7 +68,7 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // writes for this CTA's output columns (merge).
 __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, int G, int D, int DI, int esize,
                                                 int NC, int stages = kStages, int stage_bytes = kStageBytes,
-                                                bool lin_kv = false) {
+                                                bool lin_kv = false, bool wide = false) {
   DecLayout L;
   const int rpc = M / NC;
   const int kv = 2 * rpc * (D * esize + 16);
@@ -103,6 +103,7 @@ __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, i
     L.logit = off; off += align16(a > bred ? a : bred);
   }
   L.sidx = off; off += align16(rpc * 4);
+  L.wred = off; off += wide ? align16(2 * 8 * D * 4) : 0;   // wide form: [2 heads][8 warps][D] readout sums
   L.bars = off; off += kStages * 8;
   L.total = align16(off) + 1024;
   return L;
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   const int SUB = p.stage_keys;                  // keys per ring stage
   const int STB = SUB * RB;                      // bytes per ring stage
   const bool lin_kv = p.k_lin != nullptr;  // variant: linear-branch k, v of its own per query head
-  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC, NS, STB, lin_kv);
+  const DecLayout lay = dec_layout(p.kpc_max, p.L_max, M, G, D, DI, (int)sizeof(T), NC, NS, STB, lin_kv, WIDE);
   unsigned char *ring = smem + lay.region0;
   uint32_t *keys = reinterpret_cast<uint32_t *>(smem + lay.keys);
   uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist);
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
+    if constexpr (WIDE) misc[60] = 0u;   // "this cluster holds the last arrival" (wide form)
   }
   if (p.independent) {
     // The caller declared this step independent of the launch before it on the
@@ -275,19 +277,41 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   const int cq = tid % QPR;                // same float4 column for every row this thread visits
   const int gA = min(G, HP);
   float4 sv[HP][ITER];
+  if constexpr (!WIDE) {
 #pragma unroll
-  for (int hh = 0; hh < HP; ++hh) {
-    if (hh >= gA) continue;
-    const float *S = p.state + ((size_t)b * p.Hq + g * G + hh) * D * D;
+    for (int hh = 0; hh < HP; ++hh) {
+      if (hh >= gA) continue;
+      const float *S = p.state + ((size_t)b * p.Hq + g * G + hh) * D * D;
 #pragma unroll
-    for (int it = 0; it < ITER; ++it) {
-      const int idx = tid + it * kDecThreads;
-      if (idx < D * QPR) sv[hh][it] = *reinterpret_cast<const float4 *>(S + (size_t)(idx / QPR) * D + c0s + cq * 4);
+      for (int it = 0; it < ITER; ++it) {
+        const int idx = tid + it * kDecThreads;
+        if (idx < D * QPR) sv[hh][it] = *reinterpret_cast<const float4 *>(S + (size_t)(idx / QPR) * D + c0s + cq * 4);
+      }
     }
+    // heads beyond the first HP: their slab rows requested into L2 now
+    for (int i = tid; i < (G - gA) * D; i += kDecThreads)
+      prefetch_l2(p.state + ((size_t)b * p.Hq + g * G + gA + i / D) * D * D + (size_t)(i % D) * D + c0s);
   }
-  // heads beyond the first HP: their slab rows requested into L2 now
-  for (int i = tid; i < (G - gA) * D; i += kDecThreads)
-    prefetch_l2(p.state + ((size_t)b * p.Hq + g * G + gA + i / D) * D * D + (size_t)(i % D) * D + c0s);
+  // wide form: this CTA updates state rows [r_lo, r_hi) of the group's G * D
+  // rows (row r = key dim r % D of head r / D; the G heads of a group are
+  // contiguous, so the slab is one contiguous block); at most two heads,
+  // since the host keeps rps <= D
+  constexpr int SQ = D / 4;                // float4 per state row
+  constexpr int WIT = 2;                   // float4 of the slab per thread and pass
+  const int rps = (G * D + NSL - 1) / NSL;
+  const int r_lo = min(G * D, slice * rps), r_hi = min(G * D, r_lo + rps);
+  const int nf = WIDE ? (r_hi - r_lo) * SQ : 0;
+  float *Sg = p.state + ((size_t)b * p.Hq + g * G) * D * D;
+  float4 svw[WIT];
+  if constexpr (WIDE) {
+#pragma unroll
+    for (int it = 0; it < WIT; ++it) {
+      const int f = tid + it * kDecThreads;
+      if (f < nf) svw[it] = *reinterpret_cast<const float4 *>(Sg + (size_t)r_lo * D + (size_t)f * 4);
+    }
+    for (int f = tid * 8 + WIT * kDecThreads; f < nf; f += kDecThreads * 8)   // later passes: into L2
+      prefetch_l2(Sg + (size_t)r_lo * D + (size_t)f * 4);
+  }
   if (t < 0 || t >= p.L_max) {  // same value in every CTA of the cluster: all leave together
     if (rank == 0 && tid == 0) set_err(p.err_word, LISA_DEVERR_POS);
     return;
@@ -370,7 +394,69 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   // ---------------------------------------------------------------- linear state
   // S_h <- S_h + k^T v on columns [c0s, c0s + COLS); o_lin[h][c] = sum_i q_h[i] S_h[i][c].
   // Runs while the first key stages are in flight.
-  {
+  if constexpr (WIDE) {
+    // rows [r_lo, r_hi): S[r][:] += k[r % D] v, and the partial readout
+    // o_lin[h][:] += q_h[r % D] S[r][:] of the (at most two) heads of the
+    // slab, summed over the CTA into this CTA's slot of the workspace
+    const int h_lo = r_lo / D;
+    const int quad = tid % SQ;             // the same column quad for every float4 of this thread
+    float vq[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) vq[j] = vs[quad * 4 + j];
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int f0 = 0; f0 < nf; f0 += WIT * kDecThreads) {
+      float4 cur[WIT];
+#pragma unroll
+      for (int it = 0; it < WIT; ++it) {
+        const int f = f0 + tid + it * kDecThreads;
+        if (f < nf) cur[it] = f0 == 0 ? svw[it] : *reinterpret_cast<const float4 *>(Sg + (size_t)r_lo * D + (size_t)f * 4);
+      }
+#pragma unroll
+      for (int it = 0; it < WIT; ++it) {
+        const int f = f0 + tid + it * kDecThreads;
+        if (f < nf) {
+          const int r = r_lo + f / SQ, i = r % D, hh = r / D;
+          const float ki = ks[i], qi = qs[hh * D + i];
+          float4 sn = cur[it];
+          sn.x = fmaf(ki, vq[0], sn.x);
+          sn.y = fmaf(ki, vq[1], sn.y);
+          sn.z = fmaf(ki, vq[2], sn.z);
+          sn.w = fmaf(ki, vq[3], sn.w);
+          *reinterpret_cast<float4 *>(Sg + (size_t)r * D + quad * 4) = sn;
+          // the slab's first head, or the second (compile-time indices only)
+          const float q0 = hh == h_lo ? qi : 0.f, q1 = hh == h_lo ? 0.f : qi;
+          acc[0][0] = fmaf(q0, sn.x, acc[0][0]);
+          acc[0][1] = fmaf(q0, sn.y, acc[0][1]);
+          acc[0][2] = fmaf(q0, sn.z, acc[0][2]);
+          acc[0][3] = fmaf(q0, sn.w, acc[0][3]);
+          acc[1][0] = fmaf(q1, sn.x, acc[1][0]);
+          acc[1][1] = fmaf(q1, sn.y, acc[1][1]);
+          acc[1][2] = fmaf(q1, sn.z, acc[1][2]);
+          acc[1][3] = fmaf(q1, sn.w, acc[1][3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = SQ; o < 32; o <<= 1)        // lanes of a warp with the same quad
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[sl][j] += __shfl_xor_sync(0xffffffffu, acc[sl][j], o);
+    float *wred = reinterpret_cast<float *>(smem + lay.wred);   // [2][8 warps][D]
+    if (lane < SQ)
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) wred[(sl * 8 + warp) * D + quad * 4 + j] = acc[sl][j];
+    __syncthreads();
+    float *part = p.wpart + ((size_t)bg * NSL + slice) * 2 * D;
+    for (int c = tid; c < 2 * D; c += kDecThreads) {
+      float o = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < 8; ++w8) o += wred[((c / D) * 8 + w8) * D + c % D];
+      part[c] = o;
+    }
+  } else {
     float vj[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) vj[j] = vs[c0s + cq * 4 + j];
@@ -532,26 +618,49 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   __syncthreads();
 
   // ---------------------------------------------------------------- top-M
-  int *sel0 = cluster.map_shared_rank(sel, 0);
-  if (window) {
-    if (rank == 0) {
-      if (ext) {                         // the caller's list of this (b, group)
-        const int *src = p.sel_ext + ((size_t)b * p.sel_groups + (p.sel_groups == 1 ? 0 : g)) * M;
-        for (int j = tid; j < M; j += kDecThreads) sel[j] = src[j];
-      } else {                           // the M (= W) most recent positions t-M+1 .. t, or the whole prefix
-        for (int j = tid; j < M; j += kDecThreads) sel[j] = n <= M ? (j < n ? j : -1) : t - M + 1 + j;
+  // Wide form: every CTA of (b, g) arrives once, after publishing its slice in
+  // the workspace.  The CTA that arrives last returns the counter to zero and
+  // flags every CTA of its cluster; that cluster alone goes on (with every
+  // slice visible to it), the others leave.  Only local shared memory is read
+  // after the barrier, so a leaving CTA is never read by another.
+  auto wide_arrive = [&]() -> bool {
+    __threadfence();                     // this thread's workspace writes come before the arrival
+    __syncthreads();
+    if (tid == 0) {
+      const unsigned old = atomicAdd(p.wcount + bg, 1u);
+      if (old == (unsigned)NSL - 1u) {
+        atomicExch(p.wcount + bg, 0u);
+        __threadfence();
+        for (int r = 0; r < NC; ++r) cluster.map_shared_rank(misc, r)[60] = 1u;
       }
+    }
+    cluster.sync();
+    const bool last = misc[60] != 0u;
+    if (last) __threadfence();
+    return last;
+  };
+  int *sel0 = cluster.map_shared_rank(sel, 0);
+  // Every CTA builds the whole index list in its own shared memory, except on
+  // the cluster-wide radix path, which builds it in CTA 0 (local_list false).
+  bool local_list = true;
+  if (window) {
+    if (ext) {                           // the caller's list of this (b, group)
+      const int *src = p.sel_ext + ((size_t)b * p.sel_groups + (p.sel_groups == 1 ? 0 : g)) * M;
+      for (int j = tid; j < M; j += kDecThreads) sel[j] = src[j];
+    } else {                             // the M (= W) most recent positions t-M+1 .. t, or the whole prefix
+      for (int j = tid; j < M; j += kDecThreads) sel[j] = n <= M ? (j < n ? j : -1) : t - M + 1 + j;
     }
   } else if (n > M) {
     constexpr int SEG = kCandCap / NC;                  // candidate slots of each rank in CTA 0
     uint32_t *fh = hist + 1024;                         // CTA 0: 1024-bin histogram of candidate keys
     uint32_t *segp = tot + 64;                          // CTA 0: exclusive prefix of the segment sizes
-    uint32_t *misc0 = cluster.map_shared_rank(misc, 0);
     // (a) theta: every thread keeps the 4 largest of its keys; the lower edge
     //     of the 1024-bin range-histogram bin that holds the kl-th largest of
     //     those values has at least kl of this CTA's keys at or above it.
     //     Also the largest key, for the range of the exact select.
-    const int kl = (M + NSL - 1) / NSL;
+    const int ns = (n + kpc - 1) / kpc;                 // slices that hold keys (the others are empty)
+    const int kl = (M + ns - 1) / ns;
+    uint32_t theta_r = 0xFFFFFFFFu;                     // this CTA's bound (every thread holds it)
     int covered = 0;
     for (int r = 0; r < NSL; ++r) {
       const int cr = min(n, (r + 1) * kpc) - min(n, r * kpc);
@@ -605,30 +714,62 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         misc[4] = theta;
         misc[6] = vmax;
       }
+      theta_r = theta;
     }
-    cluster.sync();                                     // bounds published, every ring is free
     uint32_t lb = 0, hi = 0;
-    {
-      // lane r of every warp reads rank r's bound and maximum (one remote
-      // load per lane, not per thread and rank)
-      uint32_t mn = 0xFFFFFFFFu;
-      if (lane < NC) {
-        const uint32_t *mr = cluster.map_shared_rank(misc, lane);
-        mn = mr[4];
-        hi = mr[6];
+    if constexpr (WIDE) {
+      // publish this slice (order keys, bound, largest key) and arrive
+      {
+        uint32_t *wk = p.wkeys + (size_t)bg * p.wkeys_stride + k0;
+        for (int j = tid; j < cnt; j += kDecThreads) wk[j] = keys[j];
+        if (tid == 0) {
+          p.wtheta[((size_t)bg * NSL + slice) * 2] = misc[4];
+          p.wtheta[((size_t)bg * NSL + slice) * 2 + 1] = misc[6];
+        }
       }
+      if (!wide_arrive()) return;
+      // the last cluster: rank r takes the contiguous positions of NSL / NC
+      // slices, and the bound is the smallest over every slice
+      const int spr = (NSL / NC) * kpc;
+      k0 = min(n, rank * spr);
+      k1 = min(n, k0 + spr);
+      cnt = k1 - k0;
+      const uint32_t *wk = p.wkeys + (size_t)bg * p.wkeys_stride + k0;
+      for (int j = tid; j < cnt; j += kDecThreads) keys[j] = __ldcg(wk + j);
+      if (warp == 0) {
+        uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+        for (int w = lane; w < NSL; w += 32) {
+          mn = min(mn, __ldcg(p.wtheta + ((size_t)bg * NSL + w) * 2));
+          mx = max(mx, __ldcg(p.wtheta + ((size_t)bg * NSL + w) * 2 + 1));
+        }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        for (int o = 16; o > 0; o >>= 1) {
+          mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        if (lane == 0) {
+          misc[61] = mn;
+          misc[62] = mx;
+        }
       }
+      __syncthreads();
+      hi = misc[62];
+      if (covered >= M) lb = misc[61];
+    } else {
+      // every rank's bound into every CTA (misc[32 + rank]), then one barrier
+      if (tid < NC) cluster.map_shared_rank(misc, tid)[32 + rank] = theta_r;
+      cluster.sync();                                   // bounds published, every ring is free
+      uint32_t mn = 0xFFFFFFFFu;
+#pragma unroll
+      for (int r = 0; r < NC; ++r) mn = min(mn, misc[32 + r]);
       if (covered >= M) lb = mn;
     }
-    // (b) keys >= lb go, in position order, to this rank's segment of CTA 0's
-    //     candidate list; segment sizes to misc0[48 + rank]
+    (void)hi;
+    // (b) keys >= lb go, in position order, to this rank's segment of EVERY
+    //     CTA's candidate list; segment sizes to misc[48 + rank] of every CTA
+    uint32_t *ckl = reinterpret_cast<uint32_t *>(smem + lay.cand_key);
+    int *cpl = reinterpret_cast<int *>(smem + lay.cand_pos);
     {
-      uint32_t *ck = cluster.map_shared_rank(reinterpret_cast<uint32_t *>(smem + lay.cand_key), 0) + rank * SEG;
-      int *cp = cluster.map_shared_rank(reinterpret_cast<int *>(smem + lay.cand_pos), 0) + rank * SEG;
       const int cw = (((cnt + 7) / 8) + 31) & ~31;      // contiguous keys per warp
       const int j0 = min(cnt, warp * cw), j1 = min(cnt, j0 + cw);
       uint32_t wc = 0;
@@ -645,7 +786,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         off += w8 < warp ? c : 0u;
         total += c;
       }
-      if (tid == 0) misc0[48 + rank] = total;
+      if (tid < NC) cluster.map_shared_rank(misc, tid)[48 + rank] = total;
       if (total <= (uint32_t)SEG) {
         const unsigned lt = (1u << lane) - 1u;
         for (int base = j0; base < j1; base += 32) {
@@ -653,9 +794,14 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
           const bool act = j < j1 && keys[j] >= lb;
           const unsigned am = __ballot_sync(0xffffffffu, act);
           if (act) {
-            const uint32_t o = off + __popc(am & lt);
-            ck[o] = keys[j];
-            cp[o] = k0 + j;
+            const uint32_t o = rank * SEG + off + __popc(am & lt);
+            const uint32_t kv = keys[j];
+            const int pv = k0 + j;
+#pragma unroll 4
+            for (int d = 0; d < NC; ++d) {
+              cluster.map_shared_rank(ckl, d)[o] = kv;
+              cluster.map_shared_rank(cpl, d)[o] = pv;
+            }
           }
           off += __popc(am);
         }
@@ -663,7 +809,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     }
     cluster.sync();                                     // candidates complete
     // this CTA's candidates are likely selected: their K and V rows into L2
-    // while CTA 0 selects (after the barrier, which need not wait for them)
+    // while the list is built (after the barrier, which need not wait for them)
     for (int j = tid; j < cnt; j += kDecThreads) {
       if (keys[j] >= lb && k0 + j != t) {
         const size_t row = ((size_t)bg * p.L_max + k0 + j) * D;
@@ -676,133 +822,141 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         }
       }
     }
-    // the same answer in every CTA: lane r of every warp checks rank r's segment
-    const bool fits = __all_sync(0xffffffffu, lane >= NC || misc0[48 + lane] <= (uint32_t)SEG);
+    // the same answer in every CTA: lane r of every warp checks rank r's
+    // segment; the local select holds at most kSelIt candidates per thread
+    uint32_t cnt_l = lane < NC ? misc[48 + lane] : 0u;
+    const bool seg_ok = __all_sync(0xffffffffu, cnt_l <= (uint32_t)SEG);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt_l += __shfl_xor_sync(0xffffffffu, cnt_l, o);
+    constexpr int kSelIt = 4;
+    const bool fits = seg_ok && cnt_l <= (uint32_t)(kSelIt * kDecThreads);
+    local_list = fits;
     if (fits) {
-      if (rank == 0) {
-        // (c) CTA 0: exact M-th key among the candidates (range histograms of
-        //     1024 bins over [lb, hi], narrowed until one bin holds <= 32 keys
-        //     or a single key value), then the ascending index list by an
-        //     ordered compaction of the candidates
-        const uint32_t *ck = reinterpret_cast<const uint32_t *>(smem + lay.cand_key);
-        const int *cp = reinterpret_cast<const int *>(smem + lay.cand_pos);
+      // (c) every CTA, from its own copy of the candidates (the segments
+      //     concatenated in rank order are in position order): the exact M-th
+      //     key K* by an MSB-first radix select over 8-bit digits, then the
+      //     ascending index list by an ordered emission.  Each thread maps its
+      //     candidates c = tid + it * kDecThreads once and keeps them in
+      //     registers; the radix histograms alternate between two buffers.
+      if (tid == 0) {
+        uint32_t a = 0;
+        for (int r = 0; r < NC; ++r) {
+          segp[r] = a;
+          a += misc[48 + r];
+        }
+        segp[NC] = a;
+      }
+      uint32_t *h2 = hist;                              // [2][256]
+      h2[tid] = 0;                                      // 256 threads: the first pass's bins
+      __syncthreads();
+      const int nct = (int)segp[NC];
+      uint32_t cku[kSelIt];
+      int cpp[kSelIt];
+#pragma unroll
+      for (int it = 0; it < kSelIt; ++it) {
+        const int c = tid + it * kDecThreads;
+        cku[it] = 0u;
+        cpp[it] = -1;
+        if (c < nct) {
+          int lo = 0, hi = NC;                          // the segment holding c: segp[lo] <= c < segp[lo + 1]
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if ((int)segp[mid] <= c) lo = mid; else hi = mid;
+          }
+          const int sl = lo * SEG + (c - (int)segp[lo]);
+          cku[it] = ckl[sl];
+          cpp[it] = cpl[sl];
+        }
+      }
+      uint32_t prefix = 0, pmask = 0, rem = (uint32_t)M;
+      bool rok = nct >= M;
+#pragma unroll 1
+      for (int pass = 0; pass < 4 && rok; ++pass) {
+        const int shift = 24 - 8 * pass;
+        uint32_t *hc = h2 + (pass & 1) * 256, *hn = h2 + ((pass + 1) & 1) * 256;
+#pragma unroll
+        for (int it = 0; it < kSelIt; ++it)
+          if (tid + it * kDecThreads < nct && (cku[it] & pmask) == prefix)
+            atomicAdd(&hc[(cku[it] >> shift) & 255u], 1u);
+        __syncthreads();
+        uint32_t *res = misc + 56 + 2 * (pass & 1);    // this pass's bucket and count above it
         if (warp == 0) {
-          const uint32_t v = lane < NC ? misc[48 + lane] : 0u;
-          uint32_t inc = v;
+          uint32_t cb[8], sum = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            cb[j] = hc[255 - (8 * lane + j)];
+            sum += cb[j];
+          }
+          uint32_t inc = sum;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
             if (lane >= o) inc += y;
           }
-          if (lane < NC) segp[lane + 1] = inc;
-          if (lane == 0) segp[0] = 0;
+          const uint32_t exc = inc - sum;
+          const bool here = exc < rem && rem <= inc;
+          if (__ballot_sync(0xffffffffu, here) == 0u) {
+            if (lane == 0) res[0] = 0xFFFFFFFFu;
+          } else if (here) {
+            uint32_t cum = exc;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (cum + cb[j] >= rem) {
+                res[0] = 255u - (uint32_t)(8 * lane + j);
+                res[1] = cum;
+                break;
+              }
+              cum += cb[j];
+            }
+          }
+        } else {
+          hn[tid - 32] = 0;                             // the next pass's bins (warps 1..7, 224 threads)
+          if (tid < 64) hn[224 + tid - 32] = 0;
         }
         __syncthreads();
-        const uint32_t n_c = segp[NC];
-        const uint32_t per = (n_c + kDecThreads - 1) / kDecThreads;
-        const uint32_t c_lo = min(n_c, (uint32_t)tid * per), c_hi = min(n_c, c_lo + per);
-        int r_lo = 0;
+        const uint32_t dg = res[0], above = res[1];
+        if (dg > 255u) {
+          rok = false;                                  // inconsistent counts: cannot happen (uniform)
+          break;
+        }
+        rem -= above;
+        prefix |= dg << shift;
+        pmask |= 255u << shift;
+      }
+      if (!rok) {
+        if (tid == 0) set_err(p.err_word, LISA_DEVERR_CHECK);
+        for (int j = tid; j < M; j += kDecThreads) sel[j] = -1;
+      } else {
+        const uint32_t kstar = prefix, need_eq = rem;
+        uint32_t base_g = 0, base_e = 0;
+        bool bad = false;
+        const int iters = (nct + kDecThreads - 1) / kDecThreads;
 #pragma unroll
-        for (int r = 1; r < NC; ++r) r_lo += segp[r] <= c_lo ? 1 : 0;
-        // candidates c_lo .. c_hi-1 of the concatenation, in order: f(slot)
-        auto for_run = [&](auto &&f) {
-          int r = r_lo;
-          for (uint32_t c = c_lo; c < c_hi; ++c) {
-            while (c >= segp[r + 1]) ++r;
-            f(r * SEG + (int)(c - segp[r]));
-          }
-        };
-        uint32_t lbx = lb, ubx = hi, rem = (uint32_t)M, kstar = 0, need_eq = 0;
-        uint32_t shx = (hi - lb) < 1024u ? 0u : (uint32_t)(32 - __clz(hi - lb)) - 10u;
-        bool found = false;
-#pragma unroll 1
-        for (int iter = 0; iter < 4 && !found; ++iter) {
-          for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
-          __syncthreads();
-          for_run([&](int slot) {
-            const uint32_t u = ck[slot];
-            if (u >= lbx && u <= ubx) atomicAdd(&fh[(u - lbx) >> shx], 1u);
-          });
-          __syncthreads();
-          find_bin1024<kDecThreads>(fh, rem, misc);     // misc[0..2]; zeroes misc[3]
-          const uint32_t bin = misc[0];
-          if (bin > 1023u) break;                       // counts inconsistent: cannot happen
-          rem -= misc[1];
-          const uint32_t cb = misc[2];
-          const uint32_t blo = lbx + (bin << shx);
-          if (shx == 0) {                               // the bin is one key value
-            kstar = blo;
-            need_eq = rem;
-            found = true;
-          } else if (cb <= 32) {                        // rank the bin's keys in one warp
-            for_run([&](int slot) {
-              const uint32_t u = ck[slot];
-              if (u >= blo && u <= ubx && ((u - lbx) >> shx) == bin) {
-                const uint32_t s = atomicAdd(&misc[3], 1u);
-                if (s < 32) tot[s] = u;
-              }
-            });
-            __syncthreads();
-            if (warp == 0) {
-              const uint32_t x = lane < (int)cb ? tot[lane] : 0u;
-              uint32_t gt = 0, ge = 0;
-              for (int j = 0; j < (int)cb; ++j) {
-                const uint32_t y = __shfl_sync(0xffffffffu, x, j);
-                gt += y > x ? 1u : 0u;
-                ge += y >= x ? 1u : 0u;
-              }
-              if (lane < (int)cb && gt < rem && rem <= ge) {   // lanes holding the rem-th key agree
-                misc[5] = x;
-                misc[7] = rem - gt;
-              }
-            }
-            __syncthreads();
-            kstar = misc[5];
-            need_eq = misc[7];
-            found = true;
-          } else {                                      // narrow to the bin
-            const unsigned long long top = (unsigned long long)blo + (1ull << shx) - 1ull;
-            lbx = blo;
-            ubx = top < ubx ? (uint32_t)top : ubx;
-            shx = shx > 10u ? shx - 10u : 0u;
-          }
-          __syncthreads();                              // misc and the histogram are reused
-        }
-        if (!found) {
-          if (tid == 0) set_err(p.err_word, LISA_DEVERR_CHECK);
-          for (int j = tid; j < M; j += kDecThreads) sel[j] = -1;
-        } else {
-          uint32_t cgt = 0, ceq = 0;
-          for_run([&](int slot) {
-            const uint32_t u = ck[slot];
-            cgt += u > kstar ? 1u : 0u;
-            ceq += u == kstar ? 1u : 0u;
-          });
+        for (int it = 0; it < kSelIt; ++it) {
+          if (it >= iters) break;                       // uniform
+          const int c = tid + it * kDecThreads;         // chunk `it` in position order
+          const uint32_t u = cku[it];
+          const int pos = cpp[it];
+          const uint32_t gt = (c < nct && u > kstar) ? 1u : 0u, eq = (c < nct && u == kstar) ? 1u : 0u;
           uint32_t eg, ee, tg, te;
-          cta_scan2<kDecThreads>(cgt, ceq, eg, ee, tg, te, misc);
-          if (tid == 0 && (tg + need_eq != (uint32_t)M || te < need_eq)) set_err(p.err_word, LISA_DEVERR_CHECK);
-          for_run([&](int slot) {
-            const uint32_t u = ck[slot];
-            const int pos = cp[slot];
-            if (pos < 0 || pos >= n) {
-              set_err(p.err_word, LISA_DEVERR_CHECK);
-              return;
-            }
-            if (u > kstar) {
-              const uint32_t o = eg + min(ee, need_eq);
-              if (o < (uint32_t)M) sel[o] = pos;
-              else set_err(p.err_word, LISA_DEVERR_CHECK);
-              ++eg;
-            } else if (u == kstar) {
-              if (ee < need_eq) {
-                const uint32_t o = eg + ee;
-                if (o < (uint32_t)M) sel[o] = pos;
-                else set_err(p.err_word, LISA_DEVERR_CHECK);
-              }
-              ++ee;
-            }
-          });
+          cta_scan2<kDecThreads>(gt, eq, eg, ee, tg, te, misc);
+          const uint32_t pe = base_e + ee;
+          if ((gt || eq) && (pos < 0 || pos >= n)) {
+            bad = true;
+          } else if (gt) {
+            const uint32_t o = base_g + eg + min(pe, need_eq);
+            if (o < (uint32_t)M) sel[o] = pos;
+            else bad = true;
+          } else if (eq && pe < need_eq) {
+            const uint32_t o = base_g + eg + pe;
+            if (o < (uint32_t)M) sel[o] = pos;
+            else bad = true;
+          }
+          base_g += tg;
+          base_e += te;
         }
+        if (base_g + need_eq != (uint32_t)M || base_e < need_eq) bad = true;
+        if (bad) set_err(p.err_word, LISA_DEVERR_CHECK);
       }
     } else {
       // (d) too many keys passed the bound: cluster-wide radix select over all keys
@@ -917,12 +1071,35 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       if (!ok && rank == 0)
         for (int j = tid; j < M; j += kDecThreads) sel[j] = -1;
     }
-  } else if (rank == 0) {
+  } else {
+    if constexpr (WIDE) {
+      if (!wide_arrive()) return;
+    }
     for (int j = tid; j < M; j += kDecThreads) sel[j] = j < n ? j : -1;
   }
-  cluster.sync();                            // CTA 0 holds the full ascending index list
+  // the ascending index list: this CTA's own copy, or CTA 0's after the
+  // cluster-wide radix path (the same answer in every CTA)
+  const int *selp = sel;
+  if (local_list) {
+    __syncthreads();
+  } else {
+    cluster.sync();                          // CTA 0 holds the full ascending index list
+    selp = sel0;
+  }
+  if constexpr (WIDE) {
+    // o_lin of this CTA's output columns: the partial readouts of the CTAs
+    // whose state rows belong to each head, in a fixed order
+    for (int i = tid; i < G * COLS; i += kDecThreads) {
+      const int hh = i / COLS, c = i % COLS;
+      const int w_a = (hh * D) / rps, w_b = min(NSL - 1, ((hh + 1) * D - 1) / rps);
+      float o = 0.f;
+      for (int w = w_a; w <= w_b; ++w)
+        o += __ldcg(p.wpart + (((size_t)bg * NSL + w) * 2 + (hh - (w * rps) / D)) * D + c0s + c);
+      olin[i] = o;
+    }
+  }
   if (rank == 0 && p.idx_out)
-    for (int j = tid; j < M; j += kDecThreads) p.idx_out[(size_t)bg * M + j] = sel[j];
+    for (int j = tid; j < M; j += kDecThreads) p.idx_out[(size_t)bg * M + j] = selp[j];
 
   // The next kernel on the stream may be scheduled from here on: its CTAs
   // wait in their prologue, so a later trigger keeps them from holding SM
@@ -932,7 +1109,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   // ---------------------------------------------------------------- sparse attention (this CTA's rows)
   unsigned char *kvs = ring;                 // [rpc] K rows then [rpc] V rows, stride RS
   for (int r = tid; r < rpc; r += kDecThreads) {
-    int s = sel0[rank * rpc + r];
+    int s = selp[rank * rpc + r];
     if (s < -1 || s > t) {
       set_err(p.err_word, LISA_DEVERR_CHECK);
       s = -1;
@@ -940,6 +1117,10 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     sidx[r] = s;
   }
   __syncthreads();
+  // This CTA no longer reads its candidate lists (nor CTA 0's list): the
+  // other CTAs may write their partials into its shared memory once every
+  // CTA has arrived here (they wait just before those stores).
+  cluster_arrive_release();
   {
     // every 16-byte piece in flight at once (asynchronous copies; rows of
     // unselected slots are zero-filled)
@@ -1093,6 +1274,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   // own shared memory and nobody reads another CTA's memory again
   {
     __syncthreads();                           // part and pml are complete
+    cluster_wait_acquire();                    // every CTA is past its selection
     for (int i = tid; i < G * D; i += kDecThreads) {
       const int hh = i / D, d = i % D, owner = d / COLS, c = d % COLS;
       float *pin_o = cluster.map_shared_rank(reinterpret_cast<float *>(smem + lay.pin), owner);
@@ -1132,11 +1314,11 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
 }
 
 // ============================================================ launcher
-template <typename T, int D, int DI, int NC>
+template <typename T, int D, int DI, int NC, bool WIDE = false>
 static cudaError_t launch_cluster_t(const DecodeParams &p, const CUtensorMap &kmap, cudaStream_t st) {
-  auto kern = decode_cluster_kernel<T, D, DI, NC>;
+  auto kern = decode_cluster_kernel<T, D, DI, NC, WIDE>;
   const DecLayout lay = dec_layout(p.kpc_max, p.L_max, p.M, p.G, D, DI, (int)sizeof(T), NC, p.stages,
-                                   p.stage_keys * ScoreGeom<T, DI>::RB, p.k_lin != nullptr);
+                                   p.stage_keys * ScoreGeom<T, DI>::RB, p.k_lin != nullptr, WIDE);
   cudaError_t e = prepare_kernel(kern, lay.total);
   if (e != cudaSuccess) return e;
   if (NC > 8) {
@@ -1151,7 +1333,7 @@ static cudaError_t launch_cluster_t(const DecodeParams &p, const CUtensorMap &km
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.B * p.Hkv * NC);
+  cfg.gridDim = dim3(p.B * p.Hkv * (WIDE ? p.nw : NC));
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = lay.total;
   cfg.stream = st;
@@ -1219,10 +1401,29 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
     cache_ok16[slot] = ok16;
     cache_sms[slot] = sms;
   }
+  if (p.nw > 0) {
+    // the wide form: nw CTAs (clusters of 8, 2 ring stages) per (b, g); the
+    // last cluster's ranks each take nw / 8 key slices
+    if constexpr (sizeof(T) == 2) {
+      p.nc = 8;
+      p.stages = 2;
+      p.stage_keys = ScoreGeom<T, DI>::sub(32768);
+      p.kpc_max = (p.nw / 8) * ((((p.L_max + p.nw - 1) / p.nw) + 31) & ~31);
+      CUtensorMap kmap;
+      memset(&kmap, 0, sizeof(kmap));
+      using SG = ScoreGeom<T, DI>;
+      if (!make_tmap_2d(&kmap, p.kidx_cache, (int)sizeof(T), (unsigned long long)DI,
+                        (unsigned long long)p.B * p.Hkv * p.L_max, (unsigned long long)SG::RB, DI, p.stage_keys,
+                        SG::RB))
+        return cudaErrorInvalidValue;
+      return launch_cluster_t<T, D, DI, 8, true>(p, kmap, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   // CTAs per (sequence, KV head): 16 keeps one small step short; with many
   // (sequence, KV head) pairs in the launch, fewer CTAs per pair (two per SM)
   // spend less SM time per step.
-  int nc = p.split_req;
+  int nc = p.split_req > 16 ? 16 : p.split_req;   // 32, 64 (the wide form) where it does not apply: 16
   if (nc == 0) {
     const int pairs = p.B * p.Hkv;
     nc = pairs * 16 <= sms ? 16 : pairs * 8 <= 2 * sms ? 8 : 4;
@@ -1248,6 +1449,33 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
   if (nc == 16) return launch_cluster_t<T, D, DI, 16>(p, kmap, st);
   if (nc == 4) return launch_cluster_t<T, D, DI, 4>(p, kmap, st);
   return launch_cluster_t<T, D, DI, 8>(p, kmap, st);
+}
+
+// Workspace of the wide form, sized for nw CTAs per (b, g): arrival counters,
+// per-CTA bounds, per-CTA partial readouts and the order keys (each block
+// 256-byte aligned).
+size_t decode_wide_workspace_bytes(int B, int Hkv, int G, int D, int L_max, int nw) {
+  (void)G;
+  const size_t pairs = (size_t)B * Hkv;
+  auto r256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return r256(pairs * 4) + r256(pairs * nw * 2 * 4) + r256(pairs * nw * 2 * D * 4) +
+         r256(pairs * (size_t)((L_max + 3) & ~3) * 4);
+}
+
+// The library's choice never takes the wide form: measured on a B200 at the
+// 1.5B shape (16K context), one wide step (128 CTAs) took 24-25 us against
+// about 20 us for one 16-CTA cluster, because its publish / arrival / reload
+// steps cost more than the faster key stream saves.  It stays available on
+// request (decode_split 32 or 64).
+int decode_wide_nw(int B, int Hkv, int G, int D, int DI, int dtype, int sms) {
+  (void)B; (void)Hkv; (void)G; (void)D; (void)DI; (void)dtype; (void)sms;
+  return 0;
+}
+
+// Dynamic shared memory of the wide form (bf16; ring stages of at most 32 KB).
+int decode_wide_smem_bytes(int L_max, int M, int G, int D, int DI, int nw) {
+  const int kpc = (nw / 8) * ((((L_max + nw - 1) / nw) + 31) & ~31);
+  return dec_layout(kpc, L_max, M, G, D, DI, 2, 8, 2, kStageBytes, false, true).total;
 }
 
 int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc, bool lin_kv) {

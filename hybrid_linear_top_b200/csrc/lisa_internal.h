@@ -74,6 +74,8 @@ struct DecodeParams {
 size_t decode_wide_workspace_bytes(int B, int Hkv, int G, int D, int L_max, int nw);
 // CTAs per (b, g) the wide form would use for this layer (0: the cluster form).
 int decode_wide_nw(int B, int Hkv, int G, int D, int DI, int dtype, int sms);
+// Dynamic shared memory per CTA of the wide form.
+int decode_wide_smem_bytes(int L_max, int M, int G, int D, int DI, int nw);
 
 // Dynamic shared memory of the decode kernel for a cluster of nc CTAs.
 int decode_smem_bytes(int L_max, int M, int G, int D, int DI, int esize, int nc, bool lin_kv = false);

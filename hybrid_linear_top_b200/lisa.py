@@ -217,8 +217,10 @@ def lisa_workspace_bytes(layer, T, op):
 
 
 def alloc_workspace(layer, T, op, device="cuda"):
+    """Workspace for `op` (zero-filled: the decode step's workspace must start
+    at zero, and every call leaves it ready for the next)."""
     n = lisa_workspace_bytes(layer, T, op)
-    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
 def lisa_append_cache(layer, k, v, kidx, T, stream=None):
@@ -291,7 +293,7 @@ def lisa_workspace_bytes_variant(layer, variant, T, op):
 
 def alloc_workspace_variant(layer, variant, T, op, device="cuda"):
     n = lisa_workspace_bytes_variant(layer, variant, T, op)
-    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
 def lisa_append_cache_variant(layer, variant, k, v, kidx, T, stream=None):

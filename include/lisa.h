@@ -125,13 +125,18 @@ typedef struct {
                         (= tokens already cached) */
   int *err_word;     /* device int or NULL: LISA_DEVERR_* bits are ORed in */
   int decode_split;  /* CTAs that share one (sequence, KV head) in lisa_decode_step:
-                        0 = the library's choice (16 when all of them fit on the
-                        device at once, else 8 or 4), or 4, 8, 16 (16 falls back
-                        to 8 where 16-CTA clusters cannot be scheduled, 4 to 8
-                        where its shared memory would not fit).  16 gives the
-                        shortest single step; 4 the least SM time per step when
-                        many steps run concurrently.  Results do not depend on it
-                        beyond float summation order.  Other calls ignore it. */
+                        4, 8, 16: one thread-block cluster of that size (16 falls
+                        back to 8 where 16-CTA clusters cannot be scheduled, 4 to
+                        8 where its shared memory would not fit);
+                        32, 64: the wide form, that many CTAs in clusters of 8
+                        (bf16 storage and the decode workspace required; the
+                        window and variant forms use 16 instead);
+                        0: the library's choice: 16 when all 16-CTA clusters
+                        fit on the device at once, else 8 or 4 (never the wide
+                        form).  16 gives the shortest single step; 4 the least
+                        SM time per step when many steps run concurrently.
+                        Results do not depend on it beyond float summation
+                        order.  Other calls ignore it. */
   int independent;   /* lisa_decode_step only.  0 (default): the step waits until the
                         launch before it on the stream has finished before it touches
                         memory (it is launched with programmatic dependent launch, so
@@ -186,10 +191,20 @@ LISA_API lisa_status lisa_indexer_topk(const lisa_layer *layer, const void *qidx
  * when fuse_append != 0, also written to cache row t.  With fuse_append == 0
  * the caller must already have stored them there.  The state is updated in
  * place (S <- S + k^T v).  pos is not advanced.
- * The step keeps all intermediates on chip: lisa_workspace_bytes() returns 0
- * for LISA_OP_DECODE and `workspace` may be NULL.  The indexer keys of one
- * (sequence, KV head) live in the shared memory of one thread-block cluster,
- * which bounds L_max to about 280K tokens (LISA_ERR_UNSUPPORTED beyond).
+ * Forms (lisa_layer.decode_split).  In the cluster forms the indexer keys of
+ * one (sequence, KV head) live in the shared memory of one thread-block
+ * cluster, which bounds L_max to about 280K tokens (LISA_ERR_UNSUPPORTED
+ * beyond); `workspace` is not used and may be NULL.  The wide form spreads
+ * the key stream and the state of one (sequence, KV head) over 32 or 64 CTAs,
+ * which publish their order keys, bounds and partial readouts of the linear
+ * branch in the workspace; the last of their clusters to finish selects,
+ * attends and writes the outputs.  It needs
+ * lisa_workspace_bytes(layer, 1, LISA_OP_DECODE) bytes of workspace (0 for
+ * fp32 storage, where the wide form does not apply), zero-filled before its
+ * first use; every call leaves the workspace ready for the next one (its
+ * arrival counters return to zero).  Calls that may run at the same time on
+ * the device (steps declared independent, or steps on different streams)
+ * need workspaces of their own.
  */
 LISA_API lisa_status lisa_decode_step(const lisa_layer *layer, const void *q, const void *k, const void *v,
                              const void *kidx, const void *qidx, const float *w,

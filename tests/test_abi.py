@@ -40,6 +40,8 @@ def _layer(**kw):
     fake = 0x10000  # aligned, never dereferenced: every call below fails validation first
     for name in ["k_cache", "v_cache", "kidx_cache", "state", "pos", "err_word"]:
         setattr(c, name, kw.get(name, fake))
+    for name in ["decode_split", "independent", "debug_flags"]:
+        setattr(c, name, kw.get(name, 0))
     return c
 
 
@@ -88,9 +90,22 @@ def test_decode_rejects_null_and_misaligned_inputs():
     assert _decode(c, out=ctypes.c_void_p(0x20004)) == L.LISA_ERR_INVALID_ARG
 
 
-def test_decode_needs_no_workspace_and_bounds_context():
-    c = _layer()
-    assert L.lisa_workspace_bytes(c, 1, L.LISA_OP_DECODE) == 0
+def test_decode_workspace_is_the_wide_forms_and_context_is_bounded():
+    """The decode workspace holds the wide form's pieces, each rounded to 256
+    bytes and sized for 64 CTAs per (sequence, KV head): arrival counters,
+    per-CTA bound and largest key, per-CTA partial readouts of two heads, and
+    the order keys of every cached position."""
+    r256 = lambda x: (x + 255) // 256 * 256
+    c = _layer(B=3, L_max=1000)
+    pairs, d = 3 * 2, 128
+    want = r256(pairs * 4) + r256(pairs * 64 * 2 * 4) + r256(pairs * 64 * 2 * d * 4) + r256(pairs * 1000 * 4)
+    assert L.lisa_workspace_bytes(c, 1, L.LISA_OP_DECODE) == want
+    assert L.lisa_workspace_bytes(_layer(dtype=L.LISA_FP32), 1, L.LISA_OP_DECODE) == 0
+    # the wide form asked for explicitly needs bf16 storage and the workspace
+    assert _decode(_layer(decode_split=64), ws=None, ws_bytes=0) == L.LISA_ERR_WORKSPACE
+    assert _decode(_layer(decode_split=32), ws_bytes=16) == L.LISA_ERR_WORKSPACE
+    assert _decode(_layer(decode_split=64, dtype=L.LISA_FP32)) == L.LISA_ERR_UNSUPPORTED
+    assert _decode(_layer(decode_split=24)) == L.LISA_ERR_INVALID_ARG
     # keys of one (sequence, KV head) must fit in a cluster's shared memory
     assert _decode(_layer(L_max=1 << 22)) == L.LISA_ERR_UNSUPPORTED
 
@@ -168,7 +183,7 @@ def test_variant_workspace_sizes():
     V1, V2, V3 = L.LISA_VAR_KEY_PER_INDEXER_HEAD, L.LISA_VAR_SHARED_SET, L.LISA_VAR_LINEAR_KV_PER_QUERY_HEAD
     ws = lambda v, T, op: L.lisa_workspace_bytes_variant(c, v, T, op)
     # variant 0 needs what the default calls need
-    assert ws(0, 1, L.LISA_OP_DECODE) == 0
+    assert ws(0, 1, L.LISA_OP_DECODE) == L.lisa_workspace_bytes(c, 1, L.LISA_OP_DECODE)
     assert ws(0, 300, L.LISA_OP_PREFILL) == L.lisa_workspace_bytes(c, 300, L.LISA_OP_PREFILL)
     assert ws(0, 7, L.LISA_OP_INDEXER_TOPK) == L.lisa_workspace_bytes(c, 7, L.LISA_OP_INDEXER_TOPK)
     # the linear branch's own k / v alone keeps the fused decode kernel
@@ -231,9 +246,10 @@ def test_variant_workspace_formula():
         r256(Hkv * Lk * 4) + r256(HI * Lk * 4) + r256(Hkv * M * 4))
     # prefill: keys [Gs][T][T] + idx [T][Gs][M] + o_lin [T][Hq][d] + dS [LH][chunks][d][d] + total [LH][d][d]
     nc = (T + 63) // 64
-    for v, Gs, LH, per_head in [(0, Hkv, Hkv, False), (V2, 1, Hkv, False), (V3, Hkv, Hq, False),
-                                (V1 | V2, 1, Hkv, True)]:
+    for v, Gs, LH, per_head in [(V2, 1, Hkv, False), (V3, Hkv, Hq, False), (V1 | V2, 1, Hkv, True)]:
         want = (r256(Gs * T * T * 4) + (r256(HI * T * T * 4) if per_head else 0) + r256(T * Gs * M * 4) +
                 r256(T * Hq * d * 4) + r256(LH * nc * d * d * 4) + r256(LH * d * d * 4))
         assert L.lisa_workspace_bytes_variant(c, v, T, L.LISA_OP_PREFILL) == want, v
+    # variant 0 runs the default calls: their workspace
+    assert L.lisa_workspace_bytes_variant(c, 0, T, L.LISA_OP_PREFILL) == L.lisa_workspace_bytes(c, T, L.LISA_OP_PREFILL)
     assert B == 1

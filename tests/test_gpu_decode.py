@@ -73,10 +73,11 @@ def run_decode(cfg, layer_np, step, pos, L_max, fuse_append=True, pre_append=Fal
     return dict(ndiff=ndiff, errs=errs, lay=lay)
 
 
-@pytest.mark.parametrize("split", [0, 4, 8, 16])
+@pytest.mark.parametrize("split", [0, 4, 8, 16, 32, 64])
 def test_decode_1p5b_16k(split):
     """Full-size single-layer decode step at 16384 cached tokens, for every
-    CTA split of a (sequence, KV head)."""
+    CTA split of a (sequence, KV head): the cluster forms (4, 8, 16; the
+    library's choice 0 is 16 here) and the wide form (32, 64)."""
     cfg = get_config("decode_1p5b_16k")
     rng = make_rng(cfg.seed, 0)
     lay = gen_layer(cfg, rng, cfg.L - 1)
@@ -85,7 +86,7 @@ def test_decode_1p5b_16k(split):
     run_decode(cfg, lay, step, pos, cfg.L_max, split=split)
 
 
-@pytest.mark.parametrize("split", [0, 16])
+@pytest.mark.parametrize("split", [0, 16, 32])
 def test_decode_7b_ragged_batch(split):
     """B=32 ragged lengths in [4096, 16384] (the library's choice is 4 CTAs per
     (sequence, KV head) here)."""
@@ -98,7 +99,7 @@ def test_decode_7b_ragged_batch(split):
     run_decode(cfg, lay, step, pos, cfg.L_max, n_rows=cfg.L_hi - 1, split=split)
 
 
-@pytest.mark.parametrize("split", [0, 4])
+@pytest.mark.parametrize("split", [0, 4, 64])
 @pytest.mark.parametrize("L_ctx", [1, 2, 100, 255, 256, 257, 300, 4097])
 def test_decode_short_prefixes(L_ctx, split):
     """Prefixes around M (all kept, exactly M, M+1) and t = 0."""
@@ -155,7 +156,7 @@ def test_decode_other_shapes(dtype, d, dI, split):
     run_decode(cfg, lay, step, np.array([1499, 700]), 1500, split=split)
 
 
-@pytest.mark.parametrize("split", [4, 16])
+@pytest.mark.parametrize("split", [4, 16, 64])
 def test_decode_largest_groups_and_m(split):
     """16 query heads and 8 indexer heads per KV head, M = 1024 (the largest
     supported values)."""
@@ -249,7 +250,7 @@ def test_decode_graph_replays_are_stable():
     torch.cuda.synchronize()
 
 
-@pytest.mark.parametrize("split", [0, 4, 8])
+@pytest.mark.parametrize("split", [0, 4, 8, 32])
 @pytest.mark.parametrize("L_ctx", [16384, 3000])
 def test_decode_all_scores_equal(L_ctx, split):
     """w = 0 makes every score 0: the first M positions must be selected (the
@@ -293,7 +294,7 @@ def test_decode_inputs_and_output_in_pinned_host_memory():
     check_state(f64(lay.state), ref["S"], where="state")
 
 
-@pytest.mark.parametrize("split", [0, 4])
+@pytest.mark.parametrize("split", [0, 4, 32])
 def test_decode_long_context_100k(split):
     """100 000 cached tokens: per-CTA key slices of 6-25K keys, candidate
     segments and the exact select at a long context."""
@@ -304,19 +305,21 @@ def test_decode_long_context_100k(split):
     run_decode(cfg, lay, step, np.array([99999]), 100000, split=split)
 
 
-def test_decode_bench_launch_configuration():
+@pytest.mark.parametrize("split", [4, 64])
+def test_decode_bench_launch_configuration(split):
     """The headline workload in the launch configuration the bench times:
     full-size instances (16384 cached tokens, 1.5B shape), one stream, every
     step declared independent of the launch before it, captured in a CUDA
-    graph and replayed, the bench's CTA split.  Every instance's set, output,
-    state and appended row are checked against the oracle on the instance's
-    own data (read back from the device)."""
+    graph and replayed, each instance with a workspace of its own; the
+    cluster form with 4 CTAs and the wide form with 64.  Every instance's
+    set, output, state and appended row are checked against the oracle on
+    the instance's own data (read back from the device)."""
     import bench
     cfg = get_config("decode_1p5b_16k")
     rng = make_rng(cfg.seed, 0)
     exact = (gen_layer(cfg, rng, cfg.L - 1), gen_step(cfg, rng, 1))
     R = 6
-    inst = [bench.Instance(L, cfg, torch, 77 + i, exact if i == 0 else None, 4) for i in range(R)]
+    inst = [bench.Instance(L, cfg, torch, 77 + i, exact if i == 0 else None, split) for i in range(R)]
     for x in inst:
         x.lay.independent = 1
     n = cfg.L - 1
@@ -325,7 +328,7 @@ def test_decode_bench_launch_configuration():
                    S=a(x.lay.state)) for x in inst]
     stream = torch.cuda.Stream()
     per, n_full, tail = bench.plan_graphs(R, R)
-    g = bench._capture(torch, stream, [stream], [inst[i % R] for i in range(per)], lambda x, s_: x.step(L, None, s_))
+    g = bench._capture(torch, stream, [stream], [inst[i % R] for i in range(per)], lambda x, s_: x.step(L, x.ws, s_))
     g.replay()
     torch.cuda.synchronize()
     for i, x in enumerate(inst):

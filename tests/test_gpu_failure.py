@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 L = pytest.importorskip("hybrid_linear_top_b200.lisa")
 
 
-@pytest.mark.parametrize("split", [4, 8, 16])
+@pytest.mark.parametrize("split", [4, 8, 16, 64])
 def test_forced_timeout_then_normal_call(split):
     import dataclasses
     cfg = dataclasses.replace(get_config("decode_1p5b_16k"), B=2, L=2048)
@@ -41,9 +41,10 @@ def test_forced_timeout_then_normal_call(split):
     idx = torch.full((cfg.B, cfg.Hkv, cfg.M), -7, dtype=torch.int32, device="cuda")
     S_in = lay.state.clone()
     k_before = lay.k_cache.clone()
+    ws = L.alloc_workspace(lay, 1, L.LISA_OP_DECODE)    # used by the wide form (split 64)
 
     lay.debug_flags = L.LISA_DEBUG_FORCE_TIMEOUT
-    L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, out, idx, None)
+    L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, out, idx, ws)
     torch.cuda.synchronize()
     assert int(lay.err_word.item()) == L.LISA_DEVERR_TIMEOUT
     assert torch.isnan(out.float()).all(), "output written after the timeout"
@@ -54,7 +55,7 @@ def test_forced_timeout_then_normal_call(split):
     # the next normal call on the same layer is correct
     lay.debug_flags = 0
     lay.err_word.zero_()
-    L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, out, idx, None)
+    L.lisa_decode_step(lay, x["q"], x["k"], x["v"], x["kidx"], x["qidx"], x["w"], x["lam"], 1, out, idx, ws)
     torch.cuda.synchronize()
     assert int(lay.err_word.item()) == 0
     a = lambda z: z.astype(np.float64)

@@ -99,6 +99,70 @@ def test_prefill_1p5b_shape_small(T):
     check_prefill(cfg, layer_np, step, lay, out, idx)
 
 
+def _integer_indexer(step, seed):
+    """Small-integer indexer inputs (exact in bf16, exact fp32 sums): exact score ties."""
+    ir = np.random.default_rng(seed)
+    step.kidx = ir.integers(-1, 2, size=step.kidx.shape).astype(np.float32)
+    step.qidx = ir.integers(-1, 2, size=step.qidx.shape).astype(np.float32)
+    step.w = ir.integers(0, 3, size=step.w.shape).astype(np.float32)
+    return step
+
+
+def test_prefill_exact_ties_integer_inputs():
+    """Exact score ties in every row (integer indexer inputs): the selected sets
+    must equal the oracle's with no borderline exemption (tie -> lower
+    position), through the two-pass select's kept keys, bounds and candidates,
+    over two row passes and rows longer and shorter than the bound needs."""
+    T = 5000
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=T, S0="normal")
+    rng = make_rng(230, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = _integer_indexer(gen_step(cfg, rng, T), 5)
+    lay, out, idx = gpu_prefill(cfg, layer_np, step, T, T)
+    rows = [0, 255, 256, 257, 2047, 2048, 3000, 4095, 4096, 4999]
+    a = lambda z: z.astype(np.float64)
+    idx_g = idx.cpu().numpy().astype(np.int64)
+    for t in rows:
+        keys = np.transpose(a(step.kidx[0, :t + 1]), (1, 0, 2))
+        sc = oracle.indexer_scores(a(step.qidx[0, t]), a(step.w[0, t]), keys)
+        for g in range(cfg.Hkv):
+            check_set(idx_g[0, t, g], sc[g], cfg.M, t, exact=True, where=f"t={t} g={g}")
+    check_prefill(cfg, layer_np, step, lay, out, idx, rows=rows)
+
+
+def test_prefill_all_scores_equal():
+    """w = 0: every score is 0, so every key of a row ties with the M-th and is
+    a candidate (more than the select stages in shared memory for the long
+    rows); the first M positions must be selected."""
+    T = 6000
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=T)
+    rng = make_rng(231, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = gen_step(cfg, rng, T)
+    step.w = np.zeros_like(step.w)
+    lay, out, idx = gpu_prefill(cfg, layer_np, step, T, T)
+    idx_g = idx.cpu().numpy()
+    for t in [0, 255, 256, 300, 4095, 4500, 5999]:
+        want = np.full(cfg.M, -1)
+        n = min(cfg.M, t + 1)
+        want[:n] = np.arange(n)
+        for g in range(cfg.Hkv):
+            np.testing.assert_array_equal(idx_g[0, t, g], want, err_msg=f"t={t} g={g}")
+    check_prefill(cfg, layer_np, step, lay, out, idx, rows=[0, 256, 4500, 5999])
+
+
+def test_prefill_largest_m():
+    """M = 1024 with two indexer heads per KV head: most rows have fewer kept
+    keys than M, so every key is a candidate (bound 0)."""
+    T = 3000
+    cfg = dataclasses.replace(get_config("prefill_1p5b_16k"), T=T, M=1024, S0="normal")
+    rng = make_rng(232, 0)
+    layer_np = gen_layer(cfg, rng, 0)
+    step = gen_step(cfg, rng, T)
+    lay, out, idx = gpu_prefill(cfg, layer_np, step, T, T)
+    check_prefill(cfg, layer_np, step, lay, out, idx, rows=[0, 1023, 1024, 1025, 2047, 2999])
+
+
 @pytest.mark.slow
 def test_prefill_1p5b_16k_sampled():
     """Full 16384-token prefill; outputs and sets checked on sampled rows,
