@@ -380,10 +380,12 @@ __global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
 // ------------------------------------------------------------ bf16 on warp MMAs
 // grid (T, B*Hkv); 4 warps.  Warp w owns selected rows [w*M/4, (w+1)*M/4) of
 // the (b, tau, g) list, in tiles of 16 rows staged by cp.async (two stages per
-// warp), flash-attention style: S = Q K^T with the G query heads as the 16 rows
-// of the A operand, online softmax in registers, O += P V with P as bf16
-// hi + lo pairs.  The 4 warps' (max, sum, O) are merged through shared memory,
-// then the gate mixes in o_lin.
+// warp), flash-attention style with the selected rows as the M dimension of
+// the warp MMAs and the G query heads as the N dimension (NHT tiles of 8
+// heads): S^T = K Q^T, online softmax per head in registers, O^T += V^T P^T
+// with P^T moved from the accumulator layout into the B-operand layout by 8x8
+// transposes (movmatrix), P in bf16.  The 4 warps' (max, sum, O) are merged
+// through shared memory, then the gate mixes in o_lin.
 constexpr int kAttnWarps = 4;
 
 
@@ -393,18 +395,26 @@ constexpr int attn_mma_smem() {
   return kAttnWarps * 2 * 2 * 16 * (2 * D + 16);
 }
 
-template <int D>
+// An 8x8 b16 matrix held one row pair per lane (lane l: row l / 4, columns
+// 2 (l % 4), +1) -> its transpose in the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+template <int D, int NHT>
 __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(RowsParams p) {
   extern __shared__ __align__(16) unsigned char s_att[];
   constexpr int RS = 2 * D + 16;                 // padded row stride (bytes)
   constexpr int TILE = 16 * RS;                  // one 16-row K or V tile
-  constexpr int NT = D / 8;                      // 8-column output tiles
+  constexpr int MT = D / 16;                     // 16-row tiles of O^T (head dim)
   const int tau = blockIdx.x, bg = blockIdx.y;
   const int g = bg % p.Hkv, b = bg / p.Hkv;
   if (!rows_pos_ok(p, b)) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G;
-  const int g4 = lane >> 2, t2 = (lane & 3) * 2;
+  const int hl = lane >> 2, kq = (lane & 3) * 2;
   const int RW = p.M / kAttnWarps;               // rows of this warp (a multiple of 16)
   const int t_abs = p.pos[b] + tau;
   unsigned char *wbuf = s_att + warp * 4 * TILE; // [stage][K | V]
@@ -413,18 +423,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
   const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(p.k_cache) + (size_t)bg * p.L_max * D;
   const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(p.v_cache) + (size_t)bg * p.L_max * D;
 
-  // A fragments of q (heads = rows, padded to 16), for every 16-wide k-step
-  uint32_t qa[D / 16][4];
+  // B fragments of Q^T (k = head dim, n = query head) for every 16-wide k-step
+  uint32_t qb[NHT][D / 16][2];
   {
     const uint32_t *q32 = reinterpret_cast<const uint32_t *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
                                                              (((size_t)b * p.T + tau) * p.Hq + g * G) * D);
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const int k0 = ks * 16 + t2;
-      qa[ks][0] = g4 < G ? q32[(g4 * D + k0) >> 1] : 0u;
-      qa[ks][1] = g4 + 8 < G ? q32[((g4 + 8) * D + k0) >> 1] : 0u;
-      qa[ks][2] = g4 < G ? q32[(g4 * D + k0 + 8) >> 1] : 0u;
-      qa[ks][3] = g4 + 8 < G ? q32[((g4 + 8) * D + k0 + 8) >> 1] : 0u;
+    for (int nh = 0; nh < NHT; ++nh) {
+      const int h = nh * 8 + hl;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        qb[nh][ks][0] = h < G ? q32[(h * D + ks * 16 + kq) >> 1] : 0u;
+        qb[nh][ks][1] = h < G ? q32[(h * D + ks * 16 + kq + 8) >> 1] : 0u;
+      }
     }
   }
   // rows of tile i: positions (or -1), lanes 0..15 hold one each
@@ -453,10 +464,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
     cp_async_commit();
   };
 
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads g4 and g4 + 8
-  float o[NT][4];
+  // this lane: heads nh * 8 + kq, + 1 of every n-tile; rows hl and hl + 8 of a tile
+  float mh[NHT][2], lh[NHT][2];
+  float o[NHT][MT][4];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  for (int nh = 0; nh < NHT; ++nh) {
+    mh[nh][0] = mh[nh][1] = -INFINITY;
+    lh[nh][0] = lh[nh][1] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) o[nh][mt][0] = o[nh][mt][1] = o[nh][mt][2] = o[nh][mt][3] = 0.f;
+  }
 
   const int ntiles = RW / 16;
   int pos_cur = tile_pos(0);
@@ -479,106 +496,95 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
     }
     __syncwarp();
     const uint32_t kt = wbuf_u32 + (i & 1) * 2 * TILE, vt = kt + TILE;
-    // S = Q K^T for 16 rows (two 8-row n-tiles)
-    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    // S^T = K Q^T: 16 rows x 8 heads per n-tile
+    float sc[NHT][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nh = 0; nh < NHT; ++nh) sc[nh][0] = sc[nh][1] = sc[nh][2] = sc[nh][3] = 0.f;
 #pragma unroll
-      for (int ks2 = 0; ks2 < D / 32; ++ks2) {
-        uint32_t bk[4];
-        ldmatrix_x4(kt + (nt * 8 + (lane & 7)) * RS + ks2 * 64 + (lane >> 3) * 16, bk[0], bk[1], bk[2], bk[3]);
-        mma_16816_bf16(sc[nt], qa[2 * ks2], bk);
-        mma_16816_bf16(sc[nt], qa[2 * ks2 + 1], bk + 2);
-      }
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a[4];
+      ldmatrix_x4(kt + (lane & 15) * RS + ks * 32 + (lane >> 4) * 16, a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int nh = 0; nh < NHT; ++nh) mma_16816_bf16(sc[nh], a, qb[nh][ks]);
     }
-    // scale, mask, online softmax (rows g4 and g4 + 8; a quad holds 16 columns)
-    float mt0 = -INFINITY, mt1 = -INFINITY;
+    const int pr0 = __shfl_sync(0xffffffffu, pos_cur, hl), pr1 = __shfl_sync(0xffffffffu, pos_cur, hl + 8);
+    uint32_t pb[NHT][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nh = 0; nh < NHT; ++nh) {
+      // scale, mask; c0, c1: row hl (heads kq, kq + 1); c2, c3: row hl + 8
+      float x[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = nt * 8 + t2 + (j & 1);
-        const int s = __shfl_sync(0xffffffffu, pos_cur, r);
-        const float x = s >= 0 ? sc[nt][j] * p.scale : -INFINITY;
-        sc[nt][j] = x;
-        if (j < 2) mt0 = fmaxf(mt0, x);
-        else mt1 = fmaxf(mt1, x);
+      for (int j = 0; j < 4; ++j) x[j] = (j < 2 ? pr0 : pr1) >= 0 ? sc[nh][j] * p.scale : -INFINITY;
+      // the heads' maxima over the tile's 16 rows (lanes with the same lane % 4)
+      float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
       }
-    mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 1));
-    mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 2));
-    mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 1));
-    mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 2));
-    const float mn0 = fmaxf(m0, mt0), mn1 = fmaxf(m1, mt1);
-    const float f0 = m0 == -INFINITY ? 0.f : expf(m0 - mn0);
-    const float f1 = m1 == -INFINITY ? 0.f : expf(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    float e[2][4];
+      const float mn0 = fmaxf(mh[nh][0], mx0), mn1 = fmaxf(mh[nh][1], mx1);
+      const float f0 = mh[nh][0] == -INFINITY ? 0.f : expf(mh[nh][0] - mn0);
+      const float f1 = mh[nh][1] == -INFINITY ? 0.f : expf(mh[nh][1] - mn1);
+      mh[nh][0] = mn0;
+      mh[nh][1] = mn1;
+      const float e0 = x[0] == -INFINITY ? 0.f : expf(x[0] - mn0);
+      const float e1 = x[1] == -INFINITY ? 0.f : expf(x[1] - mn1);
+      const float e2 = x[2] == -INFINITY ? 0.f : expf(x[2] - mn0);
+      const float e3 = x[3] == -INFINITY ? 0.f : expf(x[3] - mn1);
+      lh[nh][0] = lh[nh][0] * f0 + e0 + e2;
+      lh[nh][1] = lh[nh][1] * f1 + e1 + e3;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float mm = j < 2 ? mn0 : mn1;
-        e[nt][j] = sc[nt][j] == -INFINITY ? 0.f : expf(sc[nt][j] - mm);
+      for (int mt = 0; mt < MT; ++mt) {
+        o[nh][mt][0] *= f0;
+        o[nh][mt][1] *= f1;
+        o[nh][mt][2] *= f0;
+        o[nh][mt][3] *= f1;
       }
-    l0 = l0 * f0 + e[0][0] + e[0][1] + e[1][0] + e[1][1];
-    l1 = l1 * f1 + e[0][2] + e[0][3] + e[1][2] + e[1][3];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      o[j][0] *= f0;
-      o[j][1] *= f0;
-      o[j][2] *= f1;
-      o[j][3] *= f1;
+      // P^T (k = rows, n = heads) as the B operand: transposes of the two 8x8 blocks
+      pb[nh][0] = movmatrix_trans(pack_bf16(e0, e1));
+      pb[nh][1] = movmatrix_trans(pack_bf16(e2, e3));
     }
-    // P as the A operand of a 16-row k-step: hi + lo bf16 pairs
-    uint32_t ph[4], pl[4];
-    {
-      const float pv[4][2] = {{e[0][0], e[0][1]}, {e[0][2], e[0][3]}, {e[1][0], e[1][1]}, {e[1][2], e[1][3]}};
+    // O^T += V^T P^T: A = V^T (head dim x rows) by transposing matrix loads
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        ph[j] = pack_bf16(pv[j][0], pv[j][1]);
-        const float h0 = __bfloat162float(__float2bfloat16_rn(pv[j][0]));
-        const float h1 = __bfloat162float(__float2bfloat16_rn(pv[j][1]));
-        pl[j] = pack_bf16(pv[j][0] - h0, pv[j][1] - h1);
-      }
-    }
-    // O += P V
+    for (int mt = 0; mt < MT; ++mt) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(vt + ((lane & 7) + 8 * (lane >> 4)) * RS + (mt * 16 + 8 * ((lane >> 3) & 1)) * 2, a[0], a[1],
+                        a[2], a[3]);
 #pragma unroll
-    for (int np = 0; np < NT / 2; ++np) {
-      uint32_t bv[4];
-      const int mm = lane >> 3;
-      ldmatrix_x4_trans(vt + ((mm & 1) * 8 + (lane & 7)) * RS + (np * 16 + (mm >> 1) * 8) * 2, bv[0], bv[1], bv[2],
-                        bv[3]);
-      mma_16816_bf16(o[2 * np], ph, bv);
-      mma_16816_bf16(o[2 * np], pl, bv);
-      mma_16816_bf16(o[2 * np + 1], ph, bv + 2);
-      mma_16816_bf16(o[2 * np + 1], pl, bv + 2);
+      for (int nh = 0; nh < NHT; ++nh) mma_16816_bf16(o[nh][mt], a, pb[nh]);
     }
     __syncwarp();                                  // this stage may be refilled next
     pos_cur = pos_next;
   }
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+#pragma unroll
+  for (int nh = 0; nh < NHT; ++nh)
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      lh[nh][0] += __shfl_xor_sync(0xffffffffu, lh[nh][0], off);
+      lh[nh][1] += __shfl_xor_sync(0xffffffffu, lh[nh][1], off);
+    }
 
   // merge the warps: [warp][16 heads] max and sum, [warp][16][D] O
   __syncthreads();
   float *s_ml = reinterpret_cast<float *>(s_att);                 // [4][16][2]
   float *s_o = s_ml + kAttnWarps * 32;                            // [4][16][D]
-  if ((lane & 3) == 0) {
-    s_ml[(warp * 16 + g4) * 2] = m0;
-    s_ml[(warp * 16 + g4) * 2 + 1] = l0;
-    s_ml[(warp * 16 + g4 + 8) * 2] = m1;
-    s_ml[(warp * 16 + g4 + 8) * 2 + 1] = l1;
-  }
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    const int d = j * 8 + t2;
-    s_o[(warp * 16 + g4) * D + d] = o[j][0];
-    s_o[(warp * 16 + g4) * D + d + 1] = o[j][1];
-    s_o[(warp * 16 + g4 + 8) * D + d] = o[j][2];
-    s_o[(warp * 16 + g4 + 8) * D + d + 1] = o[j][3];
+  for (int nh = 0; nh < NHT; ++nh) {
+    const int h0 = nh * 8 + kq;
+    if (lane < 4) {
+      s_ml[(warp * 16 + h0) * 2] = mh[nh][0];
+      s_ml[(warp * 16 + h0) * 2 + 1] = lh[nh][0];
+      s_ml[(warp * 16 + h0 + 1) * 2] = mh[nh][1];
+      s_ml[(warp * 16 + h0 + 1) * 2 + 1] = lh[nh][1];
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int d = mt * 16 + hl;
+      s_o[(warp * 16 + h0) * D + d] = o[nh][mt][0];
+      s_o[(warp * 16 + h0 + 1) * D + d] = o[nh][mt][1];
+      s_o[(warp * 16 + h0) * D + d + 8] = o[nh][mt][2];
+      s_o[(warp * 16 + h0 + 1) * D + d + 8] = o[nh][mt][3];
+    }
   }
   __syncthreads();
   for (int i = tid; i < G * D; i += kAttnWarps * 32) {
@@ -606,16 +612,18 @@ cudaError_t launch_prefill_attend(const RowsParams &p, int dtype, cudaStream_t s
   dim3 grid(p.T, p.B * p.Hkv);
   cudaError_t e;
   if (dtype == LISA_BF16 && p.M % (16 * kAttnWarps) == 0) {
-    if (p.D == 128) {
-      constexpr int smem = attn_mma_smem<128>();
-      if ((e = prepare_kernel(prefill_attend_mma_kernel<128>, smem)) != cudaSuccess) return e;
-      prefill_attend_mma_kernel<128><<<grid, kAttnWarps * 32, smem, st>>>(p);
-    } else {
-      constexpr int smem = attn_mma_smem<64>();
-      if ((e = prepare_kernel(prefill_attend_mma_kernel<64>, smem)) != cudaSuccess) return e;
-      prefill_attend_mma_kernel<64><<<grid, kAttnWarps * 32, smem, st>>>(p);
-    }
-    return cudaGetLastError();
+    // query heads of a group as the MMAs' N: one n-tile of 8 heads, or two
+    auto go = [&](auto kern, int smem) -> cudaError_t {
+      cudaError_t e2 = prepare_kernel(kern, smem);
+      if (e2 != cudaSuccess) return e2;
+      kern<<<grid, kAttnWarps * 32, smem, st>>>(p);
+      return cudaGetLastError();
+    };
+    if (p.D == 128)
+      return p.G <= 8 ? go(prefill_attend_mma_kernel<128, 1>, attn_mma_smem<128>())
+                      : go(prefill_attend_mma_kernel<128, 2>, attn_mma_smem<128>());
+    return p.G <= 8 ? go(prefill_attend_mma_kernel<64, 1>, attn_mma_smem<64>())
+                    : go(prefill_attend_mma_kernel<64, 2>, attn_mma_smem<64>());
   }
   if (dtype == LISA_BF16) {
     if (p.D == 128) {
