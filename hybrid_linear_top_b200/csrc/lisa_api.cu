@@ -226,7 +226,6 @@ lisa_status plan_decode_form(const lisa_layer *L, void *workspace, size_t ws_byt
   char *ws = static_cast<char *>(workspace);
   size_t off = 0;
   p.wcount = reinterpret_cast<unsigned *>(ws + off); off += round256(pairs * 4);
-  p.wtheta = reinterpret_cast<uint32_t *>(ws + off); off += round256(pairs * 64 * 2 * 4);
   p.wpart = reinterpret_cast<float *>(ws + off); off += round256(pairs * 64 * 2 * L->d * 4);
   p.wkeys = reinterpret_cast<uint32_t *>(ws + off);
   p.wkeys_stride = round4(L->L_max);

@@ -43,7 +43,6 @@ namespace lisa {
 constexpr int kDecThreads = 256;
 constexpr int kStages = 4;        // ring stages at most (the launcher picks 2 or 4)
 constexpr int kStageBytes = 32768;  // ring stage size at most (the launcher picks 16 or 32 KB)
-constexpr int kCandCap = 4096;   // candidate (key, position) pairs CTA 0 can hold
 
 template <typename T, int DI>
 struct ScoreGeom {
@@ -54,18 +53,30 @@ struct ScoreGeom {
 };
 
 struct DecLayout {
-  int region0, cand_key, cand_pos, pin;
-  int keys, hist, tot, misc, sel, qs, qi, ks, vs, kis, gl, klin, vlin, part, pml, olin, logit, sidx, wred, bars, total;
+  int region0, xin, pout, pin;
+  int keys, hist, tot, misc, sel, qs, qi, ks, vs, kis, gl, klin, vlin, olin, logit, sidx, wred, bars, total;
 };
+
+// Candidate slots each CTA of an NC-CTA cluster sends in the top-M exchange:
+// 1024 over the cluster, but 128 each for 4 CTAs (two such CTAs share an SM).
+__host__ __device__ constexpr int dec_seg(int NC) { return NC <= 4 ? 128 : 1024 / NC; }
+// Words of one candidate message: a 4-word header (bound, largest key, send
+// threshold, count) and dec_seg(NC) keys and positions.
+__host__ __device__ constexpr int dec_msg_words(int NC) { return 4 + 2 * dec_seg(NC); }
+// Floats of one merge message: a sender's partial outputs of the G heads on
+// the receiver's D / NC columns, then its G (max, sum) pairs; 16-byte multiple.
+__host__ __device__ constexpr int dec_merge_words(int G, int D, int NC) { return (G * (D / NC) + 2 * G + 3) & ~3; }
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 
 // Byte offsets of the dynamic shared-memory carve-up, relative to a
 // 1024-byte aligned base (host and device agree; `total` includes the slack
-// needed to align the base).  region0 holds, one after the other in time: the
-// TMA ring (scoring), the candidate segments (selection, in CTA 0), and the
-// gathered K / V rows (attention) followed by the partials that every rank
-// writes for this CTA's output columns (merge).
+// needed to align the base).  region0 holds the TMA ring (scoring), later the
+// gathered K / V rows (attention) followed by the merge messages (pout: this
+// CTA's, pin: the other CTAs').  Another CTA writes into pin only after it
+// has this CTA's candidate message, which is sent after the last ring stage
+// is consumed; candidate messages (xin) arrive while this CTA may still be
+// scoring, so they have a region of their own.
 __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, int G, int D, int DI, int esize,
                                                 int NC, int stages = kStages, int stage_bytes = kStageBytes,
                                                 bool lin_kv = false, bool wide = false) {
@@ -73,15 +84,14 @@ __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, i
   const int rpc = M / NC;
   const int kv = 2 * rpc * (D * esize + 16);
   const int ring = stages * stage_bytes;
-  const int sel_bytes = 8 * kCandCap;
-  const int kvp = align16(kv) + G * D * 4 + NC * 2 * G * 4;   // + [NC][G][D/NC] partials, [NC][2G] statistics
-  int r0 = ring > kvp ? ring : kvp;
-  r0 = r0 > sel_bytes ? r0 : sel_bytes;
+  const int mw = dec_merge_words(G, D, NC);
+  const int kvm = align16(kv) + 2 * NC * mw * 4;      // K / V rows, then [NC][mw] pout and [NC][mw] pin
+  const int r0 = ring > kvm ? ring : kvm;
   int off = 0;
   L.region0 = off; off += align16(r0);
-  L.cand_key = L.region0;
-  L.cand_pos = L.region0 + 4 * kCandCap;
-  L.pin = L.region0 + align16(kv);
+  L.pout = L.region0 + align16(kv);                   // [NC owners] this CTA's merge messages
+  L.pin = L.pout + NC * mw * 4;                       // [NC senders] merge messages for this CTA's columns
+  L.xin = off; off += NC * dec_msg_words(NC) * 4;     // [NC senders] candidate messages (own in slot rank)
   L.keys = off; off += align16(kpc_max * 4);
   L.hist = off; off += 8 * 256 * 4;
   L.tot = off; off += 256 * 4;
@@ -95,8 +105,6 @@ __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, i
   L.gl = off; off += align16(G * 4);
   L.klin = off; off += lin_kv ? align16(G * D * 4) : 0;   // linear-branch k, v per query head (variant)
   L.vlin = off; off += lin_kv ? align16(G * D * 4) : 0;
-  L.part = off; off += align16(G * D * 4);
-  L.pml = off; off += align16(2 * G * 4);
   L.olin = off; off += align16(G * (D / NC) * 4);
   {
     const int a = G * rpc * 4, bred = 8 * 8 * (D / NC) * 4;   // logits, or the o_lin reduction scratch
@@ -104,7 +112,7 @@ __host__ __device__ inline DecLayout dec_layout(int kpc_max, int L_max, int M, i
   }
   L.sidx = off; off += align16(rpc * 4);
   L.wred = off; off += wide ? align16(2 * 8 * D * 4) : 0;   // wide form: [2 heads][8 warps][D] readout sums
-  L.bars = off; off += kStages * 8;
+  L.bars = off; off += (kStages + 2) * 8;             // ring stages, candidate messages, merge messages
   L.total = align16(off) + 1024;
   return L;
 }
@@ -194,17 +202,25 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   float *gls = reinterpret_cast<float *>(smem + lay.gl);    // gate logits of the G heads
   float *klin = reinterpret_cast<float *>(smem + lay.klin); // [G][D] (variant only)
   float *vlin = reinterpret_cast<float *>(smem + lay.vlin); // [G][D] (variant only)
-  float *part = reinterpret_cast<float *>(smem + lay.part);
-  float *pml = reinterpret_cast<float *>(smem + lay.pml);
+  const int MW = dec_merge_words(G, D, NC);            // floats per merge message
+  float *pout = reinterpret_cast<float *>(smem + lay.pout);   // [NC owners][MW] this CTA's merge messages
+  float *pin = reinterpret_cast<float *>(smem + lay.pin);     // [NC senders][MW] messages for this CTA's columns
   float *olin = reinterpret_cast<float *>(smem + lay.olin);
   float *logit = reinterpret_cast<float *>(smem + lay.logit);
   int *sidx = reinterpret_cast<int *>(smem + lay.sidx);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
 
   // barrier init touches shared memory only: before the wait on the previous kernel
+  uint64_t *mbx = &bars[kStages];          // candidate messages of the other CTAs (top-M exchange)
+  uint64_t *mbm = &bars[kStages + 1];      // merge messages of the other CTAs
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
+    mbar_init(mbx, 1);
+    mbar_init(mbm, 1);
     fence_mbar_init();
+    // armed once: each completes when the other NC - 1 CTAs' messages are in
+    mbar_arrive_expect_tx(mbx, (uint32_t)((NC - 1) * dec_msg_words(NC) * 4));
+    mbar_arrive_expect_tx(mbm, (uint32_t)((NC - 1) * dec_merge_words(G, D, NC) * 4));
     if constexpr (WIDE) misc[60] = 0u;   // "this cluster holds the last arrival" (wide form)
   }
   if (p.independent) {
@@ -316,13 +332,18 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     if (rank == 0 && tid == 0) set_err(p.err_word, LISA_DEVERR_POS);
     return;
   }
+  // Other CTAs write into this CTA's shared memory only after the matching
+  // wait (after the key stream): by then every CTA has initialised and armed
+  // its mbarriers.
+  cluster_arrive_relaxed();
   const int n = t + 1;
   const int kpc = (((n + NSL - 1) / NSL) + 31) & ~31;
   // this CTA's key slice (the wide form's last cluster later takes wider ranges)
   int k0 = min(n, slice * kpc);
   int k1 = min(n, k0 + kpc);
   int cnt = k1 - k0;
-  const int nsub = window ? 0 : (cnt + SUB - 1) / SUB;
+  // no key stream when every position is selected (n <= M): nothing is scored
+  const int nsub = (window || n <= M) ? 0 : (cnt + SUB - 1) / SUB;
 
   // ---------------------------------------------------------------- TMA ring
   // the indexer keys are read once per step: first out of L2
@@ -603,7 +624,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     if (tid == 0 && i + NS < nsub) issue(i + NS);
   }
   // the new token's score, from the argument row (its cache row may be stale)
-  if (!window && t >= k0 && t < k1 && warp == 0) {
+  if (!window && n > M && t >= k0 && t < k1 && warp == 0) {
     const float *wsm = qis + kMaxR * DI;
     float score = 0.f;
     for (int r = 0; r < R; ++r) {
@@ -618,6 +639,7 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   __syncthreads();
 
   // ---------------------------------------------------------------- top-M
+  cluster_wait();                        // every CTA of the cluster runs and has armed its mbarriers
   // Wide form: every CTA of (b, g) arrives once, after publishing its slice in
   // the workspace.  The CTA that arrives last returns the counter to zero and
   // flags every CTA of its cluster; that cluster alone goes on (with every
@@ -651,131 +673,99 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       for (int j = tid; j < M; j += kDecThreads) sel[j] = n <= M ? (j < n ? j : -1) : t - M + 1 + j;
     }
   } else if (n > M) {
-    constexpr int SEG = kCandCap / NC;                  // candidate slots of each rank in CTA 0
-    uint32_t *fh = hist + 1024;                         // CTA 0: 1024-bin histogram of candidate keys
-    uint32_t *segp = tot + 64;                          // CTA 0: exclusive prefix of the segment sizes
-    // (a) theta: every thread keeps the 4 largest of its keys; the lower edge
-    //     of the 1024-bin range-histogram bin that holds the kl-th largest of
-    //     those values has at least kl of this CTA's keys at or above it.
-    //     Also the largest key, for the range of the exact select.
-    const int ns = (n + kpc - 1) / kpc;                 // slices that hold keys (the others are empty)
-    const int kl = (M + ns - 1) / ns;
-    uint32_t theta_r = 0xFFFFFFFFu;                     // this CTA's bound (every thread holds it)
-    int covered = 0;
-    for (int r = 0; r < NSL; ++r) {
-      const int cr = min(n, (r + 1) * kpc) - min(n, r * kpc);
-      if (cr >= kl) covered += kl;
-    }
-    {
-      uint32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
-      int kt = 0;
-      for (int j = tid; j < cnt; j += kDecThreads) {
-        const uint32_t u = keys[j];
-        ++kt;
-        if (kt > 4 && u <= t3) continue;
-        t3 = u;
-        if (t3 > t2) { const uint32_t x = t2; t2 = t3; t3 = x; }
-        if (t2 > t1) { const uint32_t x = t1; t1 = t2; t2 = x; }
-        if (t1 > t0) { const uint32_t x = t0; t0 = t1; t1 = x; }
-      }
-      kt = min(kt, 4);
-      // smallest and largest of the kept values (0xFFFFFFFF / 0 where a thread kept none)
-      uint32_t vmin = kt == 0 ? 0xFFFFFFFFu : kt == 1 ? t0 : kt == 2 ? t1 : kt == 3 ? t2 : t3;
-      uint32_t vmax = t0;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
-        vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-      }
-      if (lane == 0) {
-        tot[warp] = vmin;
-        tot[8 + warp] = vmax;
-      }
-      for (int i = tid; i < 1024; i += kDecThreads) fh[i] = 0;
-      __syncthreads();
-#pragma unroll
-      for (int w8 = 0; w8 < kDecThreads / 32; ++w8) {
-        vmin = min(vmin, tot[w8]);
-        vmax = max(vmax, tot[8 + w8]);
-      }
-      uint32_t theta = 0xFFFFFFFFu;                     // neutral for the minimum
-      if (cnt >= kl) {                                  // uniform in the CTA
-        const uint32_t sh = (vmax - vmin) < 1024u ? 0u : (uint32_t)(32 - __clz(vmax - vmin)) - 10u;
-        if (kt > 0) atomicAdd(&fh[(t0 - vmin) >> sh], 1u);
-        if (kt > 1) atomicAdd(&fh[(t1 - vmin) >> sh], 1u);
-        if (kt > 2) atomicAdd(&fh[(t2 - vmin) >> sh], 1u);
-        if (kt > 3) atomicAdd(&fh[(t3 - vmin) >> sh], 1u);
-        __syncthreads();
-        find_bin1024<kDecThreads>(fh, (uint32_t)kl, misc);
-        if (misc[0] <= 1023u) theta = vmin + (misc[0] << sh);
-        else theta = 0;                                 // counts inconsistent: no bound from this CTA
-      }
-      if (tid == 0) {
-        misc[4] = theta;
-        misc[6] = vmax;
-      }
-      theta_r = theta;
-    }
-    uint32_t lb = 0, hi = 0;
     if constexpr (WIDE) {
-      // publish this slice (order keys, bound, largest key) and arrive
+      // publish this slice's order keys and arrive; the last cluster's rank r
+      // then takes the contiguous positions of NSL / NC slices
       {
         uint32_t *wk = p.wkeys + (size_t)bg * p.wkeys_stride + k0;
         for (int j = tid; j < cnt; j += kDecThreads) wk[j] = keys[j];
-        if (tid == 0) {
-          p.wtheta[((size_t)bg * NSL + slice) * 2] = misc[4];
-          p.wtheta[((size_t)bg * NSL + slice) * 2 + 1] = misc[6];
-        }
       }
       if (!wide_arrive()) return;
-      // the last cluster: rank r takes the contiguous positions of NSL / NC
-      // slices, and the bound is the smallest over every slice
       const int spr = (NSL / NC) * kpc;
       k0 = min(n, rank * spr);
       k1 = min(n, k0 + spr);
       cnt = k1 - k0;
       const uint32_t *wk = p.wkeys + (size_t)bg * p.wkeys_stride + k0;
       for (int j = tid; j < cnt; j += kDecThreads) keys[j] = __ldcg(wk + j);
-      if (warp == 0) {
-        uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-        for (int w = lane; w < NSL; w += 32) {
-          mn = min(mn, __ldcg(p.wtheta + ((size_t)bg * NSL + w) * 2));
-          mx = max(mx, __ldcg(p.wtheta + ((size_t)bg * NSL + w) * 2 + 1));
-        }
+      __syncthreads();
+    }
+    constexpr int SEG = dec_seg(NC);                    // candidate slots each CTA sends
+    constexpr int XW = dec_msg_words(NC);
+    constexpr int SLOTS = NC * SEG / kDecThreads;       // candidate slots per thread
+    static_assert(SLOTS * kDecThreads == NC * SEG && SLOTS <= 4, "slots");
+    uint32_t *xin = reinterpret_cast<uint32_t *>(smem + lay.xin);   // [NC][XW]
+    uint32_t *xo = xin + rank * XW;                     // this CTA's message, built in its own slot
+    uint32_t *fh = hist + 1024;                         // bins of this CTA's keys
+    uint32_t *sbin = hist;                              // bins of the exact select
+    // kl: keys each CTA vouches for; covered: keys vouched for in all (at least
+    // M when every CTA that holds keys holds kl of them)
+    const int kw = WIDE ? (NSL / NC) * kpc : kpc;       // keys per CTA of the selecting cluster
+    const int ns = (n + kw - 1) / kw;                   // CTAs that hold keys
+    const int kl = (M + ns - 1) / ns;
+    int covered = 0;
+    for (int r = 0; r < NC; ++r) {
+      const int cr = min(n, (r + 1) * kw) - min(n, r * kw);
+      if (cr >= kl) covered += kl;
+    }
+    // (a) this CTA's keys into a 1024-bin range histogram over the 8 octaves
+    //     below its largest key (order keys within 8 << 23 of it).  Its bound
+    //     theta_r is the lower edge of the bin of its kl-th largest key (at
+    //     least kl keys are >= theta_r); its send threshold is the lower edge
+    //     of the bin above the one holding its SEG-th largest key (fewer than
+    //     SEG keys are >= it), or 0 (every key) when it holds at most SEG.
+    uint32_t vmin = 0xFFFFFFFFu, vmax = 0u;
+    for (int j = tid; j < cnt; j += kDecThreads) {
+      const uint32_t u = keys[j];
+      vmin = min(vmin, u);
+      vmax = max(vmax, u);
+    }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        if (lane == 0) {
-          misc[61] = mn;
-          misc[62] = mx;
-        }
+    for (int o = 16; o > 0; o >>= 1) {
+      vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+      vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    if (lane == 0) {
+      tot[warp] = vmin;
+      tot[8 + warp] = vmax;
+    }
+    for (int i = tid; i < 2048; i += kDecThreads) hist[i] = 0;   // fh and sbin
+    __syncthreads();
+#pragma unroll
+    for (int w8 = 0; w8 < kDecThreads / 32; ++w8) {
+      vmin = min(vmin, tot[w8]);
+      vmax = max(vmax, tot[8 + w8]);
+    }
+    uint32_t theta = 0xFFFFFFFFu, tsend = 0u;          // theta: neutral for the minimum
+    if (cnt > 0) {                                      // uniform in the CTA
+      const uint32_t lo = (vmax - vmin) > (8u << 23) ? vmax - (8u << 23) : vmin;
+      const uint32_t sh = (vmax - lo) < 1024u ? 0u : (uint32_t)(32 - __clz(vmax - lo)) - 10u;
+      for (int j = tid; j < cnt; j += kDecThreads) {
+        const uint32_t u = keys[j];
+        if (u >= lo) atomicAdd(&fh[(u - lo) >> sh], 1u);
       }
       __syncthreads();
-      hi = misc[62];
-      if (covered >= M) lb = misc[61];
+      find_bin1024_two<kDecThreads>(fh, (uint32_t)kl, (uint32_t)SEG, misc);
+      if (cnt >= kl) theta = misc[0] <= 1023u ? lo + (misc[0] << sh) : vmin;   // fewer than kl keys >= lo: all
+      if (cnt > SEG) {
+        if (misc[4] <= 1023u) {
+          const uint64_t e = (uint64_t)lo + ((uint64_t)(misc[4] + 1u) << sh);
+          tsend = e > 0xFFFFFFFFull ? 0xFFFFFFFFu : (uint32_t)e;
+        } else {
+          tsend = lo;                                   // fewer than SEG keys >= lo
+        }
+      }
     } else {
-      // every rank's bound into every CTA (misc[32 + rank]), then one barrier
-      if (tid < NC) cluster.map_shared_rank(misc, tid)[32 + rank] = theta_r;
-      cluster.sync();                                   // bounds published, every ring is free
-      uint32_t mn = 0xFFFFFFFFu;
-#pragma unroll
-      for (int r = 0; r < NC; ++r) mn = min(mn, misc[32 + r]);
-      if (covered >= M) lb = mn;
+      vmax = 0u;
     }
-    (void)hi;
-    // (b) keys >= lb go, in position order, to this rank's segment of EVERY
-    //     CTA's candidate list; segment sizes to misc[48 + rank] of every CTA
-    uint32_t *ckl = reinterpret_cast<uint32_t *>(smem + lay.cand_key);
-    int *cpl = reinterpret_cast<int *>(smem + lay.cand_pos);
+    // (b) keys >= tsend, in position order, into this CTA's message; warp w
+    //     owns a contiguous run of keys
     {
-      const int cw = (((cnt + 7) / 8) + 31) & ~31;      // contiguous keys per warp
+      const int cw = (((cnt + 7) / 8) + 31) & ~31;
       const int j0 = min(cnt, warp * cw), j1 = min(cnt, j0 + cw);
       uint32_t wc = 0;
       for (int base = j0; base < j1; base += 32) {
         const int j = base + lane;
-        wc += __popc(__ballot_sync(0xffffffffu, j < j1 && keys[j] >= lb));
+        wc += __popc(__ballot_sync(0xffffffffu, j < j1 && keys[j] >= tsend));
       }
       if (lane == 0) misc[24 + warp] = wc;
       __syncthreads();
@@ -786,180 +776,209 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         off += w8 < warp ? c : 0u;
         total += c;
       }
-      if (tid < NC) cluster.map_shared_rank(misc, tid)[48 + rank] = total;
       if (total <= (uint32_t)SEG) {
         const unsigned lt = (1u << lane) - 1u;
         for (int base = j0; base < j1; base += 32) {
           const int j = base + lane;
-          const bool act = j < j1 && keys[j] >= lb;
+          const bool act = j < j1 && keys[j] >= tsend;
           const unsigned am = __ballot_sync(0xffffffffu, act);
           if (act) {
-            const uint32_t o = rank * SEG + off + __popc(am & lt);
-            const uint32_t kv = keys[j];
-            const int pv = k0 + j;
-#pragma unroll 4
-            for (int d = 0; d < NC; ++d) {
-              cluster.map_shared_rank(ckl, d)[o] = kv;
-              cluster.map_shared_rank(cpl, d)[o] = pv;
-            }
+            const uint32_t o = off + __popc(am & lt);
+            xo[4 + o] = keys[j];
+            xo[4 + SEG + o] = (uint32_t)(k0 + j);
           }
           off += __popc(am);
         }
       }
-    }
-    cluster.sync();                                     // candidates complete
-    // this CTA's candidates are likely selected: their K and V rows into L2
-    // while the list is built (after the barrier, which need not wait for them)
-    for (int j = tid; j < cnt; j += kDecThreads) {
-      if (keys[j] >= lb && k0 + j != t) {
-        const size_t row = ((size_t)bg * p.L_max + k0 + j) * D;
-        const char *kr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.k_cache) + row);
-        const char *vr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.v_cache) + row);
-#pragma unroll
-        for (int c = 0; c < ROWB; c += 128) {
-          prefetch_l2(kr + c);
-          prefetch_l2(vr + c);
-        }
-      }
-    }
-    // the same answer in every CTA: lane r of every warp checks rank r's
-    // segment; the local select holds at most kSelIt candidates per thread
-    uint32_t cnt_l = lane < NC ? misc[48 + lane] : 0u;
-    const bool seg_ok = __all_sync(0xffffffffu, cnt_l <= (uint32_t)SEG);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt_l += __shfl_xor_sync(0xffffffffu, cnt_l, o);
-    constexpr int kSelIt = 4;
-    const bool fits = seg_ok && cnt_l <= (uint32_t)(kSelIt * kDecThreads);
-    local_list = fits;
-    if (fits) {
-      // (c) every CTA, from its own copy of the candidates (the segments
-      //     concatenated in rank order are in position order): the exact M-th
-      //     key K* by an MSB-first radix select over 8-bit digits, then the
-      //     ascending index list by an ordered emission.  Each thread maps its
-      //     candidates c = tid + it * kDecThreads once and keeps them in
-      //     registers; the radix histograms alternate between two buffers.
       if (tid == 0) {
-        uint32_t a = 0;
-        for (int r = 0; r < NC; ++r) {
-          segp[r] = a;
-          a += misc[48 + r];
-        }
-        segp[NC] = a;
+        xo[0] = theta;
+        xo[1] = vmax;
+        xo[2] = tsend;
+        xo[3] = total <= (uint32_t)SEG ? total : 0x80000000u;   // the top bit: too many to send
       }
-      uint32_t *h2 = hist;                              // [2][256]
-      h2[tid] = 0;                                      // 256 threads: the first pass's bins
-      __syncthreads();
-      const int nct = (int)segp[NC];
-      uint32_t cku[kSelIt];
-      int cpp[kSelIt];
+    }
+    __syncthreads();                                    // the message is complete
+    // (c) the message to every other CTA of the cluster (its slot `rank`,
+    //     counted on its candidate mbarrier), then this CTA's likely selected
+    //     K and V rows into L2 while the others' messages arrive
+    {
+      constexpr int CH = XW / 4;                        // 16-byte chunks
+      const uint32_t src = smem_u32(xo), xbar = smem_u32(mbx);
+      for (int i = tid; i < (NC - 1) * CH; i += kDecThreads) {
+        const int dd = i / CH, q = i % CH;
+        const uint32_t d = (uint32_t)(dd < rank ? dd : dd + 1);
+        st_async_v4(mapa_u32(src + 16u * q, d), *reinterpret_cast<const uint4 *>(xo + 4 * q), mapa_u32(xbar, d));
+      }
+    }
+    auto prefetch_kv = [&](int pos) {
+      const size_t row = ((size_t)bg * p.L_max + pos) * D;
+      const char *kr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.k_cache) + row);
+      const char *vr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.v_cache) + row);
 #pragma unroll
-      for (int it = 0; it < kSelIt; ++it) {
-        const int c = tid + it * kDecThreads;
-        cku[it] = 0u;
-        cpp[it] = -1;
-        if (c < nct) {
-          int lo = 0, hi = NC;                          // the segment holding c: segp[lo] <= c < segp[lo + 1]
-          while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if ((int)segp[mid] <= c) lo = mid; else hi = mid;
-          }
-          const int sl = lo * SEG + (c - (int)segp[lo]);
-          cku[it] = ckl[sl];
-          cpp[it] = cpl[sl];
-        }
+      for (int c = 0; c < ROWB; c += 128) {
+        prefetch_l2(kr + c);
+        prefetch_l2(vr + c);
       }
-      uint32_t prefix = 0, pmask = 0, rem = (uint32_t)M;
-      bool rok = nct >= M;
+    };
+    for (int j = tid; j < cnt; j += kDecThreads)
+      if (keys[j] >= theta && k0 + j != t) prefetch_kv(k0 + j);
+    if (!mbar_wait_cluster_bounded(mbx, 0u)) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+    // (d) the bound lb = min_r theta_r (when the CTAs vouch for M keys
+    //     together; else 0) and the largest key, from the headers.  The
+    //     messages hold every key >= lb iff no CTA overflowed and every send
+    //     threshold is <= lb; the same answer in every thread of every CTA.
+    uint32_t th_r = 0xFFFFFFFFu, mx_r = 0u, ts_r = 0u, ct_r = 0u;
+    if (lane < NC) {
+      const uint4 h = *reinterpret_cast<const uint4 *>(xin + lane * XW);
+      th_r = h.x;
+      mx_r = h.y;
+      ts_r = h.z;
+      ct_r = h.w;
+    }
+    uint32_t lbv = th_r, hiv = mx_r;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lbv = min(lbv, __shfl_xor_sync(0xffffffffu, lbv, o));
+      hiv = max(hiv, __shfl_xor_sync(0xffffffffu, hiv, o));
+    }
+    const uint32_t lb = covered >= M ? lbv : 0u;
+    const bool exch_ok = __all_sync(0xffffffffu, (ct_r & 0x80000000u) == 0u && ts_r <= lb);
+    local_list = exch_ok;
+    if (exch_ok) {
+      // the rest of this CTA's candidates (lb <= key < theta) into L2 as well
+      for (int j = tid; j < cnt; j += kDecThreads)
+        if (keys[j] >= lb && keys[j] < theta && k0 + j != t) prefetch_kv(k0 + j);
+      // (e) the candidates, in position order: slot s = (warp * SLOTS + i) *
+      //     32 + lane is entry s % SEG of message s / SEG; valid when that
+      //     entry was sent and its key is >= lb
+      uint32_t cku[SLOTS];
+      int cpp[SLOTS];
+      bool cv[SLOTS];
+#pragma unroll
+      for (int i = 0; i < SLOTS; ++i) {
+        const int s = (warp * SLOTS + i) * 32 + lane;
+        const uint32_t *m = xin + (s / SEG) * XW;
+        const int j = s % SEG;
+        cv[i] = j < (int)m[3];
+        cku[i] = cv[i] ? m[4 + j] : 0u;
+        cpp[i] = cv[i] ? (int)m[4 + SEG + j] : -1;
+        cv[i] = cv[i] && cku[i] >= lb;
+      }
+      // (f) the exact M-th key K*: 1024-bin range histograms over [lb, largest],
+      //     narrowed until the bin holding it is one value or holds at most 32
+      //     keys (ranked in warp 0); need_eq = keys equal to K* the top M takes
+      uint32_t kstar = 0u, need_eq = 0u;
+      bool rok = false;
+      {
+        uint32_t lbx = lb, ubx = hiv, rem = (uint32_t)M;
+        uint32_t shx = (ubx - lbx) < 1024u ? 0u : (uint32_t)(32 - __clz(ubx - lbx)) - 10u;
+        uint32_t *mem = tot + 128;                      // the keys of one bin, at most 32
 #pragma unroll 1
-      for (int pass = 0; pass < 4 && rok; ++pass) {
-        const int shift = 24 - 8 * pass;
-        uint32_t *hc = h2 + (pass & 1) * 256, *hn = h2 + ((pass + 1) & 1) * 256;
-#pragma unroll
-        for (int it = 0; it < kSelIt; ++it)
-          if (tid + it * kDecThreads < nct && (cku[it] & pmask) == prefix)
-            atomicAdd(&hc[(cku[it] >> shift) & 255u], 1u);
-        __syncthreads();
-        uint32_t *res = misc + 56 + 2 * (pass & 1);    // this pass's bucket and count above it
-        if (warp == 0) {
-          uint32_t cb[8], sum = 0;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            cb[j] = hc[255 - (8 * lane + j)];
-            sum += cb[j];
+        for (int iter = 0; iter < 4; ++iter) {
+          if (iter > 0) {
+            for (int i = tid; i < 1024; i += kDecThreads) sbin[i] = 0;
+            __syncthreads();
           }
-          uint32_t inc = sum;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
+          for (int i = 0; i < SLOTS; ++i)
+            if (cv[i] && cku[i] >= lbx && cku[i] <= ubx) atomicAdd(&sbin[(cku[i] - lbx) >> shx], 1u);
+          __syncthreads();
+          find_bin1024<kDecThreads>(sbin, rem, misc);
+          const uint32_t bin = misc[0];
+          if (bin > 1023u) break;                       // inconsistent counts (uniform)
+          rem -= misc[1];
+          const uint32_t cb = misc[2];
+          const uint32_t blo = lbx + (bin << shx);
+          if (shx == 0u) {
+            kstar = blo;
+            need_eq = rem;
+            rok = true;
+            break;
           }
-          const uint32_t exc = inc - sum;
-          const bool here = exc < rem && rem <= inc;
-          if (__ballot_sync(0xffffffffu, here) == 0u) {
-            if (lane == 0) res[0] = 0xFFFFFFFFu;
-          } else if (here) {
-            uint32_t cum = exc;
+          if (cb <= 32u) {
+            if (tid == 0) misc[7] = 0xFFFFFFFFu;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (cum + cb[j] >= rem) {
-                res[0] = 255u - (uint32_t)(8 * lane + j);
-                res[1] = cum;
-                break;
+            for (int i = 0; i < SLOTS; ++i) {
+              if (cv[i] && cku[i] >= lbx && cku[i] <= ubx && ((cku[i] - lbx) >> shx) == bin) {
+                const uint32_t s = atomicAdd(&misc[3], 1u);
+                if (s < 32u) mem[s] = cku[i];
               }
-              cum += cb[j];
             }
+            __syncthreads();
+            if (warp == 0) {
+              const uint32_t x = lane < (int)cb ? mem[lane] : 0u;
+              uint32_t gt = 0, ge = 0;
+              for (int j = 0; j < (int)cb; ++j) {
+                const uint32_t y = __shfl_sync(0xffffffffu, x, j);
+                gt += y > x ? 1u : 0u;
+                ge += y >= x ? 1u : 0u;
+              }
+              if (lane < (int)cb && gt < rem && rem <= ge) {
+                misc[5] = x;
+                misc[7] = rem - gt;
+              }
+            }
+            __syncthreads();
+            kstar = misc[5];
+            need_eq = misc[7];
+            rok = need_eq != 0xFFFFFFFFu;
+            break;
           }
-        } else {
-          hn[tid - 32] = 0;                             // the next pass's bins (warps 1..7, 224 threads)
-          if (tid < 64) hn[224 + tid - 32] = 0;
+          const uint64_t top = (uint64_t)blo + ((1ull << shx) - 1ull);
+          lbx = blo;
+          ubx = top > (uint64_t)ubx ? ubx : (uint32_t)top;
+          shx = shx > 10u ? shx - 10u : 0u;
         }
-        __syncthreads();
-        const uint32_t dg = res[0], above = res[1];
-        if (dg > 255u) {
-          rok = false;                                  // inconsistent counts: cannot happen (uniform)
-          break;
-        }
-        rem -= above;
-        prefix |= dg << shift;
-        pmask |= 255u << shift;
       }
       if (!rok) {
         if (tid == 0) set_err(p.err_word, LISA_DEVERR_CHECK);
         for (int j = tid; j < M; j += kDecThreads) sel[j] = -1;
       } else {
-        const uint32_t kstar = prefix, need_eq = rem;
-        uint32_t base_g = 0, base_e = 0;
-        bool bad = false;
-        const int iters = (nct + kDecThreads - 1) / kDecThreads;
+        // (g) the ascending index list: every key > K*, and the first need_eq
+        //     keys equal to K* in position order; each warp's slots by
+        //     ballots, the warps' offsets from their totals
+        unsigned bgt[SLOTS], beq[SLOTS];
+        uint32_t ngt = 0, neq = 0;
 #pragma unroll
-        for (int it = 0; it < kSelIt; ++it) {
-          if (it >= iters) break;                       // uniform
-          const int c = tid + it * kDecThreads;         // chunk `it` in position order
-          const uint32_t u = cku[it];
-          const int pos = cpp[it];
-          const uint32_t gt = (c < nct && u > kstar) ? 1u : 0u, eq = (c < nct && u == kstar) ? 1u : 0u;
-          uint32_t eg, ee, tg, te;
-          cta_scan2<kDecThreads>(gt, eq, eg, ee, tg, te, misc);
-          const uint32_t pe = base_e + ee;
-          if ((gt || eq) && (pos < 0 || pos >= n)) {
-            bad = true;
-          } else if (gt) {
-            const uint32_t o = base_g + eg + min(pe, need_eq);
-            if (o < (uint32_t)M) sel[o] = pos;
-            else bad = true;
-          } else if (eq && pe < need_eq) {
-            const uint32_t o = base_g + eg + pe;
-            if (o < (uint32_t)M) sel[o] = pos;
+        for (int i = 0; i < SLOTS; ++i) {
+          bgt[i] = __ballot_sync(0xffffffffu, cv[i] && cku[i] > kstar);
+          beq[i] = __ballot_sync(0xffffffffu, cv[i] && cku[i] == kstar);
+          ngt += __popc(bgt[i]);
+          neq += __popc(beq[i]);
+        }
+        if (lane == 0) {
+          misc[16 + warp] = ngt;
+          misc[24 + warp] = neq;
+        }
+        __syncthreads();
+        uint32_t gb = 0, eb = 0, gtot = 0, etot = 0;
+#pragma unroll
+        for (int w8 = 0; w8 < kDecThreads / 32; ++w8) {
+          const uint32_t a = misc[16 + w8], c = misc[24 + w8];
+          gb += w8 < warp ? a : 0u;
+          eb += w8 < warp ? c : 0u;
+          gtot += a;
+          etot += c;
+        }
+        bool bad = gtot + need_eq != (uint32_t)M || etot < need_eq;
+        const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+        for (int i = 0; i < SLOTS; ++i) {
+          const bool gt = (bgt[i] >> lane) & 1u, eq = (beq[i] >> lane) & 1u;
+          const uint32_t pe = eb + __popc(beq[i] & lt);
+          if (gt || (eq && pe < need_eq)) {
+            const uint32_t o = gb + __popc(bgt[i] & lt) + min(pe, need_eq);
+            if (o < (uint32_t)M && cpp[i] >= 0 && cpp[i] < n) sel[o] = cpp[i];
             else bad = true;
           }
-          base_g += tg;
-          base_e += te;
+          gb += __popc(bgt[i]);
+          eb += __popc(beq[i]);
         }
-        if (base_g + need_eq != (uint32_t)M || base_e < need_eq) bad = true;
         if (bad) set_err(p.err_word, LISA_DEVERR_CHECK);
       }
     } else {
-      // (d) too many keys passed the bound: cluster-wide radix select over all keys
+      // (h) the messages miss keys >= lb (a CTA had too many to send, or
+      //     sent too few): cluster-wide radix select over all keys
       uint32_t prefix = 0, pmask = 0, rem = (uint32_t)M;
       bool ok = true;
       const int iters = (cnt + kDecThreads - 1) / kDecThreads;
@@ -1117,10 +1136,6 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     sidx[r] = s;
   }
   __syncthreads();
-  // This CTA no longer reads its candidate lists (nor CTA 0's list): the
-  // other CTAs may write their partials into its shared memory once every
-  // CTA has arrived here (they wait just before those stores).
-  cluster_arrive_release();
   {
     // every 16-byte piece in flight at once (asynchronous copies; rows of
     // unselected slots are zero-filled)
@@ -1194,6 +1209,9 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     }
   }
   __syncthreads();
+  // this CTA's partial output of head hh, column d: into the merge message
+  // for the CTA that owns column d
+  auto put_part = [&](int hh, int d, float v) { pout[(d / COLS) * MW + hh * COLS + d % COLS] = v; };
   // per head: local max and sum of exponentials over this CTA's rows
   for (int hh = warp; hh < G; hh += 8) {
     float m = -INFINITY;
@@ -1207,14 +1225,15 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       l += e;
     }
     l = warp_sum(l);
-    if (lane == 0) {
-      pml[2 * hh] = m;
-      pml[2 * hh + 1] = l;
+    // (max, sum) of this head go to every owner's merge message
+    for (int o = lane; o < NC; o += 32) {
+      pout[o * MW + G * COLS + 2 * hh] = m;
+      pout[o * MW + G * COLS + 2 * hh + 1] = l;
     }
   }
   __syncthreads();
   if (mma_attn) {
-    // part[hh][d] = sum_r e[hh][r] v_r[d]: A = e (heads x rows) as bf16 hi + lo
+    // o_part[hh][d] = sum_r e[hh][r] v_r[d]: A = e (heads x rows) as bf16 hi + lo
     // pairs, B = V rows (rows x d) through transposing matrix loads
     const int g4 = lane >> 2, t2 = (lane & 3) * 2;
     const uint32_t v_u32 = smem_u32(kvs + rpc * RS);
@@ -1252,65 +1271,65 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       for (int j = 0; j < 4; ++j) {
         const int hh = g4 + (j >> 1) * 8, d = np * 16 + t2 + (j & 1);
         if (hh < G) {
-          part[hh * D + d] = c0[j];
-          part[hh * D + d + 8] = c1[j];
+          put_part(hh, d, c0[j]);
+          put_part(hh, d + 8, c1[j]);
         }
       }
     }
   } else {
-    // part[hh][d] = sum_r e[hh][r] v_r[d]
+    // o_part[hh][d] = sum_r e[hh][r] v_r[d]
     for (int i = tid; i < G * D; i += kDecThreads) {
       const int hh = i / D, d = i % D;
       const float *e = logit + hh * rpc;
       const T *vcol = reinterpret_cast<const T *>(kvs + rpc * RS) + d;
       float a = 0.f;
       for (int r = 0; r < rpc; ++r) a = fmaf(e[r], Dt<T>::to_f(vcol[(size_t)r * (RS / sizeof(T))]), a);
-      part[i] = a;
+      put_part(hh, d, a);
     }
   }
   // ---------------------------------------------------------------- merge + gate, columns of this CTA
-  // each rank writes its partials of the columns [r*D/NC, (r+1)*D/NC) and its
-  // softmax statistics into CTA r; after one barrier every CTA merges from its
-  // own shared memory and nobody reads another CTA's memory again
+  // Each CTA sends, to every other CTA r, its partial outputs of r's columns
+  // [r*D/NC, (r+1)*D/NC) and its (max, sum) per head (counted on r's merge
+  // mbarrier), then merges the NC partials of its own columns once the others'
+  // have arrived.
+  __syncthreads();                             // the merge messages are complete
   {
-    __syncthreads();                           // part and pml are complete
-    cluster_wait_acquire();                    // every CTA is past its selection
-    for (int i = tid; i < G * D; i += kDecThreads) {
-      const int hh = i / D, d = i % D, owner = d / COLS, c = d % COLS;
-      float *pin_o = cluster.map_shared_rank(reinterpret_cast<float *>(smem + lay.pin), owner);
-      pin_o[(rank * G + hh) * COLS + c] = part[i];
-    }
-    for (int i = tid; i < NC * 2 * G; i += kDecThreads) {
-      const int owner = i / (2 * G), j = i % (2 * G);
-      float *pin_o = cluster.map_shared_rank(reinterpret_cast<float *>(smem + lay.pin), owner);
-      pin_o[NC * G * COLS + rank * 2 * G + j] = pml[j];
+    const int CH = MW / 4;                     // 16-byte chunks per message
+    const uint32_t dst0 = smem_u32(pin + rank * MW), mbar = smem_u32(mbm);
+    for (int i = tid; i < (NC - 1) * CH; i += kDecThreads) {
+      const int dd = i / CH, q = i % CH;
+      const uint32_t d = (uint32_t)(dd < rank ? dd : dd + 1);
+      st_async_v4(mapa_u32(dst0 + 16u * q, d), *reinterpret_cast<const uint4 *>(pout + d * MW + 4 * q),
+                  mapa_u32(mbar, d));
     }
   }
-  cluster.sync();                            // every partial of this CTA's columns has arrived
-  {
-    const float *pin = reinterpret_cast<const float *>(smem + lay.pin);
-    const float *pml_all = pin + NC * G * COLS;                 // [NC][2G]
-    for (int i = tid; i < G * COLS; i += kDecThreads) {
-      const int hh = i / COLS, c = i % COLS, d = c0s + c;
-      float mx = -INFINITY;
+  // The matching wait ends the kernel: no CTA leaves while another may still
+  // be sending to it.
+  cluster_arrive_relaxed();
+  if (!mbar_wait_cluster_bounded(mbm, 0u)) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
+  for (int i = tid; i < G * COLS; i += kDecThreads) {
+    const int hh = i / COLS, c = i % COLS, d = c0s + c;
+    auto msg = [&](int r) -> const float * { return r == rank ? pout + rank * MW : pin + r * MW; };
+    float mx = -INFINITY;
 #pragma unroll
-      for (int r = 0; r < NC; ++r) mx = fmaxf(mx, pml_all[r * 2 * G + 2 * hh]);
-      float num = 0.f, den = 0.f;
+    for (int r = 0; r < NC; ++r) mx = fmaxf(mx, msg(r)[G * COLS + 2 * hh]);
+    float num = 0.f, den = 0.f;
 #pragma unroll
-      for (int r = 0; r < NC; ++r) {
-        const float mr = pml_all[r * 2 * G + 2 * hh];
-        if (mr == -INFINITY) continue;
-        const float f = expf(mr - mx);
-        num = fmaf(f, pin[(r * G + hh) * COLS + c], num);
-        den = fmaf(f, pml_all[r * 2 * G + 2 * hh + 1], den);
-      }
-      const int h = g * G + hh;
-      const float o_sp = num / den;
-      const float o_lin = olin[hh * COLS + c];
-      const float gam = 1.f / (1.f + expf(-gls[hh]));
-      reinterpret_cast<T *>(p.out)[((size_t)b * p.Hq + h) * D + d] = Dt<T>::from_f(gam * o_sp + (1.f - gam) * o_lin);
+    for (int r = 0; r < NC; ++r) {
+      const float *mr = msg(r);
+      const float m_r = mr[G * COLS + 2 * hh];
+      if (m_r == -INFINITY) continue;
+      const float f = expf(m_r - mx);
+      num = fmaf(f, mr[hh * COLS + c], num);
+      den = fmaf(f, mr[G * COLS + 2 * hh + 1], den);
     }
+    const int h = g * G + hh;
+    const float o_sp = num / den;
+    const float o_lin = olin[hh * COLS + c];
+    const float gam = 1.f / (1.f + expf(-gls[hh]));
+    reinterpret_cast<T *>(p.out)[((size_t)b * p.Hq + h) * D + d] = Dt<T>::from_f(gam * o_sp + (1.f - gam) * o_lin);
   }
+  cluster_wait();
 }
 
 // ============================================================ launcher
@@ -1452,14 +1471,12 @@ static cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
 }
 
 // Workspace of the wide form, sized for nw CTAs per (b, g): arrival counters,
-// per-CTA bounds, per-CTA partial readouts and the order keys (each block
-// 256-byte aligned).
+// per-CTA partial readouts and the order keys (each block 256-byte aligned).
 size_t decode_wide_workspace_bytes(int B, int Hkv, int G, int D, int L_max, int nw) {
   (void)G;
   const size_t pairs = (size_t)B * Hkv;
   auto r256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return r256(pairs * 4) + r256(pairs * nw * 2 * 4) + r256(pairs * nw * 2 * D * 4) +
-         r256(pairs * (size_t)((L_max + 3) & ~3) * 4);
+  return r256(pairs * 4) + r256(pairs * nw * 2 * D * 4) + r256(pairs * (size_t)((L_max + 3) & ~3) * 4);
 }
 
 // The library's choice never takes the wide form: measured on a B200 at the

@@ -65,7 +65,6 @@ struct DecodeParams {
   // last of their clusters to finish selects and attends.  Workspace per (b, g):
   int nw;                               // CTAs per (b, g), a multiple of 8, >= G; 0: the cluster form
   uint32_t *wkeys;                      // [B*Hkv][wkeys_stride] order keys of positions 0..t
-  uint32_t *wtheta;                     // [B*Hkv][nw][2] per-CTA bound and largest key
   float *wpart;                         // [B*Hkv][nw][2][d] per-CTA partial o_lin of (up to) two heads
   unsigned *wcount;                     // [B*Hkv] arrival counters (zero between calls)
   int wkeys_stride;

@@ -270,6 +270,57 @@ __device__ void find_bin1024(const uint32_t *fh, uint32_t rem, uint32_t *misc) {
   __syncthreads();
 }
 
+// find_bin1024 for two ranks in one scan: misc[0..2] for rank ra, misc[4..6]
+// for rank rb (bin, keys in higher bins, keys in the bin; bin 0xFFFFFFFF when
+// the counts hold fewer keys than the rank), misc[7] = keys in all bins;
+// misc[3] is zeroed.  Uses misc[8..15].  Ends with a barrier.
+template <int NT>
+__device__ void find_bin1024_two(const uint32_t *fh, uint32_t ra, uint32_t rb, uint32_t *misc) {
+  static_assert(NT * 4 == 1024, "four bins per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b0 = 1023 - 4 * tid;
+  const uint32_t cc[4] = {fh[b0], fh[b0 - 1], fh[b0 - 2], fh[b0 - 3]};
+  const uint32_t c = cc[0] + cc[1] + cc[2] + cc[3];
+  uint32_t inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) misc[8 + warp] = inc;
+  if (tid == 0) {
+    misc[0] = 0xFFFFFFFFu;
+    misc[4] = 0xFFFFFFFFu;
+    misc[3] = 0;
+  }
+  __syncthreads();
+  uint32_t off = 0, all = 0;
+#pragma unroll
+  for (int w8 = 0; w8 < NT / 32; ++w8) {
+    off += w8 < warp ? misc[8 + w8] : 0u;
+    all += misc[8 + w8];
+  }
+  const uint32_t exc = off + inc - c;
+  if (tid == 0) misc[7] = all;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t rem = k == 0 ? ra : rb;
+    if (exc < rem && rem <= exc + c) {
+      uint32_t cum = exc;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (cum < rem && rem <= cum + cc[j]) {
+          misc[4 * k] = (uint32_t)(b0 - j);
+          misc[4 * k + 1] = cum;
+          misc[4 * k + 2] = cc[j];
+        }
+        cum += cc[j];
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // CTA-wide exclusive prefix sums of two counters, plus their totals.  Uses
 // misc[32..47].
 template <int NT>

@@ -93,12 +93,12 @@ def test_decode_rejects_null_and_misaligned_inputs():
 def test_decode_workspace_is_the_wide_forms_and_context_is_bounded():
     """The decode workspace holds the wide form's pieces, each rounded to 256
     bytes and sized for 64 CTAs per (sequence, KV head): arrival counters,
-    per-CTA bound and largest key, per-CTA partial readouts of two heads, and
-    the order keys of every cached position."""
+    per-CTA partial readouts of two heads, and the order keys of every cached
+    position."""
     r256 = lambda x: (x + 255) // 256 * 256
     c = _layer(B=3, L_max=1000)
     pairs, d = 3 * 2, 128
-    want = r256(pairs * 4) + r256(pairs * 64 * 2 * 4) + r256(pairs * 64 * 2 * d * 4) + r256(pairs * 1000 * 4)
+    want = r256(pairs * 4) + r256(pairs * 64 * 2 * d * 4) + r256(pairs * 1000 * 4)
     assert L.lisa_workspace_bytes(c, 1, L.LISA_OP_DECODE) == want
     assert L.lisa_workspace_bytes(_layer(dtype=L.LISA_FP32), 1, L.LISA_OP_DECODE) == 0
     # the wide form asked for explicitly needs bf16 storage and the workspace
