@@ -194,11 +194,17 @@ __global__ void __launch_bounds__(NT) rows_select_kernel(RowsParams p, int tau0,
   int *out = p.idx + (((size_t)b * p.T + tau) * p.Hkv + g) * p.M;
   if (n >= 8 * NT) {
     // long rows (read from global memory / L2, not staged, so that several
-    // rows share an SM): a bound from every thread's 4 largest keys, then an
-    // exact select among the few keys above it
+    // rows share an SM): a bound from a sample and one pass over the keys;
+    // where that bound does not serve, a bound from every thread's 4 largest
+    // keys, then an exact select among the few keys above it
     __shared__ BoundedShared bsm;
-    const int r = block_topm_bounded<NT>(keys, n, p.M, out, bsm, cand, reinterpret_cast<int *>(cand + p.cand_cap),
-                                         p.cand_cap);
+    int r = 0;
+    if (keys == gkeys && n > p.M)
+      r = block_topm_sampled<NT>(keys, n, p.M, out, bsm, cand, reinterpret_cast<int *>(cand + p.cand_cap),
+                                 p.cand_cap);
+    if (r == 0)
+      r = block_topm_bounded<NT>(keys, n, p.M, out, bsm, cand, reinterpret_cast<int *>(cand + p.cand_cap),
+                                 p.cand_cap);
     if (r == 1) return;
     if (r < 0) {
       if (threadIdx.x == 0) set_err(p.err_word, LISA_DEVERR_CHECK);

@@ -4,7 +4,12 @@
 // "top-M"): the first min(M, n) positions in the order (key descending,
 // position ascending), written in ascending position order, padded with -1.
 //
-// Two methods:
+// Three methods:
+//  * block_topm_sampled (long rows in global memory): a bound from a 1/8 (or
+//    sparser) block sample of the keys, then one pass of 16-byte loads that
+//    compacts the keys above it per warp; the exact K* and the ordered
+//    emission work on those per-warp segments.  Falls back to the next
+//    method when fewer than M keys pass the bound or a segment is full.
 //  * block_topm_bounded (long rows): every thread keeps its 4 largest keys;
 //    the bin of the M-th largest of those values gives a bound lb with at
 //    least M keys >= lb; the keys >= lb are compacted in position order; the
@@ -545,6 +550,241 @@ __device__ int block_topm_bounded(const uint32_t *keys, int n, int M, int *out, 
       }
       ++ee;
     }
+  }
+  return __syncthreads_or(bad) ? -1 : 1;
+}
+
+// Top-M of a long row keys[0..n) (global memory, 16-byte aligned and readable
+// up to n rounded up to 4; n >= 8 * NT, n > M) with one pass over the keys:
+//  (1) a bound from a sample: the first 16 keys (one 64-byte block) of every
+//      step-th group of 128, at most 4 blocks per thread, so the sample adds
+//      no DRAM traffic to the pass that follows.  lb = the lower edge of the
+//      1024-bin range bin (over the 8 octaves below the sample's largest
+//      key) that holds the sample's r-th largest key, r chosen so that about
+//      2M keys of the row are expected at or above lb;
+//  (2) one pass of 16-byte loads: warp w compacts the keys >= lb of its
+//      contiguous run, in position order, into its own segment of (ck, cp)
+//      (cap / NW entries each) and tracks their largest key;
+//  (3) fewer than M keys >= lb, or a full segment: returns 0 and the caller's
+//      exact paths run.  Else the exact M-th key K* by range histograms over
+//      the segments, and each warp emits its segment's share of the
+//      ascending index list at offsets from the warps' counts.
+// Returns 1 (done), 0 (bound unusable) or -1 (inconsistent counts).
+template <int NT>
+__device__ __forceinline__ int block_topm_sampled(const uint32_t *keys, int n, int M, int *out, BoundedShared &sm, uint32_t *ck,
+                                  int *cp, int cap) {
+  static_assert(NT == 256, "256 threads");
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int segcap = cap / NW;
+  // (1) the sample: groups g = i * step (i < ng) of 128 keys, keys [128 g, 128 g + 16)
+  const int groups = n / 128;
+  const int step = (groups + 255) / 256;
+  const int ng = groups / step;                       // sampled groups, at most 256: 4 uint4 per thread
+  const int nsv = ng * 4;
+  uint4 sv[4];
+  uint32_t vmin = 0xFFFFFFFFu, vmax = 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int s = tid + k * NT;
+    sv[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (s < nsv) {
+      sv[k] = __ldcg(reinterpret_cast<const uint4 *>(keys + (size_t)(s >> 2) * step * 128 + (s & 3) * 4));
+      vmin = min(vmin, min(min(sv[k].x, sv[k].y), min(sv[k].z, sv[k].w)));
+      vmax = max(vmax, max(max(sv[k].x, sv[k].y), max(sv[k].z, sv[k].w)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+    vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  }
+  if (lane == 0) {
+    sm.misc[48 + warp] = vmin;
+    sm.misc[56 + warp] = vmax;
+  }
+  for (int i = tid; i < 1024; i += NT) sm.fh[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int w8 = 0; w8 < NW; ++w8) {
+    vmin = min(vmin, sm.misc[48 + w8]);
+    vmax = max(vmax, sm.misc[56 + w8]);
+  }
+  const uint32_t lo = (vmax - vmin) > (8u << 23) ? vmax - (8u << 23) : vmin;
+  const uint32_t sh = (vmax - lo) < 1024u ? 0u : (uint32_t)(32 - __clz(vmax - lo)) - 10u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (tid + k * NT < nsv) {
+      const uint32_t w4[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (w4[q] >= lo) atomicAdd(&sm.fh[(w4[q] - lo) >> sh], 1u);
+    }
+  }
+  __syncthreads();
+  // about 2M keys at or above the r-th largest of the nsv * 4 sampled keys
+  const long long r_ll = (2ll * M * nsv * 4 + n - 1) / n;
+  const uint32_t r = (uint32_t)(r_ll < 1 ? 1 : r_ll);
+  find_bin1024<NT>(sm.fh, r, sm.misc);
+  const uint32_t lb = sm.misc[0] <= 1023u ? lo + (sm.misc[0] << sh) : lo;
+  // (2) one pass: warp w's run [j0, j1) of positions, 128 per iteration
+  const int cw = (((n + NW - 1) / NW) + 127) & ~127;
+  const int j0 = min(n, warp * cw), j1 = min(n, j0 + cw);
+  uint32_t *cks = ck + warp * segcap;
+  int *cps = cp + warp * segcap;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t cnt = 0, cmax = 0u;
+  for (int base = j0; base < j1; base += 128) {
+    const int idx = base + 4 * lane;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (idx < j1) v = __ldcg(reinterpret_cast<const uint4 *>(keys + idx));
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    bool f[4];
+    unsigned bl[4];
+    uint32_t before = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      f[q] = idx + q < j1 && w4[q] >= lb;
+      bl[q] = __ballot_sync(0xffffffffu, f[q]);
+      before += __popc(bl[q] & lt);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (f[q]) {
+        const uint32_t o = cnt + before;
+        if (o < (uint32_t)segcap) {
+          cks[o] = w4[q];
+          cps[o] = idx + q;
+        }
+        cmax = max(cmax, w4[q]);
+        ++before;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) cnt += __popc(bl[q]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+  if (lane == 0) {
+    sm.misc[16 + warp] = cnt;
+    sm.misc[24 + warp] = cmax;
+  }
+  __syncthreads();
+  uint32_t total = 0, hi = 0;
+  bool full = false;
+#pragma unroll
+  for (int w8 = 0; w8 < NW; ++w8) {
+    total += sm.misc[16 + w8];
+    hi = max(hi, sm.misc[24 + w8]);
+    full = full || sm.misc[16 + w8] > (uint32_t)segcap;
+  }
+  if (full || total < (uint32_t)M) {                  // the same answer in every thread
+    __syncthreads();                                  // read by all before the caller reuses sm
+    return 0;
+  }
+  cnt = sm.misc[16 + warp];
+  // (3) K*: 1024-bin range histograms over [lb, hi] of the segments, narrowed
+  //     until the bin of the rem-th key is one value or holds <= 32 keys
+  uint32_t kstar = 0, need_eq = 0;
+  {
+    uint32_t lbx = lb, ubx = hi, rem = (uint32_t)M;
+    uint32_t shx = (ubx - lbx) < 1024u ? 0u : (uint32_t)(32 - __clz(ubx - lbx)) - 10u;
+    bool done = false;
+#pragma unroll 1
+    for (int iter = 0; iter < 4 && !done; ++iter) {
+      __syncthreads();                                // every thread is done with the previous bins
+      for (int i = tid; i < 1024; i += NT) sm.fh[i] = 0;
+      __syncthreads();
+      for (int j = lane; j < (int)cnt; j += 32) {
+        const uint32_t u = cks[j];
+        if (u >= lbx && u <= ubx) atomicAdd(&sm.fh[(u - lbx) >> shx], 1u);
+      }
+      __syncthreads();
+      find_bin1024<NT>(sm.fh, rem, sm.misc);
+      const uint32_t bin = sm.misc[0];
+      if (bin > 1023u) return -1;
+      rem -= sm.misc[1];
+      const uint32_t cb = sm.misc[2];
+      const uint32_t blo = lbx + (bin << shx);
+      if (shx == 0u) {
+        kstar = blo;
+        need_eq = rem;
+        done = true;
+      } else if (cb <= 32u) {
+        if (tid == 0) sm.misc[7] = 0xFFFFFFFFu;
+        for (int j = lane; j < (int)cnt; j += 32) {
+          const uint32_t u = cks[j];
+          if (u >= lbx && u <= ubx && ((u - lbx) >> shx) == bin) {
+            const uint32_t s = atomicAdd(&sm.misc[3], 1u);
+            if (s < 32u) sm.members[s] = u;
+          }
+        }
+        __syncthreads();
+        if (warp == 0) {
+          const uint32_t x = lane < (int)cb ? sm.members[lane] : 0u;
+          uint32_t gt = 0, ge = 0;
+          for (int j = 0; j < (int)cb; ++j) {
+            const uint32_t y = __shfl_sync(0xffffffffu, x, j);
+            gt += y > x ? 1u : 0u;
+            ge += y >= x ? 1u : 0u;
+          }
+          if (lane < (int)cb && gt < rem && rem <= ge) {
+            sm.misc[5] = x;
+            sm.misc[7] = rem - gt;
+          }
+        }
+        __syncthreads();
+        kstar = sm.misc[5];
+        need_eq = sm.misc[7];
+        if (need_eq == 0xFFFFFFFFu) return -1;
+        done = true;
+      } else {
+        const uint64_t top = (uint64_t)blo + ((1ull << shx) - 1ull);
+        lbx = blo;
+        ubx = top > (uint64_t)ubx ? ubx : (uint32_t)top;
+        shx = shx > 10u ? shx - 10u : 0u;
+      }
+    }
+    if (!done) return -1;
+  }
+  // (4) the ascending index list: each warp counts its segment's keys > K*
+  //     and == K*, then emits them at offsets from the earlier warps' counts
+  uint32_t ngt = 0, neq = 0;
+  for (int base = 0; base < (int)cnt; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = j < (int)cnt ? cks[j] : 0u;
+    ngt += __popc(__ballot_sync(0xffffffffu, j < (int)cnt && u > kstar));
+    neq += __popc(__ballot_sync(0xffffffffu, j < (int)cnt && u == kstar));
+  }
+  if (lane == 0) {
+    sm.misc[32 + warp] = ngt;
+    sm.misc[40 + warp] = neq;
+  }
+  __syncthreads();
+  uint32_t gb = 0, eb = 0, gtot = 0, etot = 0;
+#pragma unroll
+  for (int w8 = 0; w8 < NW; ++w8) {
+    const uint32_t a = sm.misc[32 + w8], c = sm.misc[40 + w8];
+    gb += w8 < warp ? a : 0u;
+    eb += w8 < warp ? c : 0u;
+    gtot += a;
+    etot += c;
+  }
+  bool bad = gtot + need_eq != (uint32_t)M || etot < need_eq;
+  for (int base = 0; base < (int)cnt; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = j < (int)cnt ? cks[j] : 0u;
+    const unsigned bgt = __ballot_sync(0xffffffffu, j < (int)cnt && u > kstar);
+    const unsigned beq = __ballot_sync(0xffffffffu, j < (int)cnt && u == kstar);
+    const uint32_t pe = eb + __popc(beq & lt);
+    const bool gt = (bgt >> lane) & 1u, eq = (beq >> lane) & 1u;
+    if (gt || (eq && pe < need_eq)) {
+      const uint32_t o = gb + __popc(bgt & lt) + min(pe, need_eq);
+      if (o < (uint32_t)M) out[o] = cps[j];
+      else bad = true;
+    }
+    gb += __popc(bgt);
+    eb += __popc(beq);
   }
   return __syncthreads_or(bad) ? -1 : 1;
 }
