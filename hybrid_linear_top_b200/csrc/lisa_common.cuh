@@ -306,6 +306,15 @@ __device__ __forceinline__ uint2 ld_nc_v2(const void *p) {
   return r;
 }
 
+// 2^x by PTX ex2.approx (one special-function instruction, about 2 ulp);
+// e^x = 2^(x log2 e), so callers keep logits in log2 units.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

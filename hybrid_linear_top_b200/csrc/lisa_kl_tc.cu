@@ -38,7 +38,6 @@ constexpr int kKlStages = 4;
 constexpr int kKlThreads = 384;    // warps 0-3: TMA, MMA, two idle; warps 4-11: epilogue
 constexpr int kKlEpiThreads = 256;
 constexpr int kKlBufCols = 256;    // per buffer: heads at j * 32, indexer heads at 96 + r * 32
-constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
 constexpr float kLn2 = 0.6931471805599453f;     // ln(2)
 
 template <int DI>
@@ -56,13 +55,8 @@ struct KlTcGeom {
   static __host__ __device__ int smem(int R) { return 1024 + bar_off(R) + 256; }
 };
 
-// 2^x (PTX ex2.approx: one special-function instruction; the epilogue keeps
-// its logits in log2 units so that no multiply precedes it)
-__device__ __forceinline__ float exp2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+// exp2_approx (lisa_common.cuh): the epilogue keeps its logits in log2 units
+// so that no multiply precedes the exponential.
 
 __device__ __forceinline__ float tree_max16(const float *x) {
   float s8[8], s4[4];

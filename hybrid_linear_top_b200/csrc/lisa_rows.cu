@@ -423,6 +423,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
   const int hl = lane >> 2, kq = (lane & 3) * 2;
   const int RW = p.M / kAttnWarps;               // rows of this warp (a multiple of 16)
   const int t_abs = p.pos[b] + tau;
+  const float scale2 = p.scale * kLog2e;         // logits in log2 units: e^x = 2^(x log2 e)
   unsigned char *wbuf = s_att + warp * 4 * TILE; // [stage][K | V]
   const uint32_t wbuf_u32 = smem_u32(wbuf);
   const int *idx = p.idx + (((size_t)b * p.T + tau) * p.sel_heads + (p.sel_heads == 1 ? 0 : g)) * p.M + warp * RW;
@@ -456,7 +457,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
     }
     return s;
   };
-  auto stage_tile = [&](int i, int my_pos) {   // cp.async 16 rows of K and V into stage i & 1
+  // cp.async 16 rows of K and V into stage i & 1; each warp instruction
+  // copies two whole rows (16 lanes x 16 bytes each), so it touches few
+  // cache lines (zero-filled where the slot holds no position)
+  auto stage_tile = [&](int i, int my_pos) {
     const uint32_t kdst = wbuf_u32 + (i & 1) * 2 * TILE, vdst = kdst + TILE;
     constexpr int CH = 2 * D / 16;               // 16-byte chunks per row
 #pragma unroll
@@ -517,10 +521,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
     uint32_t pb[NHT][2];
 #pragma unroll
     for (int nh = 0; nh < NHT; ++nh) {
-      // scale, mask; c0, c1: row hl (heads kq, kq + 1); c2, c3: row hl + 8
+      // scale (in log2 units), mask; c0, c1: row hl (heads kq, kq + 1); c2, c3: row hl + 8
       float x[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) x[j] = (j < 2 ? pr0 : pr1) >= 0 ? sc[nh][j] * p.scale : -INFINITY;
+      for (int j = 0; j < 4; ++j) x[j] = (j < 2 ? pr0 : pr1) >= 0 ? sc[nh][j] * scale2 : -INFINITY;
       // the heads' maxima over the tile's 16 rows (lanes with the same lane % 4)
       float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
@@ -529,22 +533,26 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
       }
       const float mn0 = fmaxf(mh[nh][0], mx0), mn1 = fmaxf(mh[nh][1], mx1);
-      const float f0 = mh[nh][0] == -INFINITY ? 0.f : expf(mh[nh][0] - mn0);
-      const float f1 = mh[nh][1] == -INFINITY ? 0.f : expf(mh[nh][1] - mn1);
+      // the accumulators need rescaling only where a running maximum moved
+      const bool moved = __any_sync(0xffffffffu, mn0 != mh[nh][0] || mn1 != mh[nh][1]);
+      const float f0 = mh[nh][0] == -INFINITY ? 0.f : exp2_approx(mh[nh][0] - mn0);
+      const float f1 = mh[nh][1] == -INFINITY ? 0.f : exp2_approx(mh[nh][1] - mn1);
       mh[nh][0] = mn0;
       mh[nh][1] = mn1;
-      const float e0 = x[0] == -INFINITY ? 0.f : expf(x[0] - mn0);
-      const float e1 = x[1] == -INFINITY ? 0.f : expf(x[1] - mn1);
-      const float e2 = x[2] == -INFINITY ? 0.f : expf(x[2] - mn0);
-      const float e3 = x[3] == -INFINITY ? 0.f : expf(x[3] - mn1);
+      const float e0 = x[0] == -INFINITY ? 0.f : exp2_approx(x[0] - mn0);
+      const float e1 = x[1] == -INFINITY ? 0.f : exp2_approx(x[1] - mn1);
+      const float e2 = x[2] == -INFINITY ? 0.f : exp2_approx(x[2] - mn0);
+      const float e3 = x[3] == -INFINITY ? 0.f : exp2_approx(x[3] - mn1);
       lh[nh][0] = lh[nh][0] * f0 + e0 + e2;
       lh[nh][1] = lh[nh][1] * f1 + e1 + e3;
+      if (moved) {
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        o[nh][mt][0] *= f0;
-        o[nh][mt][1] *= f1;
-        o[nh][mt][2] *= f0;
-        o[nh][mt][3] *= f1;
+        for (int mt = 0; mt < MT; ++mt) {
+          o[nh][mt][0] *= f0;
+          o[nh][mt][1] *= f1;
+          o[nh][mt][2] *= f0;
+          o[nh][mt][3] *= f1;
+        }
       }
       // P^T (k = rows, n = heads) as the B operand: transposes of the two 8x8 blocks
       pb[nh][0] = movmatrix_trans(pack_bf16(e0, e1));
@@ -601,9 +609,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
     float num = 0.f, den = 0.f;
 #pragma unroll
     for (int w = 0; w < kAttnWarps; ++w) {
-      const float mw = s_ml[(w * 16 + hh) * 2];
+      const float mw = s_ml[(w * 16 + hh) * 2];          // log2 units
       if (mw == -INFINITY) continue;
-      const float f = expf(mw - mx);
+      const float f = exp2_approx(mw - mx);
       num = fmaf(f, s_o[(w * 16 + hh) * D + d], num);
       den = fmaf(f, s_ml[(w * 16 + hh) * 2 + 1], den);
     }

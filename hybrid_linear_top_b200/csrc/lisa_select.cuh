@@ -634,10 +634,13 @@ __device__ __forceinline__ int block_topm_sampled(const uint32_t *keys, int n, i
   int *cps = cp + warp * segcap;
   const unsigned lt = (1u << lane) - 1u;
   uint32_t cnt = 0, cmax = 0u;
+  // the next iteration's 16 bytes are requested before this one's are used
+  uint4 vn = make_uint4(0u, 0u, 0u, 0u);
+  if (j0 + 4 * lane < j1) vn = __ldcg(reinterpret_cast<const uint4 *>(keys + j0 + 4 * lane));
   for (int base = j0; base < j1; base += 128) {
     const int idx = base + 4 * lane;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (idx < j1) v = __ldcg(reinterpret_cast<const uint4 *>(keys + idx));
+    const uint4 v = vn;
+    if (idx + 128 < j1) vn = __ldcg(reinterpret_cast<const uint4 *>(keys + idx + 128));
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
     bool f[4];
     unsigned bl[4];
