@@ -37,7 +37,8 @@ size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 int round4(int x) { return (x + 3) & ~3; }
 
 constexpr int kRowsStagedCap = 2048;   // keys of a row staged in shared memory by the row select
-constexpr int kCandCap = 4096;          // threshold-bucket candidates kept in shared memory
+constexpr int kCandCap = 2048;          // threshold-bucket candidates kept in shared memory (a small
+                                        // footprint lets about six select CTAs share an SM)
 constexpr int kRowChunk = 2048;         // query rows scored per pass on the row path
 constexpr int kMaxSmem = 227 * 1024;    // dynamic shared memory a CTA may use on sm_100
 

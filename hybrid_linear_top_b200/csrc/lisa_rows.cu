@@ -600,25 +600,35 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
       s_o[(warp * 16 + h0 + 1) * D + d + 8] = o[nh][mt][3];
     }
   }
-  __syncthreads();
-  for (int i = tid; i < G * D; i += kAttnWarps * 32) {
-    const int hh = i / D, d = i % D;
+  // per head, once: the warps' weights gam * 2^(m_w - m) / sum and 1 - gam
+  float *s_cf = s_o + kAttnWarps * 16 * D;                        // [G][kAttnWarps + 1]
+  if (tid < G) {
+    const int hh = tid;
     float mx = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kAttnWarps; ++w) mx = fmaxf(mx, s_ml[(w * 16 + hh) * 2]);
-    float num = 0.f, den = 0.f;
+    float f[kAttnWarps], den = 0.f;
 #pragma unroll
     for (int w = 0; w < kAttnWarps; ++w) {
       const float mw = s_ml[(w * 16 + hh) * 2];          // log2 units
-      if (mw == -INFINITY) continue;
-      const float f = exp2_approx(mw - mx);
-      num = fmaf(f, s_o[(w * 16 + hh) * D + d], num);
-      den = fmaf(f, s_ml[(w * 16 + hh) * 2 + 1], den);
+      f[w] = mw == -INFINITY ? 0.f : exp2_approx(mw - mx);
+      den = fmaf(f[w], s_ml[(w * 16 + hh) * 2 + 1], den);
     }
     const size_t row = ((size_t)b * p.T + tau) * p.Hq + g * G + hh;
     const float gam = 1.f / (1.f + expf(-p.gate[row]));
-    const float o_lin = p.olin[row * D + d];
-    reinterpret_cast<__nv_bfloat16 *>(p.out)[row * D + d] = __float2bfloat16_rn(gam * (num / den) + (1.f - gam) * o_lin);
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) s_cf[hh * (kAttnWarps + 1) + w] = gam * f[w] / den;
+    s_cf[hh * (kAttnWarps + 1) + kAttnWarps] = 1.f - gam;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kAttnWarps * 32) {
+    const int hh = i / D, d = i % D;
+    const float *cf = s_cf + hh * (kAttnWarps + 1);
+    const size_t row = ((size_t)b * p.T + tau) * p.Hq + g * G + hh;
+    float o = cf[kAttnWarps] * p.olin[row * D + d];
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) o = fmaf(cf[w], s_o[(w * 16 + hh) * D + d], o);
+    reinterpret_cast<__nv_bfloat16 *>(p.out)[row * D + d] = __float2bfloat16_rn(o);
   }
 }
 
