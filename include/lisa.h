@@ -196,9 +196,9 @@ LISA_API lisa_status lisa_indexer_topk(const lisa_layer *layer, const void *qidx
  * cluster, which bounds L_max to about 280K tokens (LISA_ERR_UNSUPPORTED
  * beyond); `workspace` is not used and may be NULL.  The wide form spreads
  * the key stream and the state of one (sequence, KV head) over 32 or 64 CTAs,
- * which publish their order keys, bounds and partial readouts of the linear
- * branch in the workspace; the last of their clusters to finish selects,
- * attends and writes the outputs.  It needs
+ * which publish their order keys and partial readouts of the linear branch
+ * in the workspace; the last of their clusters to finish selects, attends
+ * and writes the outputs.  It needs
  * lisa_workspace_bytes(layer, 1, LISA_OP_DECODE) bytes of workspace (0 for
  * fp32 storage, where the wide form does not apply), zero-filled before its
  * first use; every call leaves the workspace ready for the next one (its
