@@ -182,6 +182,14 @@ __global__ void __launch_bounds__(NT) rows_select_kernel(RowsParams p, int tau0,
   const uint32_t *gkeys = p.keys + ((size_t)bg * p.row_chunk + rr) * p.L_keys;
   const uint32_t *keys = gkeys;
   uint32_t *cand = s_dyn;
+  if (n > p.smem_keys_cap && threadIdx.x < 32) {
+    // a long row is read from global memory: all of it requested into L2 at
+    // once (32 KB bulk prefetches; rows start 16-byte aligned and hold L_keys,
+    // a multiple of 4, slots)
+    const int bytes = ((n * 4) + 15) & ~15;
+    for (int off = threadIdx.x * 32768; off < bytes; off += 32 * 32768)
+      bulk_prefetch_l2(reinterpret_cast<const char *>(gkeys) + off, (uint32_t)min(32768, bytes - off));
+  }
   if (n > p.M && n <= p.smem_keys_cap) {
     const int n4 = n & ~3;
     for (int i = threadIdx.x * 4; i < n4; i += NT * 4)
@@ -430,6 +438,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
   const __nv_bfloat16 *kc = reinterpret_cast<const __nv_bfloat16 *>(p.k_cache) + (size_t)bg * p.L_max * D;
   const __nv_bfloat16 *vc = reinterpret_cast<const __nv_bfloat16 *>(p.v_cache) + (size_t)bg * p.L_max * D;
 
+  // the epilogue's o_lin rows (written by the linear branch, G * D floats)
+  // requested into L2 now, so that its loads do not wait on DRAM at the end
+  {
+    const float *olr = p.olin + (((size_t)b * p.T + tau) * p.Hq + g * G) * D;
+    for (int i = tid * 32; i < G * D; i += kAttnWarps * 32 * 32) prefetch_l2(olr + i);
+  }
   // B fragments of Q^T (k = head dim, n = query head) for every 16-wide k-step
   uint32_t qb[NHT][D / 16][2];
   {
