@@ -149,20 +149,33 @@ __global__ void __launch_bounds__(256, 1)
     const int nc = (p.T + kLC - 1) / kLC;
     const float *S0 = p.state + ((size_t)b * p.Hq + h) * 128 * 128;
     const float *Pc = p.dS + ((size_t)bg * nc + c) * 128 * 128;
-    for (int item = tid; item < 128 * 16; item += 256) {
-      const int i = item >> 4, j0 = (item & 15) * 8;
-      float x[8];
-      const float4 a0 = *reinterpret_cast<const float4 *>(S0 + i * 128 + j0);
-      const float4 a1 = *reinterpret_cast<const float4 *>(S0 + i * 128 + j0 + 4);
-      const float4 b0 = *reinterpret_cast<const float4 *>(Pc + i * 128 + j0);
-      const float4 b1 = *reinterpret_cast<const float4 *>(Pc + i * 128 + j0 + 4);
-      x[0] = a0.x + b0.x; x[1] = a0.y + b0.y; x[2] = a0.z + b0.z; x[3] = a0.w + b0.w;
-      x[4] = a1.x + b1.x; x[5] = a1.y + b1.y; x[6] = a1.z + b1.z; x[7] = a1.w + b1.w;
-      uint4 hi, lo;
-      split8(x, hi, lo);
-      const uint32_t off = sw128_offset(i, j0, kHalf);
-      *reinterpret_cast<uint4 *>(shi + off) = hi;
-      *reinterpret_cast<uint4 *>(slo + off) = lo;
+    // 8 items of 8 columns per thread, in two batches of 4: the 16 loads of a
+    // batch are all in flight before any of them is used
+    constexpr int kBatch = 4;
+    for (int base = tid; base < 128 * 16; base += 256 * kBatch) {
+      float4 a[kBatch][2], bq[kBatch][2];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int item = base + k * 256, i = item >> 4, j0 = (item & 15) * 8;
+        a[k][0] = *reinterpret_cast<const float4 *>(S0 + i * 128 + j0);
+        a[k][1] = *reinterpret_cast<const float4 *>(S0 + i * 128 + j0 + 4);
+        bq[k][0] = *reinterpret_cast<const float4 *>(Pc + i * 128 + j0);
+        bq[k][1] = *reinterpret_cast<const float4 *>(Pc + i * 128 + j0 + 4);
+      }
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int item = base + k * 256, i = item >> 4, j0 = (item & 15) * 8;
+        float x[8];
+        x[0] = a[k][0].x + bq[k][0].x; x[1] = a[k][0].y + bq[k][0].y;
+        x[2] = a[k][0].z + bq[k][0].z; x[3] = a[k][0].w + bq[k][0].w;
+        x[4] = a[k][1].x + bq[k][1].x; x[5] = a[k][1].y + bq[k][1].y;
+        x[6] = a[k][1].z + bq[k][1].z; x[7] = a[k][1].w + bq[k][1].w;
+        uint4 hi, lo;
+        split8(x, hi, lo);
+        const uint32_t off = sw128_offset(i, j0, kHalf);
+        *reinterpret_cast<uint4 *>(shi + off) = hi;
+        *reinterpret_cast<uint4 *>(slo + off) = lo;
+      }
     }
   }
   fence_async_shared();
