@@ -556,6 +556,15 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
   }
 
   // ---------------------------------------------------------------- indexer scores
+  // Smallest and largest order key this thread writes (for the top-M's range
+  // histogram).  The cache row of position t may be stale (its key is
+  // replaced below from the argument row), so it is left out, and the new
+  // key goes in when it is written.
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  auto note_key = [&](uint32_t u) {
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  };
   for (int i = 0; i < nsub; ++i) {
     const int stage = i % NS;
     if (!mbar_wait_bounded(&bars[stage], (uint32_t)((i / NS) & 1)) && tid == 0)
@@ -586,8 +595,16 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
         if ((lane & 3) == 0) {
           const int r0 = tile * 16 + (lane >> 2);
-          if (r0 < nk) keys[s_lo - k0 + r0] = score_key(p0);
-          if (r0 + 8 < nk) keys[s_lo - k0 + r0 + 8] = score_key(p1);
+          if (r0 < nk) {
+            const uint32_t u = score_key(p0);
+            keys[s_lo - k0 + r0] = u;
+            if (s_lo + r0 != t) note_key(u);
+          }
+          if (r0 + 8 < nk) {
+            const uint32_t u = score_key(p1);
+            keys[s_lo - k0 + r0 + 8] = u;
+            if (s_lo + r0 + 8 != t) note_key(u);
+          }
         }
       }
     } else {
@@ -617,7 +634,9 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
 #pragma unroll
         for (int r = 0; r < kMaxR; ++r)
           if (r < R) score = fmaf(wsm[r], fmaxf(acc[r][0] + acc[r][1], 0.f), score);
-        keys[s_lo - k0 + kk] = score_key(score);
+        const uint32_t u = score_key(score);
+        keys[s_lo - k0 + kk] = u;
+        if (s_lo + kk != t) note_key(u);
       }
     }
     __syncthreads();   // every thread is done with this stage
@@ -633,7 +652,11 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
       dot = warp_sum(dot);
       score = fmaf(wsm[r], fmaxf(dot, 0.f), score);
     }
-    if (lane == 0) keys[t - k0] = score_key(score);
+    if (lane == 0) {
+      const uint32_t u = score_key(score);
+      keys[t - k0] = u;
+      note_key(u);
+    }
   }
 
   __syncthreads();
@@ -713,11 +736,15 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     //     least kl keys are >= theta_r); its send threshold is the lower edge
     //     of the bin above the one holding its SEG-th largest key (fewer than
     //     SEG keys are >= it), or 0 (every key) when it holds at most SEG.
-    uint32_t vmin = 0xFFFFFFFFu, vmax = 0u;
-    for (int j = tid; j < cnt; j += kDecThreads) {
-      const uint32_t u = keys[j];
-      vmin = min(vmin, u);
-      vmax = max(vmax, u);
+    uint32_t vmin = kmin, vmax = kmax;                  // from the scoring pass
+    if constexpr (WIDE) {                               // the reloaded keys of this CTA's range
+      vmin = 0xFFFFFFFFu;
+      vmax = 0u;
+      for (int j = tid; j < cnt; j += kDecThreads) {
+        const uint32_t u = keys[j];
+        vmin = min(vmin, u);
+        vmax = max(vmax, u);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -757,6 +784,16 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     } else {
       vmax = 0u;
     }
+    auto prefetch_kv = [&](int pos) {
+      const size_t row = ((size_t)bg * p.L_max + pos) * D;
+      const char *kr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.k_cache) + row);
+      const char *vr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.v_cache) + row);
+#pragma unroll
+      for (int c = 0; c < ROWB; c += 128) {
+        prefetch_l2(kr + c);
+        prefetch_l2(vr + c);
+      }
+    };
     // (b) keys >= tsend, in position order, into this CTA's message; warp w
     //     owns a contiguous run of keys
     {
@@ -799,8 +836,9 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     }
     __syncthreads();                                    // the message is complete
     // (c) the message to every other CTA of the cluster (its slot `rank`,
-    //     counted on its candidate mbarrier), then this CTA's likely selected
-    //     K and V rows into L2 while the others' messages arrive
+    //     counted on its candidate mbarrier), then the K and V rows of this
+    //     CTA's likely selected keys (>= theta, all in its message when the
+    //     exchange holds) into L2 while the others' messages arrive
     {
       constexpr int CH = XW / 4;                        // 16-byte chunks
       const uint32_t src = smem_u32(xo), xbar = smem_u32(mbx);
@@ -810,18 +848,11 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
         st_async_v4(mapa_u32(src + 16u * q, d), *reinterpret_cast<const uint4 *>(xo + 4 * q), mapa_u32(xbar, d));
       }
     }
-    auto prefetch_kv = [&](int pos) {
-      const size_t row = ((size_t)bg * p.L_max + pos) * D;
-      const char *kr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.k_cache) + row);
-      const char *vr = reinterpret_cast<const char *>(reinterpret_cast<const T *>(p.v_cache) + row);
-#pragma unroll
-      for (int c = 0; c < ROWB; c += 128) {
-        prefetch_l2(kr + c);
-        prefetch_l2(vr + c);
+    if (!(xo[3] & 0x80000000u))
+      for (int j = tid; j < (int)xo[3]; j += kDecThreads) {
+        const int pos = (int)xo[4 + SEG + j];
+        if (xo[4 + j] >= theta && pos != t) prefetch_kv(pos);
       }
-    };
-    for (int j = tid; j < cnt; j += kDecThreads)
-      if (keys[j] >= theta && k0 + j != t) prefetch_kv(k0 + j);
     if (!mbar_wait_cluster_bounded(mbx, 0u)) set_err(p.err_word, LISA_DEVERR_TIMEOUT);
     // (d) the bound lb = min_r theta_r (when the CTAs vouch for M keys
     //     together; else 0) and the largest key, from the headers.  The
@@ -845,9 +876,13 @@ __global__ void __launch_bounds__(kDecThreads, (NC <= 8 && sizeof(T) == 2) ? 2 :
     const bool exch_ok = __all_sync(0xffffffffu, (ct_r & 0x80000000u) == 0u && ts_r <= lb);
     local_list = exch_ok;
     if (exch_ok) {
-      // the rest of this CTA's candidates (lb <= key < theta) into L2 as well
-      for (int j = tid; j < cnt; j += kDecThreads)
-        if (keys[j] >= lb && keys[j] < theta && k0 + j != t) prefetch_kv(k0 + j);
+      // the rest of this CTA's candidates (lb <= key < theta) into L2 as well:
+      // they are all in its own message (every threshold is <= lb)
+      for (int j = tid; j < (int)xo[3]; j += kDecThreads) {
+        const uint32_t u = xo[4 + j];
+        const int pos = (int)xo[4 + SEG + j];
+        if (u >= lb && u < theta && pos != t) prefetch_kv(pos);
+      }
       // (e) the candidates, in position order: slot s = (warp * SLOTS + i) *
       //     32 + lane is entry s % SEG of message s / SEG; valid when that
       //     entry was sent and its key is >= lb
