@@ -392,15 +392,15 @@ __global__ void __launch_bounds__(256) prefill_attend_kernel(RowsParams p) {
 }
 
 // ------------------------------------------------------------ bf16 on warp MMAs
-// grid (T, B*Hkv); 4 warps.  Warp w owns selected rows [w*M/4, (w+1)*M/4) of
+// grid (T, B*Hkv); kAttnWarps warps.  Warp w owns a contiguous 1/kAttnWarps of
 // the (b, tau, g) list, in tiles of 16 rows staged by cp.async (two stages per
 // warp), flash-attention style with the selected rows as the M dimension of
 // the warp MMAs and the G query heads as the N dimension (NHT tiles of 8
 // heads): S^T = K Q^T, online softmax per head in registers, O^T += V^T P^T
 // with P^T moved from the accumulator layout into the B-operand layout by 8x8
-// transposes (movmatrix), P in bf16.  The 4 warps' (max, sum, O) are merged
+// transposes (movmatrix), P in bf16.  The warps' (max, sum, O) are merged
 // through shared memory, then the gate mixes in o_lin.
-constexpr int kAttnWarps = 4;
+constexpr int kAttnWarps = 1;   // warps per (b, t, g); each owns M / kAttnWarps selected rows
 
 
 template <int D>
@@ -594,8 +594,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32) prefill_attend_mma_kernel(Row
 
   // merge the warps: [warp][16 heads] max and sum, [warp][16][D] O
   __syncthreads();
-  float *s_ml = reinterpret_cast<float *>(s_att);                 // [4][16][2]
-  float *s_o = s_ml + kAttnWarps * 32;                            // [4][16][D]
+  float *s_ml = reinterpret_cast<float *>(s_att);                 // [kAttnWarps][16][2]
+  float *s_o = s_ml + kAttnWarps * 32;                            // [kAttnWarps][16][D]
 #pragma unroll
   for (int nh = 0; nh < NHT; ++nh) {
     const int h0 = nh * 8 + kq;
