@@ -48,7 +48,7 @@ WORKLOAD = "decode_1p5b_16k"
 # DRAM bytes (read + write) of one decode launch from an ncu capture of this
 # kernel on this workload, by CTA split (the ncu summary under profiles/);
 # None where no capture of the current kernel exists.
-DECODE_TRAFFIC = {4: 5396224, 8: None, 16: 5501696, 0: None, 32: None, 64: None}
+DECODE_TRAFFIC = {4: 5390336, 8: None, 16: 5497856, 0: None, 32: None, 64: None}
 # nominal HBM3e bandwidth of a B200 (about 8 TB/s), for the second fraction
 NOMINAL_HBM_GBS = 8000.0
 
