@@ -88,17 +88,9 @@ __device__ __forceinline__ void grid_dep_launch() {
 }
 
 // ---------------------------------------------------------------- cluster barrier, split
-// barrier.cluster in two halves: every thread of every CTA of the cluster
-// arrives (its earlier shared-memory accesses released), and a later wait
-// returns once all have arrived (acquire).  Work placed between the two
-// overlaps the barrier's latency.
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// The same with no memory ordering: only "every CTA got this far".
+// barrier.cluster in two halves with no memory ordering (only "every CTA of
+// the cluster got this far"): every thread arrives, and a later wait returns
+// once all have arrived.  Work placed between the two overlaps the barrier.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
@@ -293,18 +285,6 @@ __device__ __forceinline__ void set_err(int *err_word, int bits) {
   if (err_word) atomicOr(err_word, bits);
 }
 
-__device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
-  uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-__device__ __forceinline__ uint2 ld_nc_v2(const void *p) {
-  uint2 r;
-  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
 
 // 2^x by PTX ex2.approx (one special-function instruction, about 2 ulp);
 // e^x = 2^(x log2 e), so callers keep logits in log2 units.
