@@ -46,11 +46,13 @@
  *     the host saw; everything found on the device (a bad position, a bounded
  *     wait that ran out, a failed self-check) is reported through these bits,
  *     which the caller reads after synchronising.
- *   - Every wait inside a kernel on an asynchronous copy or on another warp's
- *     progress is bounded in time (LISA_WAIT_LIMIT_NS per wait, measured with
+ *   - Every mbarrier wait inside a kernel (on an asynchronous copy, on another
+ *     warp's progress, or on the messages of the other CTAs of a decode
+ *     cluster) is bounded in time (LISA_WAIT_LIMIT_NS per wait, measured with
  *     the GPU's global nanosecond timer); a wait that runs out sets
  *     LISA_DEVERR_TIMEOUT and the kernel carries on to its end without
- *     waiting again for that stage.
+ *     waiting again for that stage.  Cluster barriers have no bounded form:
+ *     every CTA of a cluster takes the same sequence of them.
  *   - Storage dtype (q, k, v, caches, out): bf16 or fp32, per lisa_layer.dtype.
  *     w, gate logits and the state are always fp32; indices are int32.
  *   - Supported shapes: d in {64, 128}; dI in {32, 64}; M a multiple of 32 in
