@@ -16,19 +16,25 @@
 //      thread per key on the CUDA cores.  Meanwhile the columns
 //      [r*d/NC, (r+1)*d/NC) of the linear state of the G query heads are
 //      loaded, updated (S += k^T v) and read out (o_lin = q S);
-//   2. exact top-M: every CTA takes the smallest of kl group maxima of its
-//      keys; if enough CTAs hold kl keys, the smallest of those values over
-//      the cluster is <= the M-th largest key, so only keys at or above it go
-//      to CTA 0 (each rank's in position order, in a segment of its own).
-//      CTA 0 finds the M-th key exactly with 1024-bin range histograms of the
-//      candidates and emits the ascending index list by an ordered
-//      compaction.  When a segment overflows, a cluster-wide radix select
-//      (histograms summed over distributed shared memory) runs instead;
+//   2. exact top-M in one round of distributed-shared-memory messages: each
+//      CTA bins its keys (1024 range bins over the 8 octaves below its
+//      largest key), takes its bound theta (the kl-th largest key's bin) and
+//      a send threshold (fewer than SEG keys above it), and sends every other
+//      CTA one fixed-size message: both values, its largest key and its keys
+//      above the threshold, in position order (st.async onto the receiver's
+//      mbarrier).  With lb = min theta, the messages hold every key >= lb iff
+//      every threshold is <= lb; then each CTA finds the M-th key exactly
+//      from the candidates (range histograms, a one-warp resolve) and emits
+//      the whole ascending index list itself.  Otherwise a cluster-wide
+//      radix select (histograms summed over distributed shared memory)
+//      builds the list in CTA 0;
 //   3. gather M/NC of the selected K/V rows, partial softmax for the G heads;
-//   4. every rank writes its partials of CTA r's columns into CTA r; after
-//      one barrier each CTA merges its column slice, applies the gate, stores.
-// Only cluster barriers synchronise; nothing leaves the cluster but the
-// outputs, the state and the appended cache row.
+//   4. every CTA sends each other CTA its partials of that CTA's columns
+//      (st.async onto a second mbarrier); each merges its column slice,
+//      applies the gate and stores.
+// The wide form (nw CTAs per (b, g)) streams and scores over nw CTAs and
+// hands the keys to the last cluster through a workspace.  Nothing else
+// leaves the cluster but the outputs, the state and the appended cache row.
 #include <cooperative_groups.h>
 #include <string.h>
 

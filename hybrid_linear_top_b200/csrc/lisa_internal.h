@@ -50,7 +50,7 @@ struct DecodeParams {
   void *out;
   int *idx_out;
   // launch geometry (filled by the launcher)
-  int split_req;                        // requested CTAs per (b, g): 0 (library's choice), 4, 8, 16
+  int split_req;                        // requested CTAs per (b, g): 0 (library's choice), 4, 8, 16, 32, 64
   int window;                           // 1: sliding-window variant (M = the window W; no indexer inputs)
   const int *sel_ext;                   // non-NULL: index lists given, [B, sel_groups, M] (no indexer inputs)
   int sel_groups;                       // selection groups of sel_ext: 1 (one set for every KV head) or Hkv
